@@ -1,0 +1,439 @@
+"""Benchmark: imatrix-weighted Q4_0 + Q8_K_128 quantization on B200.
+
+One step = one pass of the whole path over the Llama-2-7B-shaped layer set
+(32 layers x {q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008}, fp32
+weights from bf16 N(0, 0.02) with 0.1% t(3) outliers, per-tensor log-normal
+imatrix), for every tensor: weighted Q4_0 quantization, dequantization and the
+weighted-RMSE reduction; plus Q8_K_128 quantization of a 4096 x 7168 activation
+batch.  Inputs are synthetic and resident in HBM (25.9 GB of weights, far larger
+than the 126 MB L2, so no L2 flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under torchrun;
+every rank quantizes its own copy of the layer set (weak scaling, no collective
+on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Gelem/s quantized (imatrix Q4_0, Q8_K_128) on 1 B200; % of HBM/FP32 roofline"
+UNIT = "Gelem/s"
+WORKLOAD = "llama2-7b layer set x32 (q4_0 imatrix + dequant + wrmse) + q8_k128 4096x7168"
+
+# Algorithmic work per value ("Roofline"):
+#   Q4_0 weighted: 145 + 8*p binary32 lane operations per value, p = mean greedy passes;
+#   Q8_K_128: 4 + 140/128 bytes per value; dequant: 18/32 + 4; wrmse: 4 + 18/32 (+ qw from L2).
+Q4_0_OPS_BASE = 145.0
+Q4_0_OPS_PER_PASS = 8.0
+Q8_BYTES_PER_VALUE = 4.0 + 140.0 / 128.0
+DEQ_BYTES_PER_VALUE = 18.0 / 32.0 + 4.0
+RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
+B200_SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def mark(self):
+        """Start of the region whose samples count (the sampler is already running)."""
+        self.t0 = time.perf_counter()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        t1 = time.perf_counter()
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        mhz, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        t0 = getattr(self, "t0", 0.0)
+        for ts, ln in self.lines:
+            if ts < t0 or ts > t1 + 0.1:
+                continue
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _oracle_chunk(args):
+    """Worker: the oracle's whole path on one sample chunk (runs in a spawned process)."""
+    import oracle
+    from post_weight_quantization_rowwise_b200 import synth
+    kind, rows, cols, seed, bf16 = args
+    if kind == "q8":
+        a = synth.activations(rows, cols, seed=seed).numpy()
+        t0 = time.perf_counter()
+        oracle.quantize_q8_k128(a)
+        return a.size, time.perf_counter() - t0, 0, 0
+    x = synth.weight_matrix(rows, cols, seed=seed, bf16=bf16).numpy()
+    qw = synth.imatrix(cols, seed=seed + 1).numpy()
+    t0 = time.perf_counter()
+    blocks, _, passes = oracle.quantize_q4_0_w(x, qw, want_passes=True)
+    oracle.dequant_q4_0(blocks, rows, cols)
+    oracle.weighted_rmse(x, blocks, qw)
+    return x.size, time.perf_counter() - t0, int(passes.sum()), int(passes.size)
+
+
+def oracle_sample(target_seconds: float = 12.0, cores: int | None = None):
+    """Times the unchanged single-threaded oracle on a bounded sample of the workload,
+    one process per core: rows of every tensor shape of the layer set (same recipe,
+    in the layer set's proportions of values) and Q8_K_128 activation rows (in the
+    step's proportion).  The rate is the sum over processes of each process's own rate
+    (independent rows, so the copies do not interact).
+    Returns (Gelem/s, cores, sample description, mean greedy passes)."""
+    import multiprocessing as mp
+    from post_weight_quantization_rowwise_b200 import synth
+    cores = cores or os.cpu_count() or 1
+    layer = synth.LLAMA2_7B_TENSORS
+    layer_elems = sum(r * c for _, r, c in layer)
+    budget = 3.0e6 * target_seconds * cores          # values; ~3 M values/s per process
+    chunk = max(budget / (3 * cores), 4096 * 8)
+    jobs = []
+    for i, (name, r, c) in enumerate(layer):
+        rows = max(1, int(budget * (r * c) / layer_elems / c))
+        per = max(1, int(chunk // c))
+        for k, r0 in enumerate(range(0, rows, per)):
+            jobs.append(("q4", min(per, rows - r0), c, 9000 + 100 * i + k, True))
+    q8_rows = max(1, int(budget * 4096 * 7168 / (32 * layer_elems) / 7168))
+    jobs.append(("q8", q8_rows, 7168, 2, False))
+    ctx = mp.get_context("spawn")
+    t0 = time.perf_counter()
+    with ctx.Pool(cores) as pool:
+        res = pool.map(_oracle_chunk, jobs, chunksize=1)
+    wall = time.perf_counter() - t0
+    elems = sum(r[0] for r in res)
+    busy = sum(r[1] for r in res)
+    pass_sum = sum(r[2] for r in res)
+    pass_n = sum(r[3] for r in res)
+    value = elems / (busy / cores) / 1e9
+    sample = (f"{elems / 1e6:.1f} M values ({len(jobs) - 1} Q4_0 chunks over the 7 tensor shapes "
+              f"in layer-set proportion + {q8_rows} Q8_K_128 rows); {cores} processes, "
+              f"{busy:.1f} s CPU, {wall:.1f} s wall")
+    return value, cores, sample, pass_sum / max(pass_n, 1)
+
+
+# ----------------------------------------------------------------------------- the GPU step
+
+class Workload:
+    def __init__(self, dev, rank: int, layers: int = 32):
+        import torch
+        from post_weight_quantization_rowwise_b200 import synth
+        self.tensors = synth.llama2_7b_layer_set(layers)
+        self.x, self.qw, self.blocks = [], [], []
+        for t in self.tensors:
+            seed_off = 1_000_000 * rank
+            g = synth.Tensor2D(t.name, t.rows, t.cols, t.seed + seed_off, t.sigma, t.bf16,
+                               t.boost_frac)
+            self.x.append(g.weights(device=dev))
+            self.qw.append(g.qw(device=dev))
+            self.blocks.append(torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8,
+                                           device=dev))
+        maxn = max(t.numel for t in self.tensors)
+        self.y = torch.empty(maxn, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros(4, dtype=torch.float64, device=dev)
+        self.act = synth.activations(4096, 7168, seed=2 + 1_000_000 * rank, device=dev)
+        self.q8 = torch.empty(4096 * 56 * 140, dtype=torch.uint8, device=dev)
+        self.q4_elems = sum(t.numel for t in self.tensors)
+        self.q8_elems = self.act.numel()
+
+
+def run_step(iqq, w: Workload, stream, ev=None):
+    """Enqueues one step.  ev: optional list of 5 events bracketing the 4 phases."""
+    import torch
+    if ev is not None:
+        ev[0].record(stream)
+    for x, qw, b in zip(w.x, w.qw, w.blocks):
+        iqq.iqq_quantize_q4_0_w(x, qw, b, stream=stream)
+    if ev is not None:
+        ev[1].record(stream)
+    for t, b in zip(w.tensors, w.blocks):
+        iqq.iqq_dequant_q4_0(b, w.y[:t.numel].view(t.rows, t.cols), stream=stream)
+    if ev is not None:
+        ev[2].record(stream)
+    w.acc.zero_()
+    for x, qw, b in zip(w.x, w.qw, w.blocks):
+        iqq.iqq_weighted_rmse(x, b, qw, w.acc, stream=stream)
+    if ev is not None:
+        ev[3].record(stream)
+    iqq.iqq_quantize_q8_k128(w.act, w.q8, stream=stream)
+    if ev is not None:
+        ev[4].record(stream)
+    return 3 * len(w.tensors) + 1
+
+
+def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
+    """Same step through the public API from pinned host buffers: per tensor H2D of x,
+    the three kernels, D2H of the blocks; D2H of the accumulator at the end."""
+    import torch
+    n = 7 * layers
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    host_x = [pinned_copy(w.x[i]) for i in range(n)]
+    host_qw = [pinned_copy(w.qw[i]) for i in range(n)]
+    host_b = [torch.empty(w.blocks[i].numel(), dtype=torch.uint8, pin_memory=True) for i in range(n)]
+    host_act = pinned_copy(w.act)
+    host_q8 = torch.empty(w.q8.numel(), dtype=torch.uint8, pin_memory=True)
+    host_acc = torch.empty(4, dtype=torch.float64, pin_memory=True)
+    xd = torch.empty(max(t.numel for t in w.tensors[:n]), dtype=torch.float32, device=dev)
+    qd = torch.empty(max(t.cols for t in w.tensors[:n]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    h2d = sum(h.numel() * 4 for h in host_x) + sum(h.numel() * 4 for h in host_qw) + host_act.numel() * 4
+    d2h = sum(h.numel() for h in host_b) + host_q8.numel() + 32
+
+    def one():
+        w.acc.zero_()
+        for i in range(n):
+            t = w.tensors[i]
+            xv = xd[:t.numel].view(t.rows, t.cols)
+            xv.copy_(host_x[i], non_blocking=True)
+            qd[:t.cols].copy_(host_qw[i], non_blocking=True)
+            iqq.iqq_quantize_q4_0_w(xv, qd[:t.cols], w.blocks[i], stream=stream)
+            iqq.iqq_dequant_q4_0(w.blocks[i], w.y[:t.numel].view(t.rows, t.cols), stream=stream)
+            iqq.iqq_weighted_rmse(xv, w.blocks[i], qd[:t.cols], w.acc, stream=stream)
+            host_b[i].copy_(w.blocks[i], non_blocking=True)
+        w.act.copy_(host_act, non_blocking=True)
+        iqq.iqq_quantize_q8_k128(w.act, w.q8, stream=stream)
+        host_q8.copy_(w.q8, non_blocking=True)
+        host_acc.copy_(w.acc, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3 / steps
+    elems = sum(t.numel for t in w.tensors[:n]) + w.act.numel()
+    return {"value": elems / sec / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "layers": layers}
+
+
+def main_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import post_weight_quantization_rowwise_b200 as iqq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    # the oracle pool is spawned before this process touches the GPU
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(args.cpu_seconds)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    w = Workload(dev, rank, args.layers)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        run_step(iqq, w, stream)
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(1.0)  # nvidia-smi's first sample arrives after start-up
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark()
+    launches = 0
+    for s in range(args.steps):
+        launches += run_step(iqq, w, stream, ev[s])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    phase = [0.0] * 4
+    for s in range(args.steps):
+        for p in range(4):
+            phase[p] += ev[s][p].elapsed_time(ev[s][p + 1])
+    total_ms = ev[0][0].elapsed_time(ev[-1][4])
+    t = torch.tensor([total_ms] + phase, dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    total_ms, phase = float(t[0]), [float(v) for v in t[1:]]
+    acc = w.acc.cpu().tolist()
+
+    e2e = None
+    if rank == 0 and world == 1 and not args.no_e2e:
+        e2e = run_e2e(iqq, w, dev, max(1, min(args.steps, 3)), args.e2e_layers)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    K = args.steps
+    ms_step = total_ms / K
+    elems = (w.q4_elems + w.q8_elems) * world
+    value = elems / (ms_step / 1e3) / 1e9
+    pk = peaks()
+    p_mean = cpu[3] if cpu else 1.1
+    q4_ms = phase[0] / K
+    n_q4 = len(w.tensors)
+    ops_per_value = Q4_0_OPS_BASE + Q4_0_OPS_PER_PASS * p_mean
+    achieved = w.q4_elems * ops_per_value / (q4_ms / 1e3) / 1e12          # Tops/s
+    peak_ops = B200_SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
+    deq_gbs = w.q4_elems * DEQ_BYTES_PER_VALUE / (phase[1] / K / 1e3) / 1e9
+    rmse_gbs = w.q4_elems * RMSE_BYTES_PER_VALUE / (phase[2] / K / 1e3) / 1e9
+    q8_gbs = w.q8_elems * Q8_BYTES_PER_VALUE / (phase[3] / K / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; no model weights or calibration data)",
+        "config": {"workload": WORKLOAD, "layers": args.layers, "tensors": n_q4,
+                   "q4_0_values": w.q4_elems, "q8_k128_values": w.q8_elems,
+                   "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (replicas)"},
+        "roofline": {"bound": "alu", "kernel": "q4_0_w_kernel", "achieved": round(achieved, 3),
+                     "peak": round(peak_ops, 3), "unit": "Tops/s",
+                     "frac": round(achieved / peak_ops, 4), "traffic": None,
+                     "ops_per_value": round(ops_per_value, 2), "greedy_passes_mean": round(p_mean, 4),
+                     "avg_launch_ms": round(q4_ms / n_q4, 5),
+                     "peak_basis": f"{B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "
+                                   f"{pk['sm_max_mhz']:.0f} MHz ({pk['source']} max clock)"},
+        "kernels": {
+            "q4_0_w": {"ms": round(q4_ms, 4), "gelem_s": round(w.q4_elems / (q4_ms / 1e3) / 1e9, 3)},
+            "dequant_q4_0": {"ms": round(phase[1] / K, 4), "gb_s": round(deq_gbs, 1),
+                             "hbm_frac": round(deq_gbs / pk["hbm_gbs"], 4)},
+            "weighted_rmse": {"ms": round(phase[2] / K, 4), "gb_s": round(rmse_gbs, 1),
+                              "hbm_frac": round(rmse_gbs / pk["hbm_gbs"], 4),
+                              "wrmse": math.sqrt(acc[0] / acc[1]) if acc[1] else None},
+            "q8_k128": {"ms": round(phase[3] / K, 4), "gb_s": round(q8_gbs, 1),
+                        "hbm_frac": round(q8_gbs / pk["hbm_gbs"], 4),
+                        "gelem_s": round(w.q8_elems / (phase[3] / K / 1e3) / 1e9, 3)},
+        },
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if cpu:
+        out["cpu_baseline"] = {"value": round(cpu[0], 5), "unit": UNIT, "cores": cpu[1],
+                               "kind": "oracle", "sample": cpu[2]}
+    print(json.dumps(out), flush=True)
+
+
+def main_reference(args):
+    """The oracle (plain single-threaded C, one process per core) as the reference arm."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    vals, cores, sample, p = [], None, None, None
+    per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        v, cores, sample, p = oracle_sample(per_step)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    out = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+           "data": "synthetic (seeded; no model weights or calibration data)",
+           "config": {"workload": WORKLOAD, "layers": args.layers}, "impl": "reference",
+           "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--e2e-layers", type=int, default=32)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+/*
+ * iqq.h -- C ABI of the B200 (sm_100a) library for importance-matrix-weighted
+ * Q4_0 weight quantization, Q8_K_128 activation quantization, Q4_0
+ * dequantization and the round-trip weighted RMSE.
+ *
+ * Sources (page title, address, section):
+ *  [W]   "ik_llama.cpp 量化权重之谜：weight[j] = qw[j] * sqrtf(sigma2 +
+ *        xb[j]*xb[j])的由来与原理" (www.dpshk.com/news/4810665)
+ *  [Q8]  "ik_llama.cpp 量化精度修复实录：用 Q8_K_128 替代 Q8_1 根治
+ *        IQ1_S_R4 / IQ1_M_R4 的 fp16 溢出" (www.hnwysp.cn/news/39281)
+ *  [SVD] "量化方法论实证：为什么 LQER/L²QER 难以改进 ik_llama.cpp 的
+ *        k-quants 与 i-quants" (www.0539edu.com/news/4792009)
+ *
+ * Conventions shared by every entry point:
+ *  - Memory: every data pointer is DEVICE memory owned by the caller (for
+ *    example a torch CUDA tensor's data_ptr()).  The library never allocates,
+ *    frees or keeps a pointer after the call returns.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Work is enqueued asynchronously on it; the call never
+ *    synchronizes.  Results and flags are valid after the caller synchronizes
+ *    the stream.
+ *  - Errors: the return value reports host-side validation and launch
+ *    failures only.  Validation happens before any CUDA call, so a rejected
+ *    call enqueues nothing.  IQQ_ERR_CUDA means the launch itself failed;
+ *    iqq_last_cuda_error() returns the cudaError_t value.
+ *  - Data problems found on the device (NaN/Inf input, negative importance,
+ *    a scale beyond binary16) are ORed as IQQ_FLAG_* bits into the optional
+ *    caller-owned device word *d_flags (may be NULL).  Nothing on the device
+ *    traps, asserts or waits.
+ *  - Empty input (nrows == 0 or n_per_row == 0) is valid and enqueues
+ *    nothing; pointers may then be NULL.
+ *  - Layouts are row-major: element (r, j) of an [nrows, n_per_row] float
+ *    matrix is at index r*n_per_row + j, and block b of row r is the
+ *    (r*nb + b)-th block of the output, nb = n_per_row / block values.
+ */
+#ifndef IQQ_H
+#define IQQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    IQQ_OK = 0,
+    IQQ_ERR_NULL = 1,  /* a required pointer is NULL                              */
+    IQQ_ERR_SHAPE = 2, /* negative size, n_per_row not a multiple of the block,   */
+                       /* or a size whose byte count overflows int64              */
+    IQQ_ERR_ALIGN = 3, /* a pointer lacks the alignment its argument states       */
+    IQQ_ERR_CUDA = 4,  /* the kernel launch failed (see iqq_last_cuda_error)      */
+    IQQ_ERR_ARG = 5    /* an enumerated argument is out of range (weight_mode)    */
+} iqq_status;
+
+/* Device-side flag bits, ORed into *d_flags. */
+#define IQQ_FLAG_NONFINITE_INPUT 1u /* NaN or Inf in x (or in qw)                    */
+#define IQQ_FLAG_NEG_QW 2u          /* an importance qw < 0                          */
+#define IQQ_FLAG_SCALE_OVERFLOW 4u  /* a finite Q4_0 scale rounded to +-Inf in fp16 */
+
+/* Block formats. */
+#define IQQ_Q4_0_BLOCK_VALUES 32
+#define IQQ_Q4_0_BLOCK_BYTES 18
+#define IQQ_Q8_K128_BLOCK_VALUES 128
+#define IQQ_Q8_K128_BLOCK_BYTES 140
+
+/*
+ * iqq_quantize_q4_0_w -- imatrix-weighted Q4_0 quantization, [W] §一
+ * (quantize_row_q4_0_impl with make_qx_quants(QK4_0, 8, ...)).
+ *
+ * Per row r: sigma2 = sum_j x[r,j]^2 / n_per_row (binary64 sum, rounded to
+ * binary32).  Per 32-value block: weight[j] = qw[j]*sqrtf(sigma2 + x[j]^2)
+ * (weight_mode 0) or qw[j] (weight_mode 1); a weighted least-squares scale
+ * search over iscale = -(8 + 0.1k)/xmax, k = -9..9, codes clamp(rint(iscale*x),
+ * -8, 7), best sumlx^2/suml2 (ties to the lowest k); at most 5 greedy passes
+ * that move one code by +-1 in the direction of g = d*w*(x - d*l) when the
+ * weighted error drops; d = sumlx/suml2 rounded to binary16.
+ *
+ *  x          [nrows, n_per_row] float32, 16-byte aligned.
+ *  qw         imatrix rows, float32, 16-byte aligned, or NULL (qw = 1).  Row r
+ *             uses qw + (rows_per_qw > 0 ? r / rows_per_qw : 0) * n_per_row.
+ *  out        nrows * n_per_row / 32 blocks of 18 bytes, 2-byte aligned:
+ *             bytes 0-1 binary16 d (little endian), byte 2+i holds
+ *             (l[i]+8) | (l[i+16]+8) << 4 for i = 0..15.
+ *  nrows, n_per_row   n_per_row % 32 == 0, both >= 0.
+ *  rows_per_qw        >= 0; 0 = one imatrix row shared by all rows.
+ *  weight_mode        0 = qw*sqrt(sigma2 + x^2), 1 = qw.
+ *  d_flags    optional device uint32 (4-byte aligned) receiving IQQ_FLAG_*.
+ *  stream     cudaStream_t.
+ *
+ * Invalid input is flagged, not trapped: a row whose x holds NaN/Inf, or a block
+ * whose qw holds NaN/Inf or a negative value, gets unspecified bytes; all other
+ * rows and blocks are exact.
+ */
+iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64_t nrows,
+                               int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                               uint32_t* d_flags, void* stream);
+
+/*
+ * iqq_quantize_q8_k128 -- Q8_K_128 activation quantization, [Q8] 修复方案:
+ * 128-value blocks with a binary32 scale, int8 codes and one int16 sum of the
+ * codes per 32 values that is not multiplied by d, so no fp16 quantity can
+ * overflow.  amax = max|x|, d = amax/127, id = amax > 0 ? 127/amax : 0,
+ * q = clamp(rint(x*id), -127, 127) (a NaN product gives 0),
+ * bsums[i] = sum of q over values 32i..32i+31.
+ *
+ *  x          [nrows, n_per_row] float32, 16-byte aligned.
+ *  out        nrows * n_per_row / 128 blocks of 140 bytes, 4-byte aligned:
+ *             float d | int8 qs[128] | int16 bsums[4], little endian.
+ *  n_per_row  must be a multiple of 128 (the ne00 % 128 == 0 rule of [Q8]).
+ *  d_flags    optional; receives IQQ_FLAG_NONFINITE_INPUT.
+ */
+iqq_status iqq_quantize_q8_k128(const float* x, void* out, int64_t nrows, int64_t n_per_row,
+                                uint32_t* d_flags, void* stream);
+
+/*
+ * iqq_dequant_q4_0 -- y[r, 32b + i] = fp16(d) * (nibble_i - 8) for the Q4_0
+ * blocks written by iqq_quantize_q4_0_w (the inverse map of [W] §一's
+ * packing; the product is exact in binary32).
+ *
+ *  blocks     nrows * n_per_row / 32 blocks of 18 bytes, 2-byte aligned.
+ *  y          [nrows, n_per_row] float32 output, 16-byte aligned.
+ */
+iqq_status iqq_dequant_q4_0(const void* blocks, float* y, int64_t nrows, int64_t n_per_row,
+                            void* stream);
+
+/*
+ * iqq_weighted_rmse -- round-trip error of Q4_0 blocks against the source,
+ * weighted by the imatrix ([SVD] §3.2 rmse and maxerr; the weights are qw
+ * alone, not the quantizer weights).  With e = x - dequant(blocks) rounded to
+ * binary32, ADDS to the caller's binary64 accumulator
+ *     d_acc[0] += sum qw*e^2,  d_acc[1] += sum qw,  d_acc[2] += sum e^2,
+ *     d_acc[3]  = max(d_acc[3], max |e|).
+ * The caller zeroes d_acc once and may accumulate over several tensors:
+ * wrmse = sqrt(d_acc[0]/d_acc[1]), rmse = sqrt(d_acc[2]/count).  The sums use
+ * binary64 atomics, so their rounding order is not fixed (relative
+ * differences of order 1e-15 between runs).
+ *
+ *  x          [nrows, n_per_row] float32, 16-byte aligned.
+ *  blocks     Q4_0 blocks of x, 2-byte aligned.
+ *  qw         imatrix rows as in iqq_quantize_q4_0_w (NULL = 1), 16-byte aligned.
+ *  d_acc      device double[4], 8-byte aligned.
+ */
+iqq_status iqq_weighted_rmse(const float* x, const void* blocks, const float* qw, int64_t nrows,
+                             int64_t n_per_row, int64_t rows_per_qw, double* d_acc,
+                             void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* iqq_status_string(iqq_status status);
+
+/* The cudaError_t of the most recent IQQ_ERR_CUDA on this host thread (0 if none). */
+int iqq_last_cuda_error(void);
+
+/* Library build string. */
+const char* iqq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IQQ_H */

@@ -1,0 +1,230 @@
+"""imatrix-weighted Q4_0 and Q8_K_128 quantization on B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/iqq.h`` (``libiqq.so`` in this
+package).  The functions have the ABI's names; they only check and marshal
+arguments (torch CUDA tensors -> device pointers, sizes and the current CUDA
+stream).  Every step of the computation runs in the library's CUDA kernels:
+there is no CPU or PyTorch fallback, and importing this package raises if the
+library is missing or fails to load.
+
+Block formats (little endian):
+  Q4_0      18 bytes per 32 values: binary16 d | qs[16], qs[i] = (l[i]+8) | (l[i+16]+8) << 4
+  Q8_K_128  140 bytes per 128 values: float d | int8 qs[128] | int16 bsums[4]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libiqq.so")
+
+Q4_0_BLOCK_VALUES = 32
+Q4_0_BLOCK_BYTES = 18
+Q8_K128_BLOCK_VALUES = 128
+Q8_K128_BLOCK_BYTES = 140
+
+FLAG_NONFINITE_INPUT = 1
+FLAG_NEG_QW = 2
+FLAG_SCALE_OVERFLOW = 4
+
+STATUS = {0: "IQQ_OK", 1: "IQQ_ERR_NULL", 2: "IQQ_ERR_SHAPE", 3: "IQQ_ERR_ALIGN",
+          4: "IQQ_ERR_CUDA", 5: "IQQ_ERR_ARG"}
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m post_weight_quantization_rowwise_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    sigs = {
+        "iqq_quantize_q4_0_w": [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
+        "iqq_quantize_q8_k128": [_vp, _vp, _i64, _i64, _vp, _vp],
+        "iqq_dequant_q4_0": [_vp, _vp, _i64, _i64, _vp],
+        "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+    }
+    for name, args in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.iqq_status_string.argtypes = [ctypes.c_int]
+    lib.iqq_status_string.restype = ctypes.c_char_p
+    lib.iqq_last_cuda_error.argtypes = []
+    lib.iqq_last_cuda_error.restype = ctypes.c_int
+    lib.iqq_version.argtypes = []
+    lib.iqq_version.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+class IQQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = _lib.iqq_status_string(status).decode()
+        extra = ""
+        if status == 4:
+            extra = f" (cudaError {_lib.iqq_last_cuda_error()})"
+        super().__init__(f"{fn}: {STATUS.get(status, status)}: {msg}{extra}")
+        self.status = status
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise IQQError(fn, status)
+
+
+def version() -> str:
+    return _lib.iqq_version().decode()
+
+
+def status_string(status: int) -> str:
+    return _lib.iqq_status_string(status).decode()
+
+
+# ----------------------------------------------------------------------------
+# tensor marshalling (torch is used for memory and streams only)
+# ----------------------------------------------------------------------------
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None):
+    import torch
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _shape2(x):
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [nrows, n_per_row]")
+    return int(x.shape[0]), int(x.shape[1])
+
+
+def q4_0_nbytes(nrows: int, n_per_row: int) -> int:
+    return nrows * (n_per_row // Q4_0_BLOCK_VALUES) * Q4_0_BLOCK_BYTES
+
+
+def q8_k128_nbytes(nrows: int, n_per_row: int) -> int:
+    return nrows * (n_per_row // Q8_K128_BLOCK_VALUES) * Q8_K128_BLOCK_BYTES
+
+
+# ----------------------------------------------------------------------------
+# the four entry points
+# ----------------------------------------------------------------------------
+
+def iqq_quantize_q4_0_w(x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,
+                        stream=None):
+    """Q4_0 blocks of x [nrows, n_per_row] float32 into out (uint8, q4_0_nbytes)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if out.numel() < q4_0_nbytes(nrows, n):
+        raise ValueError("out is too small")
+    _check("iqq_quantize_q4_0_w",
+           _lib.iqq_quantize_q4_0_w(_ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw,
+                                    weight_mode, _ptr(flags), _stream(stream)))
+    return out
+
+
+def iqq_quantize_q8_k128(x, out, flags=None, stream=None):
+    """Q8_K_128 blocks of x [nrows, n_per_row] float32 into out (uint8, q8_k128_nbytes)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if out.numel() < q8_k128_nbytes(nrows, n):
+        raise ValueError("out is too small")
+    _check("iqq_quantize_q8_k128",
+           _lib.iqq_quantize_q8_k128(_ptr(x), _ptr(out), nrows, n, _ptr(flags), _stream(stream)))
+    return out
+
+
+def iqq_dequant_q4_0(blocks, y, stream=None):
+    """y [nrows, n_per_row] float32 from the Q4_0 blocks."""
+    import torch
+    _need_cuda("blocks", blocks, torch.uint8)
+    _need_cuda("y", y, torch.float32)
+    nrows, n = _shape2(y)
+    if blocks.numel() < q4_0_nbytes(nrows, n):
+        raise ValueError("blocks is too small")
+    _check("iqq_dequant_q4_0", _lib.iqq_dequant_q4_0(_ptr(blocks), _ptr(y), nrows, n, _stream(stream)))
+    return y
+
+
+def iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
+    """Adds {sum qw e^2, sum qw, sum e^2} to acc[0:3] and maxes acc[3] with max|e| (float64, CUDA)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("blocks", blocks, torch.uint8)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("acc", acc, torch.float64)
+    nrows, n = _shape2(x)
+    if blocks.numel() < q4_0_nbytes(nrows, n) or acc.numel() < 4:
+        raise ValueError("blocks or acc is too small")
+    _check("iqq_weighted_rmse",
+           _lib.iqq_weighted_rmse(_ptr(x), _ptr(blocks), _ptr(qw), nrows, n, rows_per_qw, _ptr(acc),
+                                  _stream(stream)))
+    return acc
+
+
+# ----------------------------------------------------------------------------
+# conveniences
+# ----------------------------------------------------------------------------
+
+def quantize_q4_0_w(x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0, flags=None, stream=None):
+    """Allocates and returns the Q4_0 blocks of x as a uint8 tensor [nrows, nb*18]."""
+    import torch
+    nrows, n = _shape2(x)
+    out = torch.empty((nrows, (n // Q4_0_BLOCK_VALUES) * Q4_0_BLOCK_BYTES), dtype=torch.uint8,
+                      device=x.device)
+    return iqq_quantize_q4_0_w(x, qw, out, rows_per_qw, weight_mode, flags, stream)
+
+
+def quantize_q8_k128(x, flags=None, stream=None):
+    import torch
+    nrows, n = _shape2(x)
+    out = torch.empty((nrows, (n // Q8_K128_BLOCK_VALUES) * Q8_K128_BLOCK_BYTES), dtype=torch.uint8,
+                      device=x.device)
+    return iqq_quantize_q8_k128(x, out, flags, stream)
+
+
+def dequant_q4_0(blocks, nrows: int, n_per_row: int, stream=None):
+    import torch
+    y = torch.empty((nrows, n_per_row), dtype=torch.float32, device=blocks.device)
+    return iqq_dequant_q4_0(blocks, y, stream)
+
+
+def weighted_rmse(x, blocks, qw=None, rows_per_qw: int = 0, stream=None):
+    """Returns the float64 accumulator [sum qw e^2, sum qw, sum e^2, max|e|] as a CUDA tensor."""
+    import torch
+    acc = torch.zeros(4, dtype=torch.float64, device=x.device)
+    return iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw, stream)
+
+
+__all__ = [n for n in dir() if n.startswith(("iqq_", "quantize", "dequant", "weighted", "Q", "FLAG",
+                                             "q4", "q8", "version", "status", "IQQError", "LIB"))]

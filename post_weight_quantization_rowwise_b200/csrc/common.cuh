@@ -1,0 +1,51 @@
+// common.cuh -- helpers shared by the library's CUDA translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "iqq.h"
+
+namespace iqq {
+
+// The cudaError_t of the last failed launch on this host thread.
+void set_last_cuda_error(cudaError_t e);
+
+// Maps the launch result to a status, remembering a failure.
+inline iqq_status launch_status()
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_last_cuda_error(e);
+        return IQQ_ERR_CUDA;
+    }
+    return IQQ_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// nrows * n_per_row * bytes_per_value fits in int64.
+inline bool size_ok(int64_t nrows, int64_t n_per_row, int64_t bytes_per_value)
+{
+    if (nrows < 0 || n_per_row < 0) return false;
+    if (nrows == 0 || n_per_row == 0) return true;
+    return nrows <= INT64_MAX / n_per_row / bytes_per_value;
+}
+
+// Streaming 16-byte load that bypasses L1 allocation (data read once).
+__device__ __forceinline__ float4 ld_stream_f4(const float4* p)
+{
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Flags word update: only lanes with a nonzero bit set touch memory.
+__device__ __forceinline__ void raise_flags(uint32_t* flags, uint32_t bits)
+{
+    if (flags != nullptr && bits != 0u) atomicOr(flags, bits);
+}
+
+}  // namespace iqq

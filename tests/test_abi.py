@@ -1,0 +1,81 @@
+"""The C-ABI library loads without a GPU, exports every function iqq.h declares, and
+rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "iqq.h"), encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(iqq_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import post_weight_quantization_rowwise_b200 as m
+    return m._lib
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("iqq_quantize_q4_0_w", "iqq_quantize_q8_k128", "iqq_dequant_q4_0",
+              "iqq_weighted_rmse", "iqq_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_exported_symbols_are_c_linkage():
+    import post_weight_quantization_rowwise_b200 as m
+    raw = ctypes.CDLL(m.LIB_PATH)
+    for n in _declared_functions():
+        ctypes.cast(getattr(raw, n), ctypes.c_void_p)  # resolvable unmangled
+
+
+def test_host_validation_without_gpu(lib):
+    V = ctypes.c_void_p
+    # shape: n_per_row not a multiple of 32 / 128, negative sizes
+    assert lib.iqq_quantize_q4_0_w(None, None, None, 4, 33, 0, 0, None, None) == 2
+    assert lib.iqq_quantize_q4_0_w(None, None, None, -1, 32, 0, 0, None, None) == 2
+    assert lib.iqq_quantize_q8_k128(None, None, 2, 96, None, None) == 2
+    assert lib.iqq_dequant_q4_0(None, None, 2, 48, None) == 2
+    assert lib.iqq_weighted_rmse(None, None, None, 2, 32, -1, None, None) == 2
+    # overflowing byte counts
+    assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 1 << 40, 1 << 30, 0, 0, None, None) == 2
+    # empty input is a no-op even with NULL pointers
+    assert lib.iqq_quantize_q4_0_w(None, None, None, 0, 64, 0, 0, None, None) == 0
+    assert lib.iqq_quantize_q8_k128(None, None, 5, 0, None, None) == 0
+    # NULL pointers
+    assert lib.iqq_quantize_q4_0_w(None, None, None, 4, 32, 0, 0, None, None) == 1
+    assert lib.iqq_weighted_rmse(V(16), V(16), None, 2, 32, 0, None, None) == 1
+    # alignment
+    assert lib.iqq_quantize_q4_0_w(V(8), None, V(16), 4, 32, 0, 0, None, None) == 3
+    assert lib.iqq_quantize_q4_0_w(V(16), V(20), V(16), 4, 32, 0, 0, None, None) == 3
+    assert lib.iqq_quantize_q4_0_w(V(16), None, V(17), 4, 32, 0, 0, None, None) == 3
+    assert lib.iqq_quantize_q8_k128(V(16), V(18), 1, 128, None, None) == 3
+    assert lib.iqq_dequant_q4_0(V(16), V(8), 1, 32, None) == 3
+    assert lib.iqq_weighted_rmse(V(16), V(16), None, 1, 32, 0, V(4), None) == 3
+    # enumerated argument
+    assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 4, 32, 0, 2, None, None) == 5
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.iqq_status_string(s)
+    assert lib.iqq_last_cuda_error() == 0
+
+
+def test_python_binding_requires_cuda_tensors():
+    import torch
+    import post_weight_quantization_rowwise_b200 as m
+    with pytest.raises(ValueError):
+        m.quantize_q4_0_w(torch.zeros(2, 64))
