@@ -15,26 +15,34 @@
 //   final sums recomputed, d = sumlx/suml2 -> binary16 (RNE);
 //   block = d16 (LE) | qs[i] = (l[i]+8) | (l[i+16]+8) << 4.
 //
-// This is ALU bound (about 150 binary32 operations per value against
-// 4.6 bytes of HBM traffic), so the design is about instruction count:
-//  - one thread owns one 32-value block with all of its state in registers,
-//    so every sum is a private sequential fmaf chain in exactly the order the
-//    definition fixes (no shuffles, no reordering: bit-exact by construction);
+// The work is ALU bound (about 150 binary32 operations per value against
+// 4.6 bytes of HBM traffic), so the design is about instruction count and
+// issue efficiency:
+//  - one thread owns one 32-value block, so every sum is a private sequential
+//    fmaf chain in exactly the order the definition fixes (no shuffles, no
+//    reordering: bit-exact by construction);
 //  - the candidate sweep runs on |x| with the sign folded out: for candidate k
 //    the code magnitude is m = min(rint(a_k*|x_j|), B_j) with a_k = c_k/|xmax|
-//    and B_j = 8 when x_j has the sign of xmax (code <= 0, clamp at -8) and 7
-//    otherwise.  Every term w*x*l then has the sign of -xmax, so
-//    |sumlx| = sum fmaf(|wx_j|, m_j, .) bit for bit (round-to-nearest is
+//    and B_j = 8 when x_j has the sign of xmax (code <= 0, clamped at -8) and
+//    7 otherwise.  With w >= 0 every term w*x*l then has the sign of -xmax, so
+//    |sumlx| = sum fmaf(|wx_j|, m_j, .) bit for bit (round to nearest is
 //    sign-symmetric) and the score needs only that magnitude;
-//  - rint of 0 <= v < 2^22 is (v + 1.5*2^23) - 1.5*2^23, two full-rate adds,
-//    and the clamp is a single min against M + B_j;
+//  - rint of 0 <= v < 2^22 is either cvt.rni (one conversion-pipe op) or
+//    (v + 1.5*2^23) - 1.5*2^23 (two FMA-pipe adds); the sweep mixes the two
+//    to balance the pipes, and the clamp is one min against B_j;
+//  - greedy pass 1 runs per thread (sequential, as defined); the few blocks
+//    whose first pass moved a code finish passes 2..5 warp-cooperatively;
 //  - sigma2 is a binary64 CTA reduction over the row (exact squares), the one
 //    place where the summation order differs from the sequential definition.
 //
 // CTA = 128 threads = 128 consecutive blocks of one row ("chunk"); each CTA
 // reduces sigma2 over its whole row (the row is read from HBM once and from L2
-// by the row's other chunks).  Built with -fmad=false: no contraction except
-// the explicit __fmaf_rn calls.
+// by the row's other chunks).  Per warp, shared memory holds the weights w of
+// its 32 blocks and a scratch area used first by the sweep (|wx| and the clamp
+// bounds in both rounding domains) and then by the later steps (x and the
+// codes), whose per-value loops then need no registers per value and stay
+// rolled (small code, fewer registers).  Built with -fmad=false: no
+// contraction except the explicit __fmaf_rn calls.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -43,8 +51,37 @@ namespace {
 
 constexpr int QK = IQQ_Q4_0_BLOCK_VALUES;
 constexpr int kThreads = 128;
+constexpr int kWarps = kThreads / 32;
 constexpr int kCand = 19;
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr unsigned kFull = 0xffffffffu;
+
+// Per-warp shared memory (floats).  Rows of 36 keep LDS.128/STS.128 16-byte
+// aligned and conflict-free (8 lanes per phase hit 8 distinct 4-bank groups);
+// rows of 33 keep scalar column accesses conflict-free.
+constexpr int kRow4 = QK + 4;
+constexpr int kRow1 = QK + 1;
+#ifndef IQQ_SWEEP_CPI
+#define IQQ_SWEEP_CPI 2  // candidates per sweep iteration
+#endif
+#ifndef IQQ_SWEEP_CVT_MASK
+#define IQQ_SWEEP_CVT_MASK 0  // bit c set: candidate c of a group rounds with cvt.rni
+#endif
+constexpr int kCvtAll = (1 << IQQ_SWEEP_CPI) - 1;
+constexpr bool kUseCvt = (IQQ_SWEEP_CVT_MASK & kCvtAll) != 0;     // some candidates round by cvt.rni
+constexpr bool kUseAdd = (IQQ_SWEEP_CVT_MASK & kCvtAll) != kCvtAll;  // some by the magic adds
+constexpr int kW = 0;                    // w[32][36]
+constexpr int kScratch = 32 * kRow4;     // sweep: |wx|, then M + B and/or B, each [32][36];
+                                         // later: x[32][33], l[32][33]
+constexpr int kAwx = kScratch;
+constexpr int kUbm = kAwx + 32 * kRow4;
+constexpr int kUb = kUbm + (kUseAdd ? 32 * kRow4 : 0);
+constexpr int kWarpFloats = kUb + (kUseCvt ? 32 * kRow4 : 0);
+static_assert(kScratch + 2 * 32 * kRow1 <= kWarpFloats, "staging fits in the sweep area");
+
+#ifndef IQQ_Q4_MIN_CTAS
+#define IQQ_Q4_MIN_CTAS 4  // resident CTAs per SM the register budget is sized for
+#endif
 
 // c_k = (float)(80 + k) / 10 for k = -9..9, each the IEEE quotient.
 __constant__ float c_cand[kCand] = {
@@ -61,29 +98,16 @@ __device__ __forceinline__ float clamp_code(float r) { return fminf(fmaxf(r, -8.
 __device__ __forceinline__ double block_reduce_sum(double v, double* s_red)
 {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) s_red[warp] = v;
     __syncthreads();
     double t = 0.0;
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) t += s_red[w];
+    for (int w = 0; w < kWarps; ++w) t += s_red[w];
     __syncthreads();
     return t;
 }
-
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kRow = QK + 1;                 // padded smem row: conflict-free both ways
-constexpr int kWarpSmemFloats = 3 * 32 * kRow;  // x, w, l of the warp's 32 blocks
-
-// One candidate's sums over the block in the folded form: |sumlx| and suml2.
-#define IQQ_SWEEP_TERM(a, s, t, j)                                                  \
-    {                                                                               \
-        const float v_ = __fmul_rn(a, fabsf(xv[j]));                                \
-        const float m_ = __fsub_rn(fminf(__fadd_rn(v_, kMagic), ub[j]), kMagic);    \
-        s = __fmaf_rn(awx[j], m_, s);                                               \
-        t = __fmaf_rn(w[j], __fmul_rn(m_, m_), t);                                  \
-    }
 
 // Running arg-max of sumlx^2/suml2 over the candidates, strictly greater wins.
 __device__ __forceinline__ void keep_best(float s, float t, int k, float& best, int& kbest)
@@ -95,57 +119,84 @@ __device__ __forceinline__ void keep_best(float s, float t, int k, float& best, 
     }
 }
 
-// Candidate sweep of one block: returns the winning k index (0..18) and its score.
-__device__ __forceinline__ void sweep_block(const float (&xv)[QK], const float (&w)[QK],
-                                            const float (&awx)[QK], const float (&ub)[QK],
-                                            float amax, float& best, int& kbest)
+// N candidates k0..k0+N-1 over the block.  Per value and candidate: v = a_k*|x|,
+// the code magnitude m = min(rint(v), B) -- rint either by cvt.rni, or as
+// min(v + M, M + B) - M -- then the two sequential sums |sumlx| += |wx|*m and
+// suml2 += w*m*m.  |wx|, B, M + B and w stream from this thread's rows of the
+// warp's shared memory (LDS.128).
+template <int N>
+__device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const float* __restrict__ my_w,
+                                            const float* __restrict__ my_awx,
+                                            const float* __restrict__ my_ubm,
+                                            const float* __restrict__ my_ub, float amax,
+                                            float& best, int& kbest)
 {
-    best = -INFINITY;
-    kbest = 0;
-#pragma unroll 1
-    for (int k = 0; k + 1 < kCand; k += 2) {
-        const float a0 = __fdiv_rn(c_cand[k], amax);      // |iscale_k|
-        const float a1 = __fdiv_rn(c_cand[k + 1], amax);
-        float s0 = 0.0f, t0 = 0.0f, s1 = 0.0f, t1 = 0.0f;
+    float a[N], s[N], t[N];
 #pragma unroll
-        for (int j = 0; j < QK; ++j) {
-            IQQ_SWEEP_TERM(a0, s0, t0, j)
-            IQQ_SWEEP_TERM(a1, s1, t1, j)
+    for (int c = 0; c < N; ++c) {
+        a[c] = __fdiv_rn(c_cand[k0 + c], amax);  // |iscale_k|
+        s[c] = 0.0f;
+        t[c] = 0.0f;
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < QK; j4 += 4) {
+        const float4 aw = *reinterpret_cast<const float4*>(my_awx + j4);
+        const float4 ww = *reinterpret_cast<const float4*>(my_w + j4);
+        float4 um = make_float4(0.f, 0.f, 0.f, 0.f), ub = um;
+        if ((IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) != ((1 << N) - 1)) um = *reinterpret_cast<const float4*>(my_ubm + j4);
+        if ((IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) != 0) ub = *reinterpret_cast<const float4*>(my_ub + j4);
+        static_assert(kUseAdd || (IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) == ((1 << N) - 1), "layout");
+        static_assert(kUseCvt || (IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) == 0, "layout");
+        const float awv[4] = {aw.x, aw.y, aw.z, aw.w};
+        const float umv[4] = {um.x, um.y, um.z, um.w};
+        const float ubv[4] = {ub.x, ub.y, ub.z, ub.w};
+        const float wv[4] = {ww.x, ww.y, ww.z, ww.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int c = 0; c < N; ++c) {
+                const float v = __fmul_rn(a[c], fabsf(xv[j4 + q]));
+                const float m = ((IQQ_SWEEP_CVT_MASK >> c) & 1)
+                                    ? fminf(rintf(v), ubv[q])
+                                    : __fsub_rn(fminf(__fadd_rn(v, kMagic), umv[q]), kMagic);
+                s[c] = __fmaf_rn(awv[q], m, s[c]);
+                t[c] = __fmaf_rn(wv[q], __fmul_rn(m, m), t[c]);
+            }
         }
-        keep_best(s0, t0, k, best, kbest);
-        keep_best(s1, t1, k + 1, best, kbest);
+#ifndef IQQ_SWEEP_NO_FENCE
+        // compiler-only fence: keeps each group's shared-memory loads beside its
+        // arithmetic instead of hoisting all of them (which costs registers)
+        asm volatile("" ::: "memory");
+#endif
     }
-    {
-        const float a0 = __fdiv_rn(c_cand[kCand - 1], amax);
-        float s0 = 0.0f, t0 = 0.0f;
 #pragma unroll
-        for (int j = 0; j < QK; ++j) IQQ_SWEEP_TERM(a0, s0, t0, j)
-        keep_best(s0, t0, kCand - 1, best, kbest);
-    }
+    for (int c = 0; c < N; ++c) keep_best(s[c], t[c], k0 + c, best, kbest);
 }
 
-// Greedy refinement of the warp's 32 blocks, one block at a time, lane j holding
-// element j.  All trial moves of a pass that precede the next accepted move see
-// the same (sumlx, suml2, score), so they are evaluated together; the lowest
-// accepting lane is the move the sequential pass accepts first.  The state then
-// advances and the scan resumes after that element, so the sequence of accepted
-// moves and every rounding is that of the sequential Gauss-Seidel passes.
-__device__ __forceinline__ void greedy_warp(float* sx, float* sw, float* sl, float sumlx,
-                                            float suml2, float score, bool active)
+// Greedy passes 2..5 for the warp's blocks whose first pass changed a code (bit
+// set in `pending`), one block at a time, lane j holding element j.  All trial
+// moves of a pass that precede the next accepted move see the same (sumlx,
+// suml2, score), so they are evaluated together; the lowest accepting lane is the
+// move the sequential pass accepts first.  The state then advances and the scan
+// resumes after that element, so the sequence of accepted moves and every
+// rounding is that of the sequential Gauss-Seidel passes.
+__device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, float* sL, unsigned pending,
+                                            float sumlx, float suml2, float score)
 {
     const int lane = threadIdx.x & 31;
 #pragma unroll 1
-    for (int bb = 0; bb < 32; ++bb) {
-        if (!__shfl_sync(kFull, static_cast<int>(active), bb)) continue;
+    while (pending != 0u) {
+        const int bb = __ffs(pending) - 1;
+        pending &= pending - 1u;
         float lx = __shfl_sync(kFull, sumlx, bb);
         float l2 = __shfl_sync(kFull, suml2, bb);
         float sc = __shfl_sync(kFull, score, bb);
-        const float xj = sx[bb * kRow + lane];
-        const float wj = sw[bb * kRow + lane];
-        float lj = sl[bb * kRow + lane];
+        const float xj = sX[bb * kRow1 + lane];
+        const float wj = sW[bb * kRow4 + lane];
+        float lj = sL[bb * kRow1 + lane];
         const float wxj = __fmul_rn(wj, xj);
         float d = __fdiv_rn(lx, l2);
-        int passes = 1, start = 0;
+        int passes = 2, start = 0;
         bool changed = false;
 #pragma unroll 1
         while (true) {
@@ -183,21 +234,28 @@ __device__ __forceinline__ void greedy_warp(float* sx, float* sw, float* sl, flo
                 start = 0;
             }
         }
-        sl[bb * kRow + lane] = lj;
+        sL[bb * kRow1 + lane] = lj;
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, IQQ_Q4_MIN_CTAS)
 q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
               int chunks_per_row, uint32_t* __restrict__ flags)
 {
     extern __shared__ float smem[];
-    __shared__ double s_red[kThreads / 32];
+    __shared__ double s_red[kWarps];
     const int lane = threadIdx.x & 31;
-    float* sx = smem + (threadIdx.x >> 5) * kWarpSmemFloats;
-    float* sw = sx + 32 * kRow;
-    float* sl = sw + 32 * kRow;
+    float* const warp_smem = smem + (threadIdx.x >> 5) * kWarpFloats;
+    float* const sW = warp_smem + kW;
+    float* const my_w = sW + lane * kRow4;
+    float* const my_awx = warp_smem + kAwx + lane * kRow4;
+    float* const my_ubm = warp_smem + kUbm + lane * kRow4;
+    float* const my_ub = warp_smem + kUb + lane * kRow4;
+    float* const sX = warp_smem + kScratch;             // x and the codes, after the sweep
+    float* const sL = warp_smem + kScratch + 32 * kRow1;
+    float* const my_x = sX + lane * kRow1;
+    float* const my_l = sL + lane * kRow1;
     const int64_t nb = n_per_row / QK;
     const int64_t nwork = nrows * chunks_per_row;
 
@@ -208,6 +266,34 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
         const int64_t qrow = rows_per_qw > 0 ? row / rows_per_qw : 0;
         const float* qr = qw != nullptr ? qw + qrow * n_per_row : nullptr;
         uint32_t bad = 0u;
+
+        // this thread's block (lanes past the row's end idle but join the warp steps);
+        // its loads are issued first so that they overlap the row reduction below
+        const int64_t b = static_cast<int64_t>(chunk) * kThreads + threadIdx.x;
+        const bool valid = b < nb;
+        float xv[QK];
+        float4 q4[QK / 4];
+        if (valid) {
+            const float4* xb4 = reinterpret_cast<const float4*>(xr + b * QK);
+#pragma unroll
+            for (int i = 0; i < QK / 4; ++i) {
+                const float4 v = __ldg(xb4 + i);
+                xv[4 * i] = v.x; xv[4 * i + 1] = v.y; xv[4 * i + 2] = v.z; xv[4 * i + 3] = v.w;
+            }
+            if (qr != nullptr) {
+                const float4* qb4 = reinterpret_cast<const float4*>(qr + b * QK);
+#pragma unroll
+                for (int i = 0; i < QK / 4; ++i) q4[i] = __ldg(qb4 + i);
+            } else {
+#pragma unroll
+                for (int i = 0; i < QK / 4; ++i) q4[i] = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < QK; ++j) xv[j] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < QK / 4; ++i) q4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
 
         // sigma2: binary64 sum of exact squares over the whole row
         double acc = 0.0;
@@ -227,149 +313,183 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
         if (chunk == 0 && nf != nf) bad |= IQQ_FLAG_NONFINITE_INPUT;
         const double sum = block_reduce_sum(acc, s_red);
         const float sigma2 = static_cast<float>(sum / static_cast<double>(n_per_row));
-        const bool check_qw = qr != nullptr && (rows_per_qw > 0 ? row % rows_per_qw == 0 : row == 0);
 
-        // ---- per thread: one block (lanes past the row's end idle but join the warp steps)
-        const int64_t b = static_cast<int64_t>(chunk) * kThreads + threadIdx.x;
-        const bool valid = b < nb;
-        float xv[QK], w[QK];
+        if (valid && qr != nullptr && (rows_per_qw > 0 ? row % rows_per_qw == 0 : row == 0)) {
+            float qmin = q4[0].x, qnf = 0.0f;
+#pragma unroll
+            for (int i = 0; i < QK / 4; ++i) {
+                qmin = fminf(fminf(qmin, q4[i].x), fminf(q4[i].y, fminf(q4[i].z, q4[i].w)));
+                qnf = __fmaf_rn(q4[i].x, 0.0f, qnf); qnf = __fmaf_rn(q4[i].y, 0.0f, qnf);
+                qnf = __fmaf_rn(q4[i].z, 0.0f, qnf); qnf = __fmaf_rn(q4[i].w, 0.0f, qnf);
+            }
+            if (qnf != qnf) bad |= IQQ_FLAG_NONFINITE_INPUT;
+            if (qmin < 0.0f) bad |= IQQ_FLAG_NEG_QW;
+        }
+
+        // importance weights (binary32, one rounding per operation) -> shared memory,
+        // then xmax (signed value of the first element of largest |x|)
+#pragma unroll
+        for (int i = 0; i < QK / 4; ++i) {
+            float4 w4 = q4[i];
+            if (weight_mode == 0) {
+                w4.x = __fmul_rn(w4.x, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i], xv[4 * i]))));
+                w4.y = __fmul_rn(w4.y, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i + 1], xv[4 * i + 1]))));
+                w4.z = __fmul_rn(w4.z, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i + 2], xv[4 * i + 2]))));
+                w4.w = __fmul_rn(w4.w, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i + 3], xv[4 * i + 3]))));
+            }
+            *reinterpret_cast<float4*>(my_w + 4 * i) = w4;
+        }
+        float amax = 0.0f, xmax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < QK; ++j) {
+            const float a = fabsf(xv[j]);
+            if (a > amax) { amax = a; xmax = xv[j]; }
+        }
+
+        // candidate sweep
+        float best = -INFINITY;
+        int kbest = 0;
+        {
+            const uint32_t sxm = __float_as_uint(xmax);
+#pragma unroll
+            for (int j4 = 0; j4 < QK; j4 += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(my_w + j4);
+                // |wx| and the clamp bound B: 8 when x_j has the sign of xmax (its code
+                // is <= 0, clamped at -8), 7 otherwise; also M + B for the adds form
+#define IQQ_DIFF(j) ((__float_as_uint(xv[j]) ^ sxm) >> 31)
+                *reinterpret_cast<float4*>(my_awx + j4) =
+                    make_float4(fabsf(__fmul_rn(w4.x, xv[j4])), fabsf(__fmul_rn(w4.y, xv[j4 + 1])),
+                                fabsf(__fmul_rn(w4.z, xv[j4 + 2])), fabsf(__fmul_rn(w4.w, xv[j4 + 3])));
+                if (kUseAdd)
+                    *reinterpret_cast<float4*>(my_ubm + j4) = make_float4(
+                        __uint_as_float(0x4B400008u - IQQ_DIFF(j4)), __uint_as_float(0x4B400008u - IQQ_DIFF(j4 + 1)),
+                        __uint_as_float(0x4B400008u - IQQ_DIFF(j4 + 2)), __uint_as_float(0x4B400008u - IQQ_DIFF(j4 + 3)));
+                if (kUseCvt)
+                    *reinterpret_cast<float4*>(my_ub + j4) =
+                        make_float4(IQQ_DIFF(j4) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 1) ? 7.0f : 8.0f,
+                                    IQQ_DIFF(j4 + 2) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 3) ? 7.0f : 8.0f);
+#undef IQQ_DIFF
+            }
+            if (amax > 0.0f) {
+                constexpr int N = IQQ_SWEEP_CPI;
+                int k0 = 0;
+#pragma unroll 1
+                for (; k0 + N <= kCand; k0 += N)
+                    sweep_group<N>(k0, xv, my_w, my_awx, my_ubm, my_ub, amax, best, kbest);
+#pragma unroll 1
+                for (; k0 < kCand; ++k0) sweep_group<1>(k0, xv, my_w, my_awx, my_ubm, my_ub, amax, best, kbest);
+            }
+        }
+        __syncwarp();  // the sweep area becomes the x / code staging area
+#pragma unroll
+        for (int j = 0; j < QK; ++j) my_x[j] = xv[j];
+
+        // codes of the winner (or of k = 0 for the fallback) and the greedy state
         int mode = 0;  // 0: nothing to search (all-zero or no block), 1: fallback, 2: search
         float sumlx = 0.0f, suml2 = 0.0f, score = 0.0f, dfb = 0.0f;
         {
-            float l[QK];
-            if (valid) {
-                const float4* xb4 = reinterpret_cast<const float4*>(xr + b * QK);
-#pragma unroll
-                for (int i = 0; i < QK / 4; ++i) {
-                    const float4 v = __ldg(xb4 + i);
-                    xv[4 * i] = v.x; xv[4 * i + 1] = v.y; xv[4 * i + 2] = v.z; xv[4 * i + 3] = v.w;
-                }
-                if (qr != nullptr) {
-                    const float4* qb4 = reinterpret_cast<const float4*>(qr + b * QK);
-#pragma unroll
-                    for (int i = 0; i < QK / 4; ++i) {
-                        const float4 v = __ldg(qb4 + i);
-                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-                    }
-                    if (check_qw) {
-                        float qmin = w[0], qnf = 0.0f;
-#pragma unroll
-                        for (int j = 0; j < QK; ++j) { qmin = fminf(qmin, w[j]); qnf = __fmaf_rn(w[j], 0.0f, qnf); }
-                        if (qnf != qnf) bad |= IQQ_FLAG_NONFINITE_INPUT;
-                        if (qmin < 0.0f) bad |= IQQ_FLAG_NEG_QW;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < QK; ++j) w[j] = 1.0f;
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < QK; ++j) { xv[j] = 0.0f; w[j] = 0.0f; }
-            }
-            // importance weights (binary32, one rounding per operation)
-            if (weight_mode == 0) {
-#pragma unroll
-                for (int j = 0; j < QK; ++j) {
-                    const float u = __fadd_rn(sigma2, __fmul_rn(xv[j], xv[j]));
-                    w[j] = __fmul_rn(w[j], __fsqrt_rn(u));
-                }
-            }
-            // xmax: signed value of the first element of largest |x|
-            float amax = 0.0f, xmax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < QK; ++j) {
-                const float a = fabsf(xv[j]);
-                if (a > amax) { amax = a; xmax = xv[j]; }
-            }
+            float iscale = 0.0f;
             if (amax > 0.0f) {
-                float best;
-                int kbest;
-                {
-                    float awx[QK], ub[QK];
-                    const uint32_t sxm = __float_as_uint(xmax);
-#pragma unroll
-                    for (int j = 0; j < QK; ++j) {
-                        awx[j] = fabsf(__fmul_rn(w[j], xv[j]));
-                        // clamp bound in the magic domain: M + 8 when x_j has the sign of
-                        // xmax (its code is <= 0, clamped at -8), M + 7 otherwise
-                        ub[j] = __uint_as_float(0x4B400008u - ((__float_as_uint(xv[j]) ^ sxm) >> 31));
-                    }
-                    sweep_block(xv, w, awx, ub, amax, best, kbest);
-                }
                 if (best == -INFINITY) {
                     // no candidate has positive weighted code energy: codes of k = 0, d = 1/iscale_0
-                    const float iscale0 = __fdiv_rn(-8.0f, xmax);
-#pragma unroll
-                    for (int j = 0; j < QK; ++j) l[j] = clamp_code(rint_small(__fmul_rn(iscale0, xv[j])));
-                    dfb = __fdiv_rn(1.0f, iscale0);
+                    iscale = __fdiv_rn(-8.0f, xmax);
+                    dfb = __fdiv_rn(1.0f, iscale);
                     mode = 1;
                 } else {
-                    const float iscale = __fdiv_rn(-c_cand[kbest], xmax);
-#pragma unroll
-                    for (int j = 0; j < QK; ++j) {
-                        l[j] = clamp_code(rint_small(__fmul_rn(iscale, xv[j])));
-                        sumlx = __fmaf_rn(__fmul_rn(w[j], xv[j]), l[j], sumlx);
-                        suml2 = __fmaf_rn(w[j], __fmul_rn(l[j], l[j]), suml2);
-                    }
+                    iscale = __fdiv_rn(-c_cand[kbest], xmax);
                     score = best;
                     mode = 2;
                 }
-            } else {
-#pragma unroll
-                for (int j = 0; j < QK; ++j) l[j] = 0.0f;
             }
-            // stage x, w and the codes for the warp's greedy step
-#pragma unroll
+#pragma unroll 4
             for (int j = 0; j < QK; ++j) {
-                sx[lane * kRow + j] = xv[j];
-                sw[lane * kRow + j] = w[j];
-                sl[lane * kRow + j] = l[j];
+                const float xj = my_x[j], wj = my_w[j];
+                const float l = clamp_code(rint_small(__fmul_rn(iscale, xj)));
+                my_l[j] = l;
+                sumlx = __fmaf_rn(__fmul_rn(wj, xj), l, sumlx);
+                suml2 = __fmaf_rn(wj, __fmul_rn(l, l), suml2);
             }
         }
-        __syncwarp();
-        greedy_warp(sx, sw, sl, sumlx, suml2, score, mode == 2);
+        // greedy pass 1: this thread's block, sequential over j, exactly as defined
+        bool changed = false;
+        if (mode == 2) {
+            float d = __fdiv_rn(sumlx, suml2);
+#pragma unroll 2
+            for (int j = 0; j < QK; ++j) {
+                const float xj = my_x[j], wj = my_w[j], lj = my_l[j];
+                const float g = __fmul_rn(d, __fmul_rn(wj, __fsub_rn(xj, __fmul_rn(d, lj))));
+                const float sg = g > 0.0f ? 1.0f : -1.0f;
+                const float ln = __fadd_rn(lj, sg);
+                const float nlx = __fadd_rn(sumlx, __fmul_rn(sg, __fmul_rn(wj, xj)));
+                const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), suml2);
+                if ((g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f) {
+                    const float ns = __fdiv_rn(__fmul_rn(nlx, nlx), nl2);
+                    if (ns > score) {
+                        my_l[j] = ln;
+                        sumlx = nlx;
+                        suml2 = nl2;
+                        score = ns;
+                        d = __fdiv_rn(sumlx, suml2);
+                        changed = true;
+                    }
+                }
+            }
+        }
+        // passes 2..5, warp-cooperatively, for the blocks whose first pass moved a code
+        const unsigned pending = __ballot_sync(kFull, changed);
+        if (pending != 0u) {
+            __syncwarp();
+            greedy_warp(sX, sW, sL, pending, sumlx, suml2, score);
+        }
         __syncwarp();
 
+        // final sums from the final codes, d, and the packed nibbles
         uint16_t d16 = 0;
-        uint32_t nib[QK / 2];
+        uint32_t qs[4];  // 16 bytes: byte i = (l[i]+8) | (l[i+16]+8) << 4
         {
-            float l[QK];
-#pragma unroll
-            for (int j = 0; j < QK; ++j) l[j] = sl[lane * kRow + j];
             float d = dfb;
             if (mode == 2) {
-                sumlx = 0.0f;
-                suml2 = 0.0f;
-#pragma unroll
+                float sfx = 0.0f, sf2 = 0.0f;
+#pragma unroll 4
                 for (int j = 0; j < QK; ++j) {
-                    sumlx = __fmaf_rn(__fmul_rn(w[j], xv[j]), l[j], sumlx);
-                    suml2 = __fmaf_rn(w[j], __fmul_rn(l[j], l[j]), suml2);
+                    const float xj = my_x[j], wj = my_w[j], lj = my_l[j];
+                    sfx = __fmaf_rn(__fmul_rn(wj, xj), lj, sfx);
+                    sf2 = __fmaf_rn(wj, __fmul_rn(lj, lj), sf2);
                 }
-                d = __fdiv_rn(sumlx, suml2);
+                d = __fdiv_rn(sfx, sf2);
             }
             if (mode != 0) {
                 d16 = __half_as_ushort(__float2half_rn(d));
                 if ((d16 & 0x7fffu) == 0x7c00u && isfinite(d)) bad |= IQQ_FLAG_SCALE_OVERFLOW;
             }
 #pragma unroll
-            for (int i = 0; i < QK / 2; ++i) {
-                const uint32_t lo = static_cast<uint32_t>(static_cast<int>(l[i]) + 8);
-                const uint32_t hi = static_cast<uint32_t>(static_cast<int>(l[i + QK / 2]) + 8);
-                nib[i] = lo | (hi << 4);
+            for (int i = 0; i < 4; ++i) {
+                uint32_t word = 0u;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // code + 8 from the float code: the low bits of (l + M + 8)
+                    const uint32_t lo = __float_as_uint(__fadd_rn(my_l[4 * i + k], kMagic + 8.0f)) & 0xfu;
+                    const uint32_t hi = __float_as_uint(__fadd_rn(my_l[4 * i + k + 16], kMagic + 8.0f)) & 0xfu;
+                    word |= (lo | (hi << 4)) << (8 * k);
+                }
+                qs[i] = word;
             }
         }
         if (valid) {
             uint16_t* o16 = reinterpret_cast<uint16_t*>(out + (row * nb + b) * IQQ_Q4_0_BLOCK_BYTES);
             o16[0] = d16;
 #pragma unroll
-            for (int i = 0; i < QK / 4; ++i) o16[1 + i] = static_cast<uint16_t>(nib[2 * i] | (nib[2 * i + 1] << 8));
+            for (int i = 0; i < 4; ++i) {
+                o16[1 + 2 * i] = static_cast<uint16_t>(qs[i] & 0xffffu);
+                o16[2 + 2 * i] = static_cast<uint16_t>(qs[i] >> 16);
+            }
         }
         iqq::raise_flags(flags, bad);
-        __syncwarp();  // the warp's staging area is rewritten by the next row
+        __syncwarp();  // the warp's shared memory is rewritten by the next row
     }
 }
 
-constexpr size_t kDynSmem = sizeof(float) * kWarpSmemFloats * (kThreads / 32);
+constexpr size_t kDynSmem = sizeof(float) * kWarpFloats * kWarps;
 
 }  // namespace
 
