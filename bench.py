@@ -44,6 +44,10 @@ DEQ_BYTES_PER_VALUE = 18.0 / 32.0 + 4.0
 RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
+# DRAM bytes (read + write) per value of q4_0_w_kernel from one ncu capture of the current
+# kernel (4096x4096 launch: 67.18 MB read + 2.87 MB written for 16,777,216 values); set
+# to None whenever the kernel changes until it is captured again.
+Q4_0_DRAM_BYTES_PER_VALUE = 70.06e6 / 16777216
 
 
 def peaks():
@@ -364,7 +368,10 @@ def main_ours(args):
                    "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (replicas)"},
         "roofline": {"bound": "alu", "kernel": "q4_0_w_kernel", "achieved": round(achieved, 3),
                      "peak": round(peak_ops, 3), "unit": "Tops/s",
-                     "frac": round(achieved / peak_ops, 4), "traffic": None,
+                     "frac": round(achieved / peak_ops, 4),
+                     "traffic": (None if Q4_0_DRAM_BYTES_PER_VALUE is None else
+                                 round(Q4_0_DRAM_BYTES_PER_VALUE * w.q4_elems / n_q4)),
+                     "traffic_unit": "bytes per launch (ncu dram read+write, scaled by values)",
                      "ops_per_value": round(ops_per_value, 2), "greedy_passes_mean": round(p_mean, 4),
                      "avg_launch_ms": round(q4_ms / n_q4, 5),
                      "peak_basis": f"{B200_SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x "

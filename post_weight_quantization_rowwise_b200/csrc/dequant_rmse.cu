@@ -49,24 +49,69 @@ __device__ __forceinline__ float code_value(uint32_t nib4, int k)
     return static_cast<float>(static_cast<int>((nib4 >> (4 * k)) & 0xfu) - 8);
 }
 
+#ifndef IQQ_DQ_UNROLL
+#define IQQ_DQ_UNROLL 1  // independent quads in flight per thread (dequant)
+#endif
+#ifndef IQQ_DQ_CTAS
+#define IQQ_DQ_CTAS 16   // CTAs per SM in the grid (dequant)
+#endif
+#ifndef IQQ_RMSE_UNROLL
+#define IQQ_RMSE_UNROLL 2  // independent rows in flight per thread (weighted RMSE)
+#endif
+#ifndef IQQ_RMSE_CTAS
+#define IQQ_RMSE_CTAS 16   // CTAs per SM in the grid (weighted RMSE)
+#endif
+#ifndef IQQ_RMSE_MIN_ROWS
+#define IQQ_RMSE_MIN_ROWS 8  // rows per CTA at least (weighted RMSE)
+#endif
+constexpr int kUnroll = IQQ_DQ_UNROLL;
+constexpr int kRowUnroll = IQQ_RMSE_UNROLL;
+
 __global__ void __launch_bounds__(kThreads)
 dequant_q4_0_kernel(const uint8_t* __restrict__ blocks, float4* __restrict__ y, int64_t nquads)
 {
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; t < nquads; t += stride) {
-        const int64_t g = t >> 3;
-        const int qd = static_cast<int>(t & 7);
-        const Quad q = load_quad(blocks + g * IQQ_Q4_0_BLOCK_BYTES, qd);
-        float4 o;
-        o.x = __fmul_rn(q.d, code_value(q.nib4, 0));
-        o.y = __fmul_rn(q.d, code_value(q.nib4, 1));
-        o.z = __fmul_rn(q.d, code_value(q.nib4, 2));
-        o.w = __fmul_rn(q.d, code_value(q.nib4, 3));
-        __stcs(y + t, o);  // streaming store: the output is not re-read here
+    // each iteration handles kUnroll quads spaced kThreads apart, so every warp-level
+    // store stays contiguous; all loads of an iteration are issued before any store
+    const int64_t step = static_cast<int64_t>(gridDim.x) * kThreads * kUnroll;
+    for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * kThreads * kUnroll + threadIdx.x; t0 < nquads;
+         t0 += step) {
+        Quad q[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t t = t0 + u * kThreads;
+            if (t < nquads) q[u] = load_quad(blocks + (t >> 3) * IQQ_Q4_0_BLOCK_BYTES, static_cast<int>(t & 7));
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t t = t0 + u * kThreads;
+            if (t < nquads) {
+                float4 o;
+                o.x = __fmul_rn(q[u].d, code_value(q[u].nib4, 0));
+                o.y = __fmul_rn(q[u].d, code_value(q[u].nib4, 1));
+                o.z = __fmul_rn(q[u].d, code_value(q[u].nib4, 2));
+                o.w = __fmul_rn(q[u].d, code_value(q[u].nib4, 3));
+                __stcs(y + t, o);  // streaming store: the output is not re-read here
+            }
+        }
+    }
+}
+
+// Adds the squared errors of one row's quad to the per-column accumulators.
+__device__ __forceinline__ void rmse_quad(const float4 xv, const Quad q, double (&col)[4], float& emax)
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float xk = k == 0 ? xv.x : k == 1 ? xv.y : k == 2 ? xv.z : xv.w;
+        const float e = __fsub_rn(xk, __fmul_rn(q.d, code_value(q.nib4, k)));
+        emax = fmaxf(emax, fabsf(e));
+        const double ed = static_cast<double>(e);
+        col[k] = fma(ed, ed, col[k]);
     }
 }
 
 // Rows [blockIdx.y*rows_per_cta, ...) x column quad blockIdx.x*kThreads + threadIdx.x.
+// Per column the thread keeps sum_r e^2 (binary64) and multiplies by qw once per
+// imatrix row, so qw is read and converted once per row segment, not per value.
 __global__ void __launch_bounds__(kThreads)
 weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ blocks,
                      const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
@@ -83,47 +128,38 @@ weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ bl
     if (cq < nq) {
         const int64_t b = cq >> 3;
         const int qd = static_cast<int>(cq & 7);
-        double col[4] = {0.0, 0.0, 0.0, 0.0};
-        double qd4[4] = {1.0, 1.0, 1.0, 1.0};
-        int64_t cur = -1, nrow_cur = 0;
-        for (int64_t r = r0; r < r1; ++r) {
-            const int64_t qrow = rows_per_qw > 0 ? r / rows_per_qw : 0;
-            if (qrow != cur) {
-                if (cur >= 0) {
+        for (int64_t s0 = r0; s0 < r1;) {
+            // a segment of rows sharing one imatrix row
+            const int64_t qrow = rows_per_qw > 0 ? s0 / rows_per_qw : 0;
+            const int64_t s1 = rows_per_qw > 0 ? min(r1, (qrow + 1) * rows_per_qw) : r1;
+            double col[4] = {0.0, 0.0, 0.0, 0.0};
+            int64_t r = s0;
+            for (; r + kRowUnroll <= s1; r += kRowUnroll) {
+                float4 xv[kRowUnroll];
+                Quad q[kRowUnroll];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        sw = fma(qd4[k], col[k], sw);
-                        se += col[k];
-                        sq = fma(qd4[k], static_cast<double>(nrow_cur), sq);
-                        col[k] = 0.0;
-                    }
+                for (int u = 0; u < kRowUnroll; ++u) {
+                    xv[u] = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + (r + u) * n_per_row) + cq);
+                    q[u] = load_quad(blocks + ((r + u) * nb + b) * IQQ_Q4_0_BLOCK_BYTES, qd);
                 }
-                if (qw != nullptr) {
-                    const float4 w = __ldg(reinterpret_cast<const float4*>(qw + qrow * n_per_row) + cq);
-                    qd4[0] = w.x; qd4[1] = w.y; qd4[2] = w.z; qd4[3] = w.w;
-                }
-                cur = qrow;
-                nrow_cur = 0;
-            }
-            const float4 xv = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + r * n_per_row) + cq);
-            const Quad q = load_quad(blocks + (r * nb + b) * IQQ_Q4_0_BLOCK_BYTES, qd);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float xk = k == 0 ? xv.x : k == 1 ? xv.y : k == 2 ? xv.z : xv.w;
-                const float e = __fsub_rn(xk, __fmul_rn(q.d, code_value(q.nib4, k)));
-                emax = fmaxf(emax, fabsf(e));
-                const double ed = static_cast<double>(e);
-                col[k] = fma(ed, ed, col[k]);
+                for (int u = 0; u < kRowUnroll; ++u) rmse_quad(xv[u], q[u], col, emax);
             }
-            ++nrow_cur;
-        }
-        if (cur >= 0) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                sw = fma(qd4[k], col[k], sw);
-                se += col[k];
-                sq = fma(qd4[k], static_cast<double>(nrow_cur), sq);
+            for (; r < s1; ++r) {
+                const float4 xv = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + r * n_per_row) + cq);
+                rmse_quad(xv, load_quad(blocks + (r * nb + b) * IQQ_Q4_0_BLOCK_BYTES, qd), col, emax);
             }
+            float4 w = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            if (qw != nullptr) w = __ldg(reinterpret_cast<const float4*>(qw + qrow * n_per_row) + cq);
+            const double nr = static_cast<double>(s1 - s0);
+            sw = fma(static_cast<double>(w.x), col[0], sw);
+            sw = fma(static_cast<double>(w.y), col[1], sw);
+            sw = fma(static_cast<double>(w.z), col[2], sw);
+            sw = fma(static_cast<double>(w.w), col[3], sw);
+            se += (col[0] + col[1]) + (col[2] + col[3]);
+            sq = fma(static_cast<double>(w.x) + static_cast<double>(w.y) + static_cast<double>(w.z) +
+                         static_cast<double>(w.w), nr, sq);
+            s0 = s1;
         }
     }
 
@@ -171,8 +207,8 @@ extern "C" iqq_status iqq_dequant_q4_0(const void* blocks, float* y, int64_t nro
     if (blocks == nullptr || y == nullptr) return IQQ_ERR_NULL;
     if (!iqq::aligned(blocks, 2) || !iqq::aligned(y, 16)) return IQQ_ERR_ALIGN;
     const int64_t nquads = nrows * n_per_row / 4;
-    const int64_t need = (nquads + kThreads - 1) / kThreads;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    const int64_t need = (nquads + kThreads * kUnroll - 1) / (kThreads * kUnroll);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * IQQ_DQ_CTAS;
     const int grid = static_cast<int>(need < cap ? need : cap);
     dequant_q4_0_kernel<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint8_t*>(blocks), reinterpret_cast<float4*>(y), nquads);
@@ -192,12 +228,12 @@ extern "C" iqq_status iqq_weighted_rmse(const float* x, const void* blocks, cons
         return IQQ_ERR_ALIGN;
     const int64_t nq = n_per_row / 4;
     const int64_t gx = (nq + kThreads - 1) / kThreads;
-    // about 16 resident CTAs' worth per SM, at least 8 rows per CTA
-    const int64_t target = static_cast<int64_t>(sm_count()) * 16;
+    // IQQ_RMSE_CTAS CTAs per SM, at least IQQ_RMSE_MIN_ROWS rows per CTA
+    const int64_t target = static_cast<int64_t>(sm_count()) * IQQ_RMSE_CTAS;
     int64_t gy = target / gx;
     if (gy < 1) gy = 1;
     int64_t rpc = (nrows + gy - 1) / gy;
-    if (rpc < 8) rpc = 8;
+    if (rpc < IQQ_RMSE_MIN_ROWS) rpc = IQQ_RMSE_MIN_ROWS;
     gy = (nrows + rpc - 1) / rpc;
     if (gx > 0x7fffffff || gy > 65535) return IQQ_ERR_SHAPE;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));

@@ -14,13 +14,13 @@
 // 16-byte load, so a warp reads 512 contiguous bytes), writes qs[4t..4t+3]
 // as one 32-bit store (a warp writes 128 contiguous bytes), and lanes 0, 8,
 // 16, 24 write the four sums.  The work is HBM bound (4 B read + 140/128 B
-// written per value); each warp keeps two blocks in flight.
+// written per value); each warp keeps four blocks in flight.
 #include "common.cuh"
 
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 2;
+constexpr int kUnroll = 4;
 
 // rint with the cvt.rni saturating conversion: +-Inf -> INT_MAX / INT_MIN,
 // NaN -> 0; then the symmetric int8 clamp.
