@@ -146,7 +146,7 @@ def _oracle_chunk(args):
     return x.size, time.perf_counter() - t0, int(passes.sum()), int(passes.size)
 
 
-def oracle_sample(target_seconds: float = 12.0, cores: int | None = None):
+def oracle_sample(target_seconds: float = 12.0, cores: int | None = None, pool=None):
     """Times the unchanged single-threaded oracle on a bounded sample of the workload,
     one process per core: rows of every tensor shape of the layer set (same recipe,
     in the layer set's proportions of values) and Q8_K_128 activation rows (in the
@@ -168,9 +168,11 @@ def oracle_sample(target_seconds: float = 12.0, cores: int | None = None):
             jobs.append(("q4", min(per, rows - r0), c, 9000 + 100 * i + k, True))
     q8_rows = max(1, int(budget * 4096 * 7168 / (32 * layer_elems) / 7168))
     jobs.append(("q8", q8_rows, 7168, 2, False))
-    ctx = mp.get_context("spawn")
     t0 = time.perf_counter()
-    with ctx.Pool(cores) as pool:
+    if pool is None:
+        with mp.get_context("spawn").Pool(cores) as own:
+            res = own.map(_oracle_chunk, jobs, chunksize=1)
+    else:
         res = pool.map(_oracle_chunk, jobs, chunksize=1)
     wall = time.perf_counter() - t0
     elems = sum(r[0] for r in res)
@@ -192,8 +194,9 @@ class Workload:
         from post_weight_quantization_rowwise_b200 import synth
         self.tensors = synth.llama2_7b_layer_set(layers)
         self.x, self.qw, self.blocks = [], [], []
+        from post_weight_quantization_rowwise_b200 import replicas
+        seed_off = replicas.rank_seed_offset(rank)
         for t in self.tensors:
-            seed_off = 1_000_000 * rank
             g = synth.Tensor2D(t.name, t.rows, t.cols, t.seed + seed_off, t.sigma, t.bf16,
                                t.boost_frac)
             self.x.append(g.weights(device=dev))
@@ -203,7 +206,7 @@ class Workload:
         maxn = max(t.numel for t in self.tensors)
         self.y = torch.empty(maxn, dtype=torch.float32, device=dev)
         self.acc = torch.zeros(4, dtype=torch.float64, device=dev)
-        self.act = synth.activations(4096, 7168, seed=2 + 1_000_000 * rank, device=dev)
+        self.act = synth.activations(4096, 7168, seed=2 + seed_off, device=dev)
         self.q8 = torch.empty(4096 * 56 * 140, dtype=torch.uint8, device=dev)
         self.q4_elems = sum(t.numel for t in self.tensors)
         self.q8_elems = self.act.numel()
@@ -328,11 +331,11 @@ def main_ours(args):
         for p in range(4):
             phase[p] += ev[s][p].elapsed_time(ev[s][p + 1])
     total_ms = ev[0][0].elapsed_time(ev[-1][4])
-    t = torch.tensor([total_ms] + phase, dtype=torch.float64, device=dev)
+    from post_weight_quantization_rowwise_b200 import replicas
+    times = replicas.max_over_ranks([total_ms] + phase, device=dev)  # the slowest rank
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
-    total_ms, phase = float(t[0]), [float(v) for v in t[1:]]
+    total_ms, phase = times[0], times[1:]
     acc = w.acc.cpu().tolist()
 
     e2e = None
@@ -403,15 +406,21 @@ def main_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import multiprocessing as mp
     vals, cores, sample, p = [], None, None, None
-    per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
-    for i in range(args.warmup + args.steps):
-        v, cores, sample, p = oracle_sample(per_step)
-        if i >= args.warmup:
-            vals.append(v)
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    ncores = os.cpu_count() or 1
+    with mp.get_context("spawn").Pool(ncores) as pool:
+        for i in range(args.warmup + args.steps):
+            v, cores, sample, p = oracle_sample(per_step, ncores, pool)
+            if i >= args.warmup:
+                vals.append(v)
     value = statistics.median(vals)
+    from post_weight_quantization_rowwise_b200 import synth
+    full = sum(t.numel for t in synth.llama2_7b_layer_set(args.layers)) + 4096 * 7168
     out = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(full / (value * 1e9) * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
            "data": "synthetic (seeded; no model weights or calibration data)",
            "config": {"workload": WORKLOAD, "layers": args.layers}, "impl": "reference",
