@@ -47,7 +47,7 @@ FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of q4_0_w_kernel from one ncu capture of the current
 # kernel (4096x4096 launch: 67.18 MB read + 2.87 MB written for 16,777,216 values); set
 # to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = 70.06e6 / 16777216
+Q4_0_DRAM_BYTES_PER_VALUE = None
 
 
 def peaks():

@@ -39,9 +39,9 @@
 // reduces sigma2 over its whole row (the row is read from HBM once and from L2
 // by the row's other chunks).  Per warp, shared memory holds the weights w of
 // its 32 blocks and a scratch area used first by the sweep (|wx| and the clamp
-// bounds in both rounding domains) and then by the later steps (x and the
-// codes), whose per-value loops then need no registers per value and stay
-// rolled (small code, fewer registers).  Built with -fmad=false: no
+// bounds) and then by the later steps (x and the codes), whose per-value loops
+// then need no registers per value and stay rolled (small code, fewer
+// registers).  Built with -fmad=false: no
 // contraction except the explicit __fmaf_rn calls.
 #include <cuda_fp16.h>
 
@@ -65,18 +65,13 @@ constexpr int kRow1 = QK + 1;
 #define IQQ_SWEEP_CPI 2  // candidates per sweep iteration
 #endif
 #ifndef IQQ_SWEEP_CVT_MASK
-#define IQQ_SWEEP_CVT_MASK 0  // bit c set: candidate c of a group rounds with cvt.rni
+#define IQQ_SWEEP_CVT_MASK 1  // bit c set: candidate c of a group rounds with cvt.rni
 #endif
-constexpr int kCvtAll = (1 << IQQ_SWEEP_CPI) - 1;
-constexpr bool kUseCvt = (IQQ_SWEEP_CVT_MASK & kCvtAll) != 0;     // some candidates round by cvt.rni
-constexpr bool kUseAdd = (IQQ_SWEEP_CVT_MASK & kCvtAll) != kCvtAll;  // some by the magic adds
 constexpr int kW = 0;                    // w[32][36]
-constexpr int kScratch = 32 * kRow4;     // sweep: |wx|, then M + B and/or B, each [32][36];
-                                         // later: x[32][33], l[32][33]
+constexpr int kScratch = 32 * kRow4;     // sweep: |wx|[32][36], B[32][36]; later: x[32][33], l[32][33]
 constexpr int kAwx = kScratch;
-constexpr int kUbm = kAwx + 32 * kRow4;
-constexpr int kUb = kUbm + (kUseAdd ? 32 * kRow4 : 0);
-constexpr int kWarpFloats = kUb + (kUseCvt ? 32 * kRow4 : 0);
+constexpr int kUb = kAwx + 32 * kRow4;
+constexpr int kWarpFloats = kUb + 32 * kRow4;
 static_assert(kScratch + 2 * 32 * kRow1 <= kWarpFloats, "staging fits in the sweep area");
 
 #ifndef IQQ_Q4_MIN_CTAS
@@ -119,6 +114,7 @@ __device__ __forceinline__ void keep_best(float s, float t, int k, float& best, 
     }
 }
 
+
 // N candidates k0..k0+N-1 over the block.  Per value and candidate: v = a_k*|x|,
 // the code magnitude m = min(rint(v), B) -- rint either by cvt.rni, or as
 // min(v + M, M + B) - M -- then the two sequential sums |sumlx| += |wx|*m and
@@ -127,10 +123,10 @@ __device__ __forceinline__ void keep_best(float s, float t, int k, float& best, 
 template <int N>
 __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const float* __restrict__ my_w,
                                             const float* __restrict__ my_awx,
-                                            const float* __restrict__ my_ubm,
                                             const float* __restrict__ my_ub, float amax,
                                             float& best, int& kbest)
 {
+    constexpr int kMask = IQQ_SWEEP_CVT_MASK & ((1 << N) - 1);
     float a[N], s[N], t[N];
 #pragma unroll
     for (int c = 0; c < N; ++c) {
@@ -141,14 +137,9 @@ __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const
 #pragma unroll
     for (int j4 = 0; j4 < QK; j4 += 4) {
         const float4 aw = *reinterpret_cast<const float4*>(my_awx + j4);
+        const float4 ub = *reinterpret_cast<const float4*>(my_ub + j4);
         const float4 ww = *reinterpret_cast<const float4*>(my_w + j4);
-        float4 um = make_float4(0.f, 0.f, 0.f, 0.f), ub = um;
-        if ((IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) != ((1 << N) - 1)) um = *reinterpret_cast<const float4*>(my_ubm + j4);
-        if ((IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) != 0) ub = *reinterpret_cast<const float4*>(my_ub + j4);
-        static_assert(kUseAdd || (IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) == ((1 << N) - 1), "layout");
-        static_assert(kUseCvt || (IQQ_SWEEP_CVT_MASK & ((1 << N) - 1)) == 0, "layout");
         const float awv[4] = {aw.x, aw.y, aw.z, aw.w};
-        const float umv[4] = {um.x, um.y, um.z, um.w};
         const float ubv[4] = {ub.x, ub.y, ub.z, ub.w};
         const float wv[4] = {ww.x, ww.y, ww.z, ww.w};
 #pragma unroll
@@ -156,9 +147,9 @@ __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const
 #pragma unroll
             for (int c = 0; c < N; ++c) {
                 const float v = __fmul_rn(a[c], fabsf(xv[j4 + q]));
-                const float m = ((IQQ_SWEEP_CVT_MASK >> c) & 1)
-                                    ? fminf(rintf(v), ubv[q])
-                                    : __fsub_rn(fminf(__fadd_rn(v, kMagic), umv[q]), kMagic);
+                // rint(v): one conversion-pipe op, or two FMA-pipe adds
+                const float r = ((kMask >> c) & 1) ? rintf(v) : rint_small(v);
+                const float m = fminf(r, ubv[q]);
                 s[c] = __fmaf_rn(awv[q], m, s[c]);
                 t[c] = __fmaf_rn(wv[q], __fmul_rn(m, m), t[c]);
             }
@@ -250,7 +241,6 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
     float* const sW = warp_smem + kW;
     float* const my_w = sW + lane * kRow4;
     float* const my_awx = warp_smem + kAwx + lane * kRow4;
-    float* const my_ubm = warp_smem + kUbm + lane * kRow4;
     float* const my_ub = warp_smem + kUb + lane * kRow4;
     float* const sX = warp_smem + kScratch;             // x and the codes, after the sweep
     float* const sL = warp_smem + kScratch + 32 * kRow1;
@@ -360,14 +350,9 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 *reinterpret_cast<float4*>(my_awx + j4) =
                     make_float4(fabsf(__fmul_rn(w4.x, xv[j4])), fabsf(__fmul_rn(w4.y, xv[j4 + 1])),
                                 fabsf(__fmul_rn(w4.z, xv[j4 + 2])), fabsf(__fmul_rn(w4.w, xv[j4 + 3])));
-                if (kUseAdd)
-                    *reinterpret_cast<float4*>(my_ubm + j4) = make_float4(
-                        __uint_as_float(0x4B400008u - IQQ_DIFF(j4)), __uint_as_float(0x4B400008u - IQQ_DIFF(j4 + 1)),
-                        __uint_as_float(0x4B400008u - IQQ_DIFF(j4 + 2)), __uint_as_float(0x4B400008u - IQQ_DIFF(j4 + 3)));
-                if (kUseCvt)
-                    *reinterpret_cast<float4*>(my_ub + j4) =
-                        make_float4(IQQ_DIFF(j4) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 1) ? 7.0f : 8.0f,
-                                    IQQ_DIFF(j4 + 2) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 3) ? 7.0f : 8.0f);
+                *reinterpret_cast<float4*>(my_ub + j4) =
+                    make_float4(IQQ_DIFF(j4) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 1) ? 7.0f : 8.0f,
+                                IQQ_DIFF(j4 + 2) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 3) ? 7.0f : 8.0f);
 #undef IQQ_DIFF
             }
             if (amax > 0.0f) {
@@ -375,9 +360,9 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 int k0 = 0;
 #pragma unroll 1
                 for (; k0 + N <= kCand; k0 += N)
-                    sweep_group<N>(k0, xv, my_w, my_awx, my_ubm, my_ub, amax, best, kbest);
+                    sweep_group<N>(k0, xv, my_w, my_awx, my_ub, amax, best, kbest);
 #pragma unroll 1
-                for (; k0 < kCand; ++k0) sweep_group<1>(k0, xv, my_w, my_awx, my_ubm, my_ub, amax, best, kbest);
+                for (; k0 < kCand; ++k0) sweep_group<1>(k0, xv, my_w, my_awx, my_ub, amax, best, kbest);
             }
         }
         __syncwarp();  // the sweep area becomes the x / code staging area
@@ -422,8 +407,14 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 const float ln = __fadd_rn(lj, sg);
                 const float nlx = __fadd_rn(sumlx, __fmul_rn(sg, __fmul_rn(wj, xj)));
                 const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), suml2);
-                if ((g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f) {
-                    const float ns = __fdiv_rn(__fmul_rn(nlx, nlx), nl2);
+                const float a2 = __fmul_rn(nlx, nlx);
+                // rejected for certain when fl(nlx^2) <= thr = fl(fl(score*nl2)*(1 - 2^-22)):
+                // with no underflow or overflow (thr in [1e-30, 1e30]) thr < score*nl2, so
+                // then nlx^2/nl2 < score exactly and its rounded quotient cannot exceed score
+                const float thr = __fmul_rn(__fmul_rn(score, nl2), 0.99999976158142089844f);
+                const bool maybe = !(a2 <= thr && thr >= 1e-30f && thr <= 1e30f);
+                if (maybe && (g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f) {
+                    const float ns = __fdiv_rn(a2, nl2);
                     if (ns > score) {
                         my_l[j] = ln;
                         sumlx = nlx;
