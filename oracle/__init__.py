@@ -56,6 +56,8 @@ def lib():
         L.oracle_fp16_from_float_array.argtypes = [_f32p, ctypes.POINTER(ctypes.c_uint16), _i64]
         L.oracle_fp16_to_float_array.restype = None
         L.oracle_fp16_to_float_array.argtypes = [ctypes.POINTER(ctypes.c_uint16), _f32p, _i64]
+        L.oracle_quantize_q8_1.restype = ctypes.c_int64
+        L.oracle_quantize_q8_1.argtypes = [_f32p, _u8p, _i64, _i64]
         L.oracle_quantize_q8_k128.restype = ctypes.c_int
         L.oracle_quantize_q8_k128.argtypes = [_f32p, _u8p, _i64, _i64, _u32p]
         _LIB = L
@@ -177,6 +179,30 @@ def quantize_q8_k128(x):
     if rc != 0:
         raise ValueError("oracle_quantize_q8_k128: bad shape")
     return out, int(flags[0])
+
+
+Q8_1_BYTES = 36
+
+
+def quantize_q8_1(x):
+    """Q8_1 blocks of a [nrows, n_per_row] float32 matrix; returns (blocks uint8, overflow count)."""
+    x = _f32(x)
+    nrows, n = x.shape
+    out = np.zeros((nrows, (n // 32) * Q8_1_BYTES), np.uint8)
+    cnt = lib().oracle_quantize_q8_1(_ptr(x, _f32p), _ptr(out, _u8p), nrows, n)
+    if cnt < 0:
+        raise ValueError("oracle_quantize_q8_1: bad shape")
+    return out, int(cnt)
+
+
+def decode_q8_1(blocks, nrows: int, n_per_row: int):
+    """Split Q8_1 bytes into (d uint16 [nrows, nb], s uint16 [nrows, nb], qs int8 [nrows, n])."""
+    nb = n_per_row // 32
+    b = np.ascontiguousarray(blocks, dtype=np.uint8).reshape(nrows, nb, Q8_1_BYTES)
+    d = b[:, :, 0:2].copy().view(np.uint16).reshape(nrows, nb)
+    s = b[:, :, 2:4].copy().view(np.uint16).reshape(nrows, nb)
+    qs = b[:, :, 4:36].copy().view(np.int8).reshape(nrows, n_per_row)
+    return d, s, qs
 
 
 def decode_q8_k128(blocks, nrows: int, n_per_row: int):

@@ -123,19 +123,32 @@ float oracle_row_sigma2(const float *x, int64_t n)
 /* Importance weights of one block, [W] §一:                           */
 /*   mode 0: weight[j] = qw[j] * sqrtf(sigma2 + xb[j]*xb[j])           */
 /*   mode 1: weight[j] = qw[j]      (the variant [W] §一/§二 discusses) */
-/* qw == NULL means qw[j] = 1.  Each operation rounds to binary32:     */
-/* t = x*x, u = sigma2 + t, s = sqrtf(u), w = qw*s.                    */
+/* and the magnitude forms [W] §二 lists as tried before imatrix       */
+/* existed (x^2, |x|, sigma^2 + x^2, sigma + |x|), here times qw:       */
+/*   mode 2: qw * (x*x)        mode 3: qw * |x|                         */
+/*   mode 4: qw * (sigma2 + x*x)   mode 5: qw * (sqrtf(sigma2) + |x|)   */
+/* qw == NULL means qw[j] = 1 (the pure magnitude forms).  Each         */
+/* operation rounds to binary32: t = x*x, u = sigma2 + t, s = sqrtf(u), */
+/* w = qw*s; sigma = sqrtf(sigma2).                                     */
 /* ------------------------------------------------------------------ */
 void oracle_block_weights(const float *xb, const float *qwb, int n, float sigma2,
                           int weight_mode, float *w)
 {
+    const float sigma = sqrtf(sigma2);
     for (int j = 0; j < n; ++j) {
         float q = qwb ? qwb[j] : 1.0f;
-        if (weight_mode == 1) { w[j] = q; continue; }
-        float t = xb[j] * xb[j];
-        float u = sigma2 + t;
-        float s = sqrtf(u);
-        w[j] = q * s;
+        float x = xb[j];
+        float t = x * x;
+        float m;
+        switch (weight_mode) {
+        case 1: m = 1.0f; break;
+        case 2: m = t; break;
+        case 3: m = fabsf(x); break;
+        case 4: m = sigma2 + t; break;
+        case 5: m = sigma + fabsf(x); break;
+        default: m = sqrtf(sigma2 + t); break;
+        }
+        w[j] = weight_mode == 1 ? q : q * m;
     }
 }
 
@@ -302,6 +315,7 @@ int oracle_quantize_q4_0_w(const float *x, const float *qw, uint8_t *out, int64_
                            uint32_t *flags, int32_t *passes)
 {
     if (n_per_row % ORACLE_QK4_0 != 0 || nrows < 0 || n_per_row < 0) return -1;
+    if (weight_mode < 0 || weight_mode > 5) return -1;
     const int64_t nb = n_per_row / ORACLE_QK4_0;
     float w[ORACLE_QK4_0];
     int8_t L[ORACLE_QK4_0];
@@ -425,6 +439,50 @@ int oracle_quantize_q8_k128(const float *x, uint8_t *out, int64_t nrows, int64_t
         }
     }
     return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Q8_1 activation quantization, the format [Q8] 修复前的数值隐患       */
+/* describes: blocks of 32 values with a binary16 scale d = x_max/127  */
+/* and a binary16 sum s = d * sum(q).  s can overflow binary16 even    */
+/* when d fits, which is the failure Q8_K_128 removes.                 */
+/* Readings (same code rule as Q8_K_128): amax = max|x|, d = amax/127, */
+/* id = amax > 0 ? 127/amax : 0, q = clamp(rint(x*id), -127, 127)      */
+/* (a NaN product gives 0); s = d * (float)sum(q) in binary32; both     */
+/* stored as binary16 RNE.  Layout: half d | half s | int8 qs[32]      */
+/* = 36 bytes.  Returns the number of blocks whose stored s is +-Inf   */
+/* while d is finite.                                                  */
+/* ------------------------------------------------------------------ */
+int64_t oracle_quantize_q8_1(const float *x, uint8_t *out, int64_t nrows, int64_t n_per_row)
+{
+    if (n_per_row % 32 != 0 || nrows < 0 || n_per_row < 0) return -1;
+    const int64_t nblk = nrows * (n_per_row / 32);
+    int64_t overflow = 0;
+    for (int64_t g = 0; g < nblk; ++g) {
+        const float *xb = x + g * 32;
+        uint8_t *blk = out + g * 36;
+        float amax = 0.0f;
+        for (int j = 0; j < 32; ++j) {
+            float a = fabsf(xb[j]);
+            if (a > amax) amax = a;
+        }
+        float d = amax / 127.0f;
+        float id = amax > 0.0f ? 127.0f / amax : 0.0f;
+        int sum = 0;
+        for (int j = 0; j < 32; ++j) {
+            float v = xb[j] * id;
+            int q = 0;
+            if (v == v) q = (int)fminf(fmaxf(rintf(v), -127.0f), 127.0f);
+            blk[4 + j] = (uint8_t)(int8_t)q;
+            sum += q;
+        }
+        float sf = d * (float)sum;
+        uint16_t hd = oracle_fp16_from_float(d), hs = oracle_fp16_from_float(sf);
+        memcpy(blk, &hd, 2);
+        memcpy(blk + 2, &hs, 2);
+        if ((hs & 0x7fffu) == 0x7c00u && (hd & 0x7fffu) != 0x7c00u) ++overflow;
+    }
+    return overflow;
 }
 
 /* Layout constants, for the test suite's self-description checks. */

@@ -77,6 +77,43 @@ def test_weights_closed_form_and_asymptotes(orc):
                        np.sqrt(np.float64(s2) + x.astype(np.float64) ** 2), rtol=3e-7)
 
 
+def test_magnitude_weight_forms(orc):
+    """[W] §二: the importance forms tried before imatrix existed -- x^2, |x|,
+    sigma^2 + x^2, sigma + |x| (weight modes 2..5), times qw when given."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal(32) * 0.02).astype(np.float32)
+    qw = np.exp(rng.standard_normal(32)).astype(np.float32)
+    s2 = np.float32(4e-4)
+    xd, qd, sd = x.astype(np.float64), qw.astype(np.float64), float(s2)
+    refs = {2: xd * xd, 3: np.abs(xd), 4: sd + xd * xd, 5: np.sqrt(sd) + np.abs(xd)}
+    for mode, ref in refs.items():
+        w = orc.block_weights(x, qw, float(s2), mode)
+        assert np.all(np.abs(w - qd * ref) <= 3 * 2.0 ** -24 * qd * ref), mode
+        w1 = orc.block_weights(x, None, float(s2), mode)
+        assert np.all(np.abs(w1 - ref) <= 2 * 2.0 ** -24 * ref), mode
+    with pytest.raises(ValueError):
+        orc.quantize_q4_0_w(x.reshape(1, 32), qw, weight_mode=6)
+
+
+@pytest.mark.parametrize("mode", [2, 3, 4, 5])
+def test_magnitude_forms_keep_the_symmetries(orc, mode):
+    """Every form is even in x and homogeneous in a power-of-two scale of x, so the
+    codes survive x -> -x and x -> 2^k x, and d follows the sign and the scale."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal((16, 256)) * 0.02).astype(np.float32)
+    qw = np.exp(rng.standard_normal(256)).astype(np.float32)
+    a, _ = orc.quantize_q4_0_w(x, qw, weight_mode=mode)
+    b, _ = orc.quantize_q4_0_w(-x, qw, weight_mode=mode)
+    c, _ = orc.quantize_q4_0_w(x * np.float32(4.0), qw, weight_mode=mode)
+    da, ca = orc.decode_q4_0(a, 16, 256)
+    db, cb = orc.decode_q4_0(b, 16, 256)
+    dc, cc = orc.decode_q4_0(c, 16, 256)
+    assert np.array_equal(ca, cb) and np.array_equal(da ^ 0x8000, db)
+    assert np.array_equal(ca, cc)
+    assert np.array_equal(da.view(np.float16).astype(np.float32) * np.float32(4.0),
+                          dc.view(np.float16).astype(np.float32))
+
+
 # ------------------------------------------------------------------ exact blocks (golden)
 
 def _expected_block_bytes(d0, n):

@@ -126,3 +126,33 @@ def test_nonfinite_flag_and_shape_error(orc):
     assert orc.quantize_q8_k128(x)[1] & 1
     with pytest.raises(ValueError):
         orc.quantize_q8_k128(np.zeros((1, 96), np.float32))
+
+
+# ------------------------------------------------------------------ Q8_1 (the overflowing format)
+
+def test_q8_1_invariants_and_overflow_count(orc):
+    """[Q8] 修复前的数值隐患: Q8_1 keeps d = x_max/127 and s = d*sum(q) as fp16 per 32
+    values; s overflows on blocks whose d still fits."""
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((16, 1024)).astype(np.float32)
+    m = rng.random(x.shape) < 2e-3
+    x[m] = (rng.uniform(6e4, 2e5, m.sum()) * rng.choice([-1, 1], m.sum())).astype(np.float32)
+    out, n_over = orc.quantize_q8_1(x)
+    d16, s16, qs = orc.decode_q8_1(out, 16, 1024)
+    xb = x.reshape(16, 32, 32)
+    amax = np.abs(xb).max(axis=2)
+    d = amax / np.float32(127.0)
+    assert np.array_equal(d16, d.astype(np.float16).view(np.uint16))
+    q = qs.reshape(16, 32, 32).astype(np.int64)
+    assert np.abs(q).max() <= 127 and np.all(np.abs(q).max(axis=2) == 127)
+    with np.errstate(over="ignore"):
+        s_ref = (d * q.sum(axis=2).astype(np.float32)).astype(np.float16)
+    assert np.array_equal(s16, s_ref.view(np.uint16))
+    assert n_over == int(np.count_nonzero(np.isinf(s_ref) & np.isfinite(d.astype(np.float16))))
+    assert n_over > 0
+    err = np.abs(xb.astype(np.float64) - d[:, :, None].astype(np.float64) * q)
+    assert np.all(err <= 0.5001 * d[:, :, None])
+    # the same values quantized to Q8_K_128 stay finite
+    k_out, flags = orc.quantize_q8_k128(x)
+    kd, _, kbs = orc.decode_q8_k128(k_out, 16, 1024)
+    assert flags == 0 and np.isfinite(kd).all()
