@@ -49,7 +49,7 @@ typedef enum {
                        /* or a size whose byte count overflows int64              */
     IQQ_ERR_ALIGN = 3, /* a pointer lacks the alignment its argument states       */
     IQQ_ERR_CUDA = 4,  /* the kernel launch failed (see iqq_last_cuda_error)      */
-    IQQ_ERR_ARG = 5    /* an enumerated argument is out of range (weight_mode)    */
+    IQQ_ERR_ARG = 5    /* an enumerated argument is out of range (weight_mode 0..5) */
 } iqq_status;
 
 /* Device-side flag bits, ORed into *d_flags. */
@@ -83,7 +83,10 @@ typedef enum {
  *             (l[i]+8) | (l[i+16]+8) << 4 for i = 0..15.
  *  nrows, n_per_row   n_per_row % 32 == 0, both >= 0.
  *  rows_per_qw        >= 0; 0 = one imatrix row shared by all rows.
- *  weight_mode        0 = qw*sqrt(sigma2 + x^2), 1 = qw.
+ *  weight_mode        0 = qw*sqrt(sigma2 + x^2), 1 = qw, and the magnitude forms
+ *                     [W] §二 lists as tried before imatrix existed, times qw:
+ *                     2 = qw*x^2, 3 = qw*|x|, 4 = qw*(sigma2 + x^2),
+ *                     5 = qw*(sqrt(sigma2) + |x|)  (qw = NULL: the pure forms).
  *  d_flags    optional device uint32 (4-byte aligned) receiving IQQ_FLAG_*.
  *  stream     cudaStream_t.
  *
@@ -111,6 +114,27 @@ iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64
  */
 iqq_status iqq_quantize_q8_k128(const float* x, void* out, int64_t nrows, int64_t n_per_row,
                                 uint32_t* d_flags, void* stream);
+
+/*
+ * iqq_quantize_q8_1 -- Q8_1 activation quantization, the format [Q8]
+ * 修复前的数值隐患 describes and Q8_K_128 replaces: per 32 values a binary16
+ * d = amax/127 and a binary16 s = d*sum(q), int8 codes as for Q8_K_128
+ * (q = clamp(rint(x*id), -127, 127), id = amax > 0 ? 127/amax : 0).  s can
+ * overflow binary16 although d fits; the number of such blocks (stored s
+ * +-Inf, d finite) is added to *d_overflow.  Provided to measure that failure
+ * next to Q8_K_128.
+ *
+ *  x          [nrows, n_per_row] float32, 16-byte aligned.
+ *  out        nrows * n_per_row / 32 blocks of 36 bytes, 4-byte aligned:
+ *             half d | half s | int8 qs[32], little endian.
+ *  n_per_row  a multiple of 32.
+ *  d_overflow optional device uint64 (8-byte aligned); the count is ADDED.
+ *  d_flags    optional; receives IQQ_FLAG_NONFINITE_INPUT.
+ */
+#define IQQ_Q8_1_BLOCK_VALUES 32
+#define IQQ_Q8_1_BLOCK_BYTES 36
+iqq_status iqq_quantize_q8_1(const float* x, void* out, int64_t nrows, int64_t n_per_row,
+                             unsigned long long* d_overflow, uint32_t* d_flags, void* stream);
 
 /*
  * iqq_dequant_q4_0 -- y[r, 32b + i] = fp16(d) * (nibble_i - 8) for the Q4_0

@@ -39,12 +39,13 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m post_weight_quantization_rowwise_b200.build` (nvcc, sm_100a)")
+            "`python post_weight_quantization_rowwise_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     sigs = {
         "iqq_quantize_q4_0_w": [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_quantize_q8_k128": [_vp, _vp, _i64, _i64, _vp, _vp],
         "iqq_dequant_q4_0": [_vp, _vp, _i64, _i64, _vp],
+        "iqq_quantize_q8_1": [_vp, _vp, _i64, _i64, _vp, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -164,6 +165,23 @@ def iqq_quantize_q8_k128(x, out, flags=None, stream=None):
     return out
 
 
+def iqq_quantize_q8_1(x, out, overflow=None, flags=None, stream=None):
+    """Q8_1 blocks (36 bytes per 32 values) of x; adds the count of blocks whose fp16
+    sum overflowed to `overflow` (int64 CUDA tensor of one element) when given."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("overflow", overflow, torch.int64)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if out.numel() < nrows * (n // 32) * 36:
+        raise ValueError("out is too small")
+    _check("iqq_quantize_q8_1",
+           _lib.iqq_quantize_q8_1(_ptr(x), _ptr(out), nrows, n, _ptr(overflow), _ptr(flags),
+                                  _stream(stream)))
+    return out
+
+
 def iqq_dequant_q4_0(blocks, y, stream=None):
     """y [nrows, n_per_row] float32 from the Q4_0 blocks."""
     import torch
@@ -211,6 +229,13 @@ def quantize_q8_k128(x, flags=None, stream=None):
     out = torch.empty((nrows, (n // Q8_K128_BLOCK_VALUES) * Q8_K128_BLOCK_BYTES), dtype=torch.uint8,
                       device=x.device)
     return iqq_quantize_q8_k128(x, out, flags, stream)
+
+
+def quantize_q8_1(x, overflow=None, flags=None, stream=None):
+    import torch
+    nrows, n = _shape2(x)
+    out = torch.empty((nrows, (n // 32) * 36), dtype=torch.uint8, device=x.device)
+    return iqq_quantize_q8_1(x, out, overflow, flags, stream)
 
 
 def dequant_q4_0(blocks, nrows: int, n_per_row: int, stream=None):

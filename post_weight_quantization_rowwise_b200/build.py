@@ -1,6 +1,8 @@
 """Build libiqq.so (the C-ABI library, CUDA for sm_100a) in the package directory.
 
-    python -m post_weight_quantization_rowwise_b200.build [--force] [--verbose]
+    python post_weight_quantization_rowwise_b200/build.py [--force] [--verbose]
+
+(run as a script: importing the package itself needs the library this builds)
 
 nvcc cross-compiles for sm_100a without a GPU.  The kernels are compiled with
 -fmad=false (no contraction except explicit fmaf) and IEEE division and square

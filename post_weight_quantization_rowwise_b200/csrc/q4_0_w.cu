@@ -316,16 +316,28 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
             if (qmin < 0.0f) bad |= IQQ_FLAG_NEG_QW;
         }
 
-        // importance weights (binary32, one rounding per operation) -> shared memory,
-        // then xmax (signed value of the first element of largest |x|)
+        // importance weights (binary32, one rounding per operation) -> shared memory:
+        // mode 0 qw*sqrt(sigma2 + x*x), 1 qw, 2 qw*(x*x), 3 qw*|x|, 4 qw*(sigma2 + x*x),
+        // 5 qw*(sqrt(sigma2) + |x|); then xmax (signed value of the first largest |x|)
+        const float sigma = weight_mode == 5 ? __fsqrt_rn(sigma2) : 0.0f;
 #pragma unroll
         for (int i = 0; i < QK / 4; ++i) {
             float4 w4 = q4[i];
-            if (weight_mode == 0) {
-                w4.x = __fmul_rn(w4.x, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i], xv[4 * i]))));
-                w4.y = __fmul_rn(w4.y, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i + 1], xv[4 * i + 1]))));
-                w4.z = __fmul_rn(w4.z, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i + 2], xv[4 * i + 2]))));
-                w4.w = __fmul_rn(w4.w, __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xv[4 * i + 3], xv[4 * i + 3]))));
+            float* wp[4] = {&w4.x, &w4.y, &w4.z, &w4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float xj = xv[4 * i + k];
+                const float t = __fmul_rn(xj, xj);
+                float m;
+                switch (weight_mode) {
+                case 0: m = __fsqrt_rn(__fadd_rn(sigma2, t)); break;
+                case 2: m = t; break;
+                case 3: m = fabsf(xj); break;
+                case 4: m = __fadd_rn(sigma2, t); break;
+                case 5: m = __fadd_rn(sigma, fabsf(xj)); break;
+                default: m = 1.0f; break;
+                }
+                if (weight_mode != 1) *wp[k] = __fmul_rn(*wp[k], m);
             }
             *reinterpret_cast<float4*>(my_w + 4 * i) = w4;
         }
@@ -490,7 +502,7 @@ extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void*
 {
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
     if (n_per_row % QK != 0) return IQQ_ERR_SHAPE;
-    if (weight_mode != 0 && weight_mode != 1) return IQQ_ERR_ARG;
+    if (weight_mode < 0 || weight_mode > 5) return IQQ_ERR_ARG;
     if (nrows == 0 || n_per_row == 0) return IQQ_OK;
     if (x == nullptr || out == nullptr) return IQQ_ERR_NULL;
     if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||

@@ -25,7 +25,7 @@ def lib():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("iqq_quantize_q4_0_w", "iqq_quantize_q8_k128", "iqq_dequant_q4_0",
-              "iqq_weighted_rmse", "iqq_status_string"):
+              "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string"):
         assert n in names
 
 
@@ -62,10 +62,14 @@ def test_host_validation_without_gpu(lib):
     assert lib.iqq_quantize_q4_0_w(V(16), V(20), V(16), 4, 32, 0, 0, None, None) == 3
     assert lib.iqq_quantize_q4_0_w(V(16), None, V(17), 4, 32, 0, 0, None, None) == 3
     assert lib.iqq_quantize_q8_k128(V(16), V(18), 1, 128, None, None) == 3
+    assert lib.iqq_quantize_q8_1(V(16), V(16), 1, 48, None, None, None) == 2
+    assert lib.iqq_quantize_q8_1(None, V(16), 1, 32, None, None, None) == 1
+    assert lib.iqq_quantize_q8_1(V(16), V(16), 1, 32, V(12), None, None) == 3
     assert lib.iqq_dequant_q4_0(V(16), V(8), 1, 32, None) == 3
     assert lib.iqq_weighted_rmse(V(16), V(16), None, 1, 32, 0, V(4), None) == 3
     # enumerated argument
-    assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 4, 32, 0, 2, None, None) == 5
+    assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 4, 32, 0, 6, None, None) == 5
+    assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 4, 32, 0, -1, None, None) == 5
 
 
 def test_status_strings(lib):

@@ -55,6 +55,18 @@ def test_q4_0_single_matrix_1024x4096(iqq, synth, mode):
     compare_q4_0(x, qw, g, o, weight_mode=mode)
 
 
+@pytest.mark.parametrize("mode", [2, 3, 4, 5])
+def test_q4_0_magnitude_weight_forms(iqq, synth, mode):
+    """The importance forms x^2, |x|, sigma^2 + x^2, sigma + |x| (times qw, and alone)."""
+    x = synth.weight_matrix(96, 4096, seed=40 + mode).numpy()
+    qw = synth.imatrix(4096, seed=50 + mode).numpy()
+    for q in (qw, None):
+        g, gf = _gpu_q4_0(iqq, x, q, mode=mode)
+        o, of = oracle.quantize_q4_0_w(x, q, weight_mode=mode)
+        assert gf == of == 0
+        compare_q4_0(x, q, g, o, weight_mode=mode)
+
+
 @pytest.mark.parametrize("rows,n", [(37, 4192), (3, 32), (5, 11008), (9, 2048), (2, 7168), (1, 12320)])
 def test_q4_0_ragged_shapes(iqq, synth, rows, n):
     """Several 128-block chunks per row with a ragged last chunk, single-block rows."""
@@ -185,6 +197,33 @@ def test_q8_k128_shapes(iqq, rows, n):
     assert np.array_equal(g, o)
 
 
+# ------------------------------------------------------------------ Q8_1 (overflow contrast)
+
+def test_q8_1_bit_exact_and_overflow_count(iqq, synth):
+    """On the activation batch with spikes beyond fp16, Q8_1's fp16 sums overflow in
+    some blocks (counted identically on both sides) while Q8_K_128 stays finite."""
+    x = synth.activation_batch_4096x7168().numpy()
+    xd = torch.from_numpy(x).cuda()
+    cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = iqq.quantize_q8_1(xd, cnt, flags)
+    torch.cuda.synchronize()
+    o, n_over = oracle.quantize_q8_1(x)
+    assert np.array_equal(g.cpu().numpy(), o)
+    assert int(cnt.item()) == n_over > 0 and int(flags.item()) == 0
+    k = iqq.quantize_q8_k128(xd)
+    d, _, _ = oracle.decode_q8_k128(k.cpu().numpy(), 4096, 7168)
+    assert np.isfinite(d).all()
+
+
+@pytest.mark.parametrize("rows,n", [(1, 32), (3, 96), (5, 160), (7, 4096)])
+def test_q8_1_ragged_shapes(iqq, rows, n):
+    x = (np.random.default_rng(rows * n).standard_normal((rows, n)) * 5e3).astype(np.float32)
+    g = iqq.quantize_q8_1(torch.from_numpy(x).cuda()).cpu().numpy()
+    o, _ = oracle.quantize_q8_1(x)
+    assert np.array_equal(g, o)
+
+
 # ------------------------------------------------------------------ dequant, weighted RMSE
 
 def test_dequant_bit_exact(iqq, synth):
@@ -234,7 +273,7 @@ def test_abi_rejects_bad_arguments(iqq):
     with pytest.raises(iqq.IQQError, match="SHAPE"):
         iqq.quantize_q8_k128(torch.zeros(2, 96, device="cuda"))
     with pytest.raises(iqq.IQQError, match="ARG"):
-        iqq.quantize_q4_0_w(x, None, weight_mode=2)
+        iqq.quantize_q4_0_w(x, None, weight_mode=6)
     # empty input is a no-op
     iqq.quantize_q4_0_w(torch.zeros(0, 64, device="cuda"))
 
