@@ -56,6 +56,15 @@ def lib():
         L.oracle_fp16_from_float_array.argtypes = [_f32p, ctypes.POINTER(ctypes.c_uint16), _i64]
         L.oracle_fp16_to_float_array.restype = None
         L.oracle_fp16_to_float_array.argtypes = [ctypes.POINTER(ctypes.c_uint16), _f32p, _i64]
+        L.oracle_qx_block_search.restype = ctypes.c_float
+        L.oracle_qx_block_search.argtypes = [ctypes.c_int, ctypes.c_int, _f32p, _f32p, _i8p, _i8p, _i32p]
+        L.oracle_quantize_qx_0_w.restype = ctypes.c_int
+        L.oracle_quantize_qx_0_w.argtypes = [ctypes.c_int, _f32p, _f32p, _u8p, _i64, _i64, _i64,
+                                             ctypes.c_int, _u32p]
+        L.oracle_dequant_qx_0.restype = ctypes.c_int
+        L.oracle_dequant_qx_0.argtypes = [ctypes.c_int, _u8p, _f32p, _i64, _i64]
+        L.oracle_qx_block_bytes.restype = ctypes.c_int
+        L.oracle_qx_block_bytes.argtypes = [ctypes.c_int]
         L.oracle_quantize_q8_1.restype = ctypes.c_int64
         L.oracle_quantize_q8_1.argtypes = [_f32p, _u8p, _i64, _i64]
         L.oracle_quantize_q8_k128.restype = ctypes.c_int
@@ -124,6 +133,52 @@ def block_search(xb, w):
     d = lib().oracle_q4_0_block_search(n, _ptr(xb, _f32p), _ptr(w, _f32p), _ptr(L, _i8p),
                                        _ptr(Ls, _i8p), _ptr(info, _i32p))
     return np.float32(d), L, Ls, info
+
+
+NMAX = {4: 8, 5: 16, 6: 32, 8: 128}
+
+
+def qx_block_bytes(bits: int) -> int:
+    return int(lib().oracle_qx_block_bytes(bits))
+
+
+def qx_block_search(xb, w, nmax: int):
+    """Scale search of one block with codes in [-nmax, nmax-1]; as block_search."""
+    xb = _f32(xb)
+    w = _f32(w)
+    n = xb.size
+    L = np.zeros(n, np.int8)
+    Ls = np.zeros(n, np.int8)
+    info = np.zeros(4, np.int32)
+    d = lib().oracle_qx_block_search(n, nmax, _ptr(xb, _f32p), _ptr(w, _f32p), _ptr(L, _i8p),
+                                     _ptr(Ls, _i8p), _ptr(info, _i32p))
+    return np.float32(d), L, Ls, info
+
+
+def quantize_qx_0_w(bits: int, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0):
+    """Weighted quantization to the 32-value format with `bits` (4, 5, 6, 8); (blocks, flags)."""
+    x = _f32(x)
+    nrows, n = x.shape
+    qw = None if qw is None else _f32(qw)
+    bb = qx_block_bytes(bits)
+    if bb < 0:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    out = np.zeros((nrows, (n // 32) * bb), np.uint8)
+    flags = np.zeros(1, np.uint32)
+    rc = lib().oracle_quantize_qx_0_w(bits, _ptr(x, _f32p), _ptr(qw, _f32p), _ptr(out, _u8p), nrows, n,
+                                      rows_per_qw, weight_mode, _ptr(flags, _u32p))
+    if rc != 0:
+        raise ValueError("oracle_quantize_qx_0_w: bad arguments")
+    return out, int(flags[0])
+
+
+def dequant_qx_0(bits: int, blocks, nrows: int, n_per_row: int):
+    blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
+    y = np.empty((nrows, n_per_row), np.float32)
+    rc = lib().oracle_dequant_qx_0(bits, _ptr(blocks, _u8p), _ptr(y, _f32p), nrows, n_per_row)
+    if rc != 0:
+        raise ValueError("oracle_dequant_qx_0: bad arguments")
+    return y
 
 
 def quantize_q4_0_w(x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0,

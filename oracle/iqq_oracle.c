@@ -186,12 +186,13 @@ void oracle_block_weights(const float *xb, const float *qwb, int n, float sigma2
 /* Returns d (binary32).  n is 32 for Q4_0; small n serves the toy     */
 /* brute-force checks.                                                 */
 /* ------------------------------------------------------------------ */
-static void candidate_codes(int n, const float *xb, float iscale, float *l)
+static void candidate_codes(int n, int nmax, const float *xb, float iscale, float *l)
 {
+    const float lo = (float)(-nmax), hi = (float)(nmax - 1);
     for (int j = 0; j < n; ++j) {
         float v = iscale * xb[j];
         float r = rintf(v);
-        l[j] = fminf(fmaxf(r, -8.0f), 7.0f);
+        l[j] = fminf(fmaxf(r, lo), hi);
     }
 }
 
@@ -207,11 +208,18 @@ static void block_sums(int n, const float *wx, const float *w, const float *l,
     *suml2 = b;
 }
 
-float oracle_q4_0_block_search(int n, const float *xb, const float *w, int8_t *L,
-                               int8_t *L_sweep, int32_t *info)
+/* The same search for the other 32-value formats of the family (Q5_0, Q6_0,
+ * Q8_0, [W] §一: "the same formula appears in quantize_row_q5_0_impl ..."):
+ * nmax = 16, 32, 128 with codes in [-nmax, nmax-1].  Reading: the candidates
+ * scale with nmax, c_k = (float)(nmax*(80+k)) / 80.0f (for nmax = 8 exactly
+ * the Q4_0 set (80+k)/10); every other step is unchanged. */
+float oracle_qx_block_search(int n, int nmax, const float *xb, const float *w, int8_t *L,
+                             int8_t *L_sweep, int32_t *info)
 {
     float wx[64], l[64], lbest[64];
     if (n <= 0 || n > 64) return NAN;
+    if (nmax != 8 && nmax != 16 && nmax != 32 && nmax != 128) return NAN;
+    const float lo = (float)(-nmax), hi = (float)(nmax - 1);
     if (info) { info[0] = 0; info[1] = 0; info[2] = 0; info[3] = 0; }
 
     float amax = 0.0f, xmax = 0.0f;
@@ -228,9 +236,9 @@ float oracle_q4_0_block_search(int n, const float *xb, const float *w, int8_t *L
     float best = -INFINITY;
     int kbest = 0;
     for (int k = -9; k <= 9; ++k) {
-        float c = (float)(80 + k) / 10.0f;
+        float c = (float)(nmax * (80 + k)) / 80.0f;
         float iscale = -c / xmax;
-        candidate_codes(n, xb, iscale, l);
+        candidate_codes(n, nmax, xb, iscale, l);
         float sumlx, suml2;
         block_sums(n, wx, w, l, &sumlx, &suml2);
         float score = suml2 > 0.0f ? (sumlx * sumlx) / suml2 : -INFINITY;
@@ -243,8 +251,8 @@ float oracle_q4_0_block_search(int n, const float *xb, const float *w, int8_t *L
 
     if (best == -INFINITY) {
         /* no candidate has a positive weighted code energy */
-        float iscale0 = -8.0f / xmax;
-        candidate_codes(n, xb, iscale0, l);
+        float iscale0 = -(float)nmax / xmax;
+        candidate_codes(n, nmax, xb, iscale0, l);
         for (int j = 0; j < n; ++j) {
             L[j] = (int8_t)l[j];
             if (L_sweep) L_sweep[j] = (int8_t)l[j];
@@ -267,7 +275,7 @@ float oracle_q4_0_block_search(int n, const float *xb, const float *w, int8_t *L
             if (g == 0.0f || g != g) continue;
             float s = g > 0.0f ? 1.0f : -1.0f;
             float ln = lbest[j] + s;
-            if (ln < -8.0f || ln > 7.0f) continue;
+            if (ln < lo || ln > hi) continue;
             float nlx = sumlx + s * wx[j];
             float nl2 = fmaf(w[j], 2.0f * s * lbest[j] + 1.0f, suml2);
             if (!(nl2 > 0.0f)) continue;
@@ -286,6 +294,12 @@ float oracle_q4_0_block_search(int n, const float *xb, const float *w, int8_t *L
     for (int j = 0; j < n; ++j) L[j] = (int8_t)lbest[j];
     if (info) { info[0] = kbest; info[1] = passes; info[2] = 0; }
     return sumlx / suml2;
+}
+
+float oracle_q4_0_block_search(int n, const float *xb, const float *w, int8_t *L,
+                               int8_t *L_sweep, int32_t *info)
+{
+    return oracle_qx_block_search(n, 8, xb, w, L, L_sweep, info);
 }
 
 /* ------------------------------------------------------------------ */
@@ -339,6 +353,118 @@ int oracle_quantize_q4_0_w(const float *x, const float *qw, uint8_t *out, int64_
             pack_q4_0(d, L, out + (r * nb + b) * ORACLE_Q4_0_BYTES, flags);
             if (passes) passes[r * nb + b] = info[1];
         }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* The other 32-value formats (reading; the pages name the types, not  */
+/* their bytes).  n = l + nmax is the biased code.                     */
+/*   bits 5 (Q5_0, 22 B): d16 | qh (u32 LE, bit j = (n_j >> 4) & 1)    */
+/*                        | qs[16], qs[i] = (n_i & 15) | (n_{i+16} & 15) << 4 */
+/*   bits 6 (Q6_0, 26 B): d16 | qh (u64 LE, bits 2j..2j+1 = n_j >> 4)  */
+/*                        | qs[16] as for Q5_0                          */
+/*   bits 8 (Q8_0, 34 B): d16 | int8 qs[32] = l_j                       */
+/*   bits 4 (Q4_0, 18 B): as above                                      */
+/* ------------------------------------------------------------------ */
+int oracle_qx_block_bytes(int bits)
+{
+    switch (bits) {
+    case 4: return 18;
+    case 5: return 22;
+    case 6: return 26;
+    case 8: return 34;
+    default: return -1;
+    }
+}
+
+static int nmax_of(int bits) { return bits == 8 ? 128 : 1 << (bits - 1); }
+
+static void pack_qx(int bits, float d, const int8_t *L, uint8_t *blk, uint32_t *flags)
+{
+    if (bits == 4) { pack_q4_0(d, L, blk, flags); return; }
+    uint16_t h = oracle_fp16_from_float(d);
+    if ((h & 0x7fffu) == 0x7c00u && isfinite(d) && flags) *flags |= FLAG_SCALE_OVERFLOW;
+    blk[0] = (uint8_t)(h & 0xff);
+    blk[1] = (uint8_t)(h >> 8);
+    if (bits == 8) {
+        for (int j = 0; j < 32; ++j) blk[2 + j] = (uint8_t)L[j];
+        return;
+    }
+    const int nmax = nmax_of(bits);
+    const int hb = bits == 5 ? 4 : 8;          /* bytes of high bits */
+    uint64_t qh = 0;
+    for (int j = 0; j < 32; ++j) {
+        unsigned n = (unsigned)(L[j] + nmax);
+        if (bits == 5) qh |= (uint64_t)((n >> 4) & 1u) << j;
+        else qh |= (uint64_t)((n >> 4) & 3u) << (2 * j);
+    }
+    for (int b = 0; b < hb; ++b) blk[2 + b] = (uint8_t)(qh >> (8 * b));
+    for (int i = 0; i < 16; ++i) {
+        unsigned lo = (unsigned)(L[i] + nmax) & 15u, hi = (unsigned)(L[i + 16] + nmax) & 15u;
+        blk[2 + hb + i] = (uint8_t)(lo | (hi << 4));
+    }
+}
+
+static int unpack_code(int bits, const uint8_t *blk, int j)
+{
+    if (bits == 8) return (int8_t)blk[2 + j];
+    const int nmax = nmax_of(bits);
+    if (bits == 4) {
+        int nib = j < 16 ? (blk[2 + j] & 0xf) : (blk[2 + j - 16] >> 4);
+        return nib - nmax;
+    }
+    const int hb = bits == 5 ? 4 : 8;
+    uint64_t qh = 0;
+    for (int b = 0; b < hb; ++b) qh |= (uint64_t)blk[2 + b] << (8 * b);
+    int low = j < 16 ? (blk[2 + hb + j] & 0xf) : (blk[2 + hb + j - 16] >> 4);
+    int high = bits == 5 ? (int)((qh >> j) & 1u) : (int)((qh >> (2 * j)) & 3u);
+    return (low | (high << 4)) - nmax;
+}
+
+/* Weighted quantization of a tensor to any of the 32-value formats. */
+int oracle_quantize_qx_0_w(int bits, const float *x, const float *qw, uint8_t *out, int64_t nrows,
+                           int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                           uint32_t *flags)
+{
+    const int bb = oracle_qx_block_bytes(bits);
+    if (bb < 0 || n_per_row % 32 != 0 || nrows < 0 || n_per_row < 0) return -1;
+    if (weight_mode < 0 || weight_mode > 5) return -1;
+    const int nmax = nmax_of(bits);
+    const int64_t nb = n_per_row / 32;
+    float w[32];
+    int8_t L[32];
+    for (int64_t r = 0; r < nrows; ++r) {
+        const float *xr = x + r * n_per_row;
+        const float *qr = qw ? qw + (rows_per_qw > 0 ? r / rows_per_qw : 0) * n_per_row : NULL;
+        if (flags) {
+            for (int64_t j = 0; j < n_per_row; ++j) {
+                if (!isfinite(xr[j])) *flags |= FLAG_NONFINITE;
+                if (qr && !isfinite(qr[j])) *flags |= FLAG_NONFINITE;
+                if (qr && qr[j] < 0.0f) *flags |= FLAG_NEG_QW;
+            }
+        }
+        float sigma2 = oracle_row_sigma2(xr, n_per_row);
+        for (int64_t b = 0; b < nb; ++b) {
+            const float *xb = xr + b * 32;
+            oracle_block_weights(xb, qr ? qr + b * 32 : NULL, 32, sigma2, weight_mode, w);
+            float d = oracle_qx_block_search(32, nmax, xb, w, L, NULL, NULL);
+            pack_qx(bits, d, L, out + (r * nb + b) * bb, flags);
+        }
+    }
+    return 0;
+}
+
+/* y = fp16_to_float(d) * l for any of the 32-value formats (exact in binary32). */
+int oracle_dequant_qx_0(int bits, const uint8_t *blocks, float *y, int64_t nrows, int64_t n_per_row)
+{
+    const int bb = oracle_qx_block_bytes(bits);
+    if (bb < 0 || n_per_row % 32 != 0) return -1;
+    const int64_t nblk = nrows * (n_per_row / 32);
+    for (int64_t g = 0; g < nblk; ++g) {
+        const uint8_t *blk = blocks + g * bb;
+        float d = oracle_fp16_to_float((uint16_t)(blk[0] | (blk[1] << 8)));
+        for (int j = 0; j < 32; ++j) y[g * 32 + j] = d * (float)unpack_code(bits, blk, j);
     }
     return 0;
 }

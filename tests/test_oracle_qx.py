@@ -1,0 +1,156 @@
+"""Pins of the oracle's weighted Q5_0 / Q6_0 / Q8_0 quantizers: the same search as
+Q4_0 with nmax = 16, 32, 128 and codes in [-nmax, nmax-1].
+
+[W] = "ik_llama.cpp 量化权重之谜：weight[j] = qw[j] * sqrtf(sigma2 + xb[j]*xb[j])的由来与原理"
+      (www.dpshk.com/news/4810665), §一: the same weighting appears in
+      quantize_row_q5_0_impl, quantize_row_q6_0_impl, ... (and make_qx_quants takes nmax).
+Byte layouts (reading; the pages do not print them), biased code n = l + nmax:
+  Q5_0 22 B: d16 | qh u32 (bit j = n_j >> 4 & 1) | qs[16] (low nibbles, j and j+16 paired)
+  Q6_0 26 B: d16 | qh u64 (bits 2j, 2j+1 = n_j >> 4) | qs[16]
+  Q8_0 34 B: d16 | int8 l[32]
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+BITS = (5, 6, 8)
+
+
+def _pack(bits, d, codes, orc):
+    nmax = orc.NMAX[bits]
+    h = int(np.float16(d).view(np.uint16))
+    head = [h & 0xFF, h >> 8]
+    if bits == 8:
+        return bytes(head + [c & 0xFF for c in codes])
+    n = [c + nmax for c in codes]
+    if bits == 5:
+        qh = sum(((v >> 4) & 1) << j for j, v in enumerate(n))
+        hb = qh.to_bytes(4, "little")
+    else:
+        qh = sum(((v >> 4) & 3) << (2 * j) for j, v in enumerate(n))
+        hb = qh.to_bytes(8, "little")
+    qs = [(n[i] & 15) | ((n[i + 16] & 15) << 4) for i in range(16)]
+    return bytes(head) + hb + bytes(qs)
+
+
+def _err(x, w, l):
+    x, w, l = (a.astype(np.float64) for a in (x, w, l))
+    b = np.sum(w * l * l)
+    d = np.sum(w * x * l) / b
+    return float(np.sum(w * (x - d * l) ** 2))
+
+
+def test_block_sizes(orc):
+    assert [orc.qx_block_bytes(b) for b in (4, 5, 6, 8)] == [18, 22, 26, 34]
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_exact_blocks_and_layout(orc, bits):
+    """x = d0 * n with integer codes n spanning [-nmax, nmax-1], the extreme -nmax
+    unique: the search returns codes n and d0 exactly (weights 1), and the bytes follow
+    the layout reading."""
+    nmax = orc.NMAX[bits]
+    rng = np.random.default_rng(bits)
+    for d0 in (2.0 ** -7, -0.25, 3.0):
+        codes = rng.integers(-nmax + 1, nmax, 32)
+        codes[5] = -nmax
+        codes[9] = 1                        # no common factor
+        x = (np.float32(d0) * codes.astype(np.float32)).reshape(1, 32)
+        out, flags = orc.quantize_qx_0_w(bits, x, np.ones(32, np.float32), weight_mode=1)
+        assert flags == 0
+        assert bytes(out[0]) == _pack(bits, d0, codes.tolist(), orc)
+        y = orc.dequant_qx_0(bits, out, 1, 32)
+        assert np.array_equal(y, x)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_dequant_is_the_exact_product(orc, bits):
+    nmax = orc.NMAX[bits]
+    rng = np.random.default_rng(10 + bits)
+    blocks, expect = [], []
+    for _ in range(200):
+        h = np.uint16(rng.integers(0, 0x7C00)) | np.uint16(rng.integers(0, 2) << 15)
+        d = h.view(np.float16)
+        codes = rng.integers(-nmax, nmax, 32)
+        blocks.append(np.frombuffer(_pack(bits, d, codes.tolist(), orc), np.uint8))
+        expect.append(np.float64(d) * codes)
+    y = orc.dequant_qx_0(bits, np.stack(blocks), 200, 32)
+    assert np.array_equal(y.astype(np.float64), np.stack(expect))
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_symmetries(orc, bits):
+    rng = np.random.default_rng(20 + bits)
+    x = (rng.standard_normal((16, 256)) * 0.02).astype(np.float32)
+    qw = np.exp(rng.standard_normal(256)).astype(np.float32)
+    a, _ = orc.quantize_qx_0_w(bits, x, qw)
+    b, _ = orc.quantize_qx_0_w(bits, -x, qw)
+    c, _ = orc.quantize_qx_0_w(bits, x * np.float32(8.0), qw)
+    ya, yb, yc = (orc.dequant_qx_0(bits, t, 16, 256) for t in (a, b, c))
+    assert np.array_equal(ya, -yb)
+    assert np.array_equal(ya * np.float32(8.0), yc)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_search_never_worse_than_candidates_and_locally_optimal(orc, bits):
+    """As for Q4_0: the result is at least as good as every candidate's rounding and no
+    single +-1 move improves it beyond the binary32 resolution of the score."""
+    nmax = orc.NMAX[bits]
+    rng = np.random.default_rng(30 + bits)
+    u = 2.0 ** -24
+    for _ in range(300):
+        x = (rng.standard_normal(32) * 0.02).astype(np.float32)
+        w = np.exp(rng.standard_normal(32)).astype(np.float32)
+        d, L, Ls, info = orc.qx_block_search(x, w, nmax)
+        energy = float(np.sum(w.astype(np.float64) * x.astype(np.float64) ** 2))
+        tol = (18 * 32 + 2) * u * energy
+        ef = _err(x, w, L)
+        xmax = x[int(np.argmax(np.abs(x)))]
+        for k in range(-9, 10):
+            c = np.float32(nmax * (80 + k)) / np.float32(80.0)
+            iscale = np.float32(-c) / xmax
+            cand = np.clip(np.rint(np.float32(iscale) * x), -nmax, nmax - 1)
+            assert ef <= _err(x, w, cand) + tol
+        if info[1] < 5:
+            for j in range(32):
+                for s in (-1, 1):
+                    if -nmax <= L[j] + s <= nmax - 1:
+                        M = L.copy()
+                        M[j] += s
+                        assert _err(x, w, M) >= ef - tol
+
+
+def test_brute_force_three_values_q5(orc):
+    """3-value toy blocks with nmax = 16: every one of the 32^3 code vectors bounds
+    the search from below."""
+    rng = np.random.default_rng(40)
+    codes = np.array(list(itertools.product(range(-16, 16), repeat=3)), np.float64)
+    hits = 0
+    for _ in range(200):
+        x = rng.standard_normal(3).astype(np.float32)
+        w = np.exp(rng.standard_normal(3)).astype(np.float32)
+        d, L, Ls, info = orc.qx_block_search(x, w, 16)
+        xd, wd = x.astype(np.float64), w.astype(np.float64)
+        A = codes @ (wd * xd)
+        B = (codes * codes) @ wd
+        ok = B > 0
+        E = np.full(len(codes), np.sum(wd * xd * xd))
+        E[ok] -= A[ok] ** 2 / B[ok]
+        eg = max(float(E.min()), 0.0)
+        eo = _err(x, w, L)
+        assert eg <= eo * (1 + 1e-9) + 1e-12
+        hits += eo - eg <= 1e-9 * max(eo, 1e-30)
+    assert hits > 100
+
+
+def test_more_bits_less_error(orc):
+    rng = np.random.default_rng(50)
+    x = (rng.standard_normal((32, 512)) * 0.02).astype(np.float32)
+    qw = np.exp(rng.standard_normal(512)).astype(np.float32)
+    errs = []
+    for bits in (4, 5, 6, 8):
+        out, _ = orc.quantize_qx_0_w(bits, x, qw)
+        y = orc.dequant_qx_0(bits, out, 32, 512)
+        errs.append(float(np.sum(qw * (x - y).astype(np.float64) ** 2)))
+    assert errs[0] > errs[1] > errs[2] > errs[3]
