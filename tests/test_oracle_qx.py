@@ -103,6 +103,7 @@ def test_search_never_worse_than_candidates_and_locally_optimal(orc, bits):
         x = (rng.standard_normal(32) * 0.02).astype(np.float32)
         w = np.exp(rng.standard_normal(32)).astype(np.float32)
         d, L, Ls, info = orc.qx_block_search(x, w, nmax)
+        L = L.astype(np.int64)                      # int8 codes would wrap at +-128
         energy = float(np.sum(w.astype(np.float64) * x.astype(np.float64) ** 2))
         tol = (18 * 32 + 2) * u * energy
         ef = _err(x, w, L)
