@@ -44,10 +44,10 @@ DEQ_BYTES_PER_VALUE = 18.0 / 32.0 + 4.0
 RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
-# DRAM bytes (read + write) per value of q4_0_w_kernel from one ncu capture of the current
-# kernel (4096x4096 launch: 67.18 MB read + 2.87 MB written for 16,777,216 values); set
+# DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
+# kernel (4096x4096 launch: 67.187 MB read + 2.091 MB written for 16,777,216 values); set
 # to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = None
+Q4_0_DRAM_BYTES_PER_VALUE = 4.1293
 
 
 def peaks():
@@ -369,7 +369,7 @@ def main_ours(args):
         "config": {"workload": WORKLOAD, "layers": args.layers, "tensors": n_q4,
                    "q4_0_values": w.q4_elems, "q8_k128_values": w.q8_elems,
                    "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (replicas)"},
-        "roofline": {"bound": "alu", "kernel": "q4_0_w_kernel", "achieved": round(achieved, 3),
+        "roofline": {"bound": "alu", "kernel": "qx_0_w_kernel<4>", "achieved": round(achieved, 3),
                      "peak": round(peak_ops, 3), "unit": "Tops/s",
                      "frac": round(achieved / peak_ops, 4),
                      "traffic": (None if Q4_0_DRAM_BYTES_PER_VALUE is None else

@@ -99,6 +99,26 @@ iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64
                                uint32_t* d_flags, void* stream);
 
 /*
+ * iqq_quantize_qx_0_w -- the same weighted search for the other 32-value formats
+ * of the family ([W] §一: the weighting appears in quantize_row_q5_0_impl,
+ * quantize_row_q6_0_impl, ...): bits = 4 (Q4_0, exactly iqq_quantize_q4_0_w),
+ * 5 (Q5_0), 6 (Q6_0) or 8 (Q8_0); nmax = 8, 16, 32, 128, codes in
+ * [-nmax, nmax-1], candidates iscale = -c_k/xmax with c_k = (float)(nmax*(80+k))/80.
+ * Other arguments as for iqq_quantize_q4_0_w; out holds 18/22/26/34-byte blocks
+ * (2-byte aligned).  With n = l + nmax the biased code:
+ *   Q5_0 (22 B): d16 | qh u32 LE, bit j = (n_j >> 4) & 1 | qs[16], qs[i] = (n_i & 15) | (n_{i+16} & 15) << 4
+ *   Q6_0 (26 B): d16 | qh u64 LE, bits 2j..2j+1 = n_j >> 4 | qs[16] as for Q5_0
+ *   Q8_0 (34 B): d16 | int8 l[32]
+ * bits outside {4, 5, 6, 8} return IQQ_ERR_ARG.
+ */
+#define IQQ_Q5_0_BLOCK_BYTES 22
+#define IQQ_Q6_0_BLOCK_BYTES 26
+#define IQQ_Q8_0_BLOCK_BYTES 34
+iqq_status iqq_quantize_qx_0_w(int bits, const float* x, const float* qw, void* out, int64_t nrows,
+                               int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                               uint32_t* d_flags, void* stream);
+
+/*
  * iqq_quantize_q8_k128 -- Q8_K_128 activation quantization, [Q8] 修复方案:
  * 128-value blocks with a binary32 scale, int8 codes and one int16 sum of the
  * codes per 32 values that is not multiplied by d, so no fp16 quantity can
@@ -145,6 +165,14 @@ iqq_status iqq_quantize_q8_1(const float* x, void* out, int64_t nrows, int64_t n
  *  y          [nrows, n_per_row] float32 output, 16-byte aligned.
  */
 iqq_status iqq_dequant_q4_0(const void* blocks, float* y, int64_t nrows, int64_t n_per_row,
+                            void* stream);
+
+/*
+ * iqq_dequant_qx_0 -- y = fp16(d) * l for blocks written by iqq_quantize_qx_0_w with
+ * the same bits (4, 5, 6, 8); exact in binary32.  blocks 2-byte aligned, y 16-byte
+ * aligned.
+ */
+iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, int64_t nrows, int64_t n_per_row,
                             void* stream);
 
 /*

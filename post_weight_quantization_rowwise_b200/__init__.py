@@ -46,6 +46,8 @@ def _load():
         "iqq_quantize_q8_k128": [_vp, _vp, _i64, _i64, _vp, _vp],
         "iqq_dequant_q4_0": [_vp, _vp, _i64, _i64, _vp],
         "iqq_quantize_q8_1": [_vp, _vp, _i64, _i64, _vp, _vp, _vp],
+        "iqq_quantize_qx_0_w": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
+        "iqq_dequant_qx_0": [ctypes.c_int, _vp, _vp, _i64, _i64, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -151,6 +153,41 @@ def iqq_quantize_q4_0_w(x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, 
     return out
 
 
+QX_0_BLOCK_BYTES = {4: 18, 5: 22, 6: 26, 8: 34}
+
+
+def iqq_quantize_qx_0_w(bits, x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,
+                        stream=None):
+    """Weighted Q4_0/Q5_0/Q6_0/Q8_0 (bits 4/5/6/8) blocks of x into out (uint8)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
+        raise ValueError("out is too small")
+    _check("iqq_quantize_qx_0_w",
+           _lib.iqq_quantize_qx_0_w(bits, _ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw,
+                                    weight_mode, _ptr(flags), _stream(stream)))
+    return out
+
+
+def iqq_dequant_qx_0(bits, blocks, y, stream=None):
+    import torch
+    _need_cuda("blocks", blocks, torch.uint8)
+    _need_cuda("y", y, torch.float32)
+    nrows, n = _shape2(y)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
+        raise ValueError("blocks is too small")
+    _check("iqq_dequant_qx_0", _lib.iqq_dequant_qx_0(bits, _ptr(blocks), _ptr(y), nrows, n, _stream(stream)))
+    return y
+
+
 def iqq_quantize_q8_k128(x, out, flags=None, stream=None):
     """Q8_K_128 blocks of x [nrows, n_per_row] float32 into out (uint8, q8_k128_nbytes)."""
     import torch
@@ -229,6 +266,20 @@ def quantize_q8_k128(x, flags=None, stream=None):
     out = torch.empty((nrows, (n // Q8_K128_BLOCK_VALUES) * Q8_K128_BLOCK_BYTES), dtype=torch.uint8,
                       device=x.device)
     return iqq_quantize_q8_k128(x, out, flags, stream)
+
+
+def quantize_qx_0_w(bits, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,
+                    stream=None):
+    import torch
+    nrows, n = _shape2(x)
+    out = torch.empty((nrows, (n // 32) * QX_0_BLOCK_BYTES[bits]), dtype=torch.uint8, device=x.device)
+    return iqq_quantize_qx_0_w(bits, x, qw, out, rows_per_qw, weight_mode, flags, stream)
+
+
+def dequant_qx_0(bits, blocks, nrows: int, n_per_row: int, stream=None):
+    import torch
+    y = torch.empty((nrows, n_per_row), dtype=torch.float32, device=blocks.device)
+    return iqq_dequant_qx_0(bits, blocks, y, stream)
 
 
 def quantize_q8_1(x, overflow=None, flags=None, stream=None):

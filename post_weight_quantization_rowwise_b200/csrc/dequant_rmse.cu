@@ -189,6 +189,59 @@ weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ bl
     }
 }
 
+// Q5_0 / Q6_0 / Q8_0 (layouts in iqq.h): the four codes of quad qd (values 4qd..4qd+3).
+template <int BITS>
+__device__ __forceinline__ void load_quad_qx(const uint8_t* blk, int qd, float& d, int (&c)[4])
+{
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(blk);
+    d = __half2float(__ushort_as_half(__ldg(h)));
+    if (BITS == 8) {
+        const uint32_t b = static_cast<uint32_t>(__ldg(h + 1 + 2 * qd)) |
+                           (static_cast<uint32_t>(__ldg(h + 2 + 2 * qd)) << 16);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) c[k] = static_cast<int>(static_cast<int8_t>((b >> (8 * k)) & 0xffu));
+        return;
+    }
+    constexpr int nmax = BITS == 5 ? 16 : 32;
+    constexpr int hw = BITS == 5 ? 2 : 4;  // 16-bit words of high bits
+    const int m = qd & 3;
+    const uint32_t lo4 = static_cast<uint32_t>(__ldg(h + 1 + hw + 2 * m)) |
+                         (static_cast<uint32_t>(__ldg(h + 2 + hw + 2 * m)) << 16);
+    const uint32_t sel = qd < 4 ? lo4 : (lo4 >> 4);
+    uint32_t hi;
+    if (BITS == 5) {
+        const uint32_t qh = static_cast<uint32_t>(__ldg(h + 1)) | (static_cast<uint32_t>(__ldg(h + 2)) << 16);
+        hi = qh >> (4 * qd);  // bit k = high bit of value 4qd + k
+    } else {
+        hi = static_cast<uint32_t>(__ldg(h + 1 + (qd >> 1))) >> (8 * (qd & 1));  // 2 bits per value
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t low = (sel >> (8 * k)) & 0xfu;
+        const uint32_t high = BITS == 5 ? ((hi >> k) & 1u) : ((hi >> (2 * k)) & 3u);
+        c[k] = static_cast<int>(low | (high << 4)) - nmax;
+    }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads)
+dequant_qx_kernel(const uint8_t* __restrict__ blocks, float4* __restrict__ y, int64_t nquads)
+{
+    constexpr int kBytes = BITS == 5 ? 22 : (BITS == 6 ? 26 : 34);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; t < nquads; t += stride) {
+        float d;
+        int c[4];
+        load_quad_qx<BITS>(blocks + (t >> 3) * kBytes, static_cast<int>(t & 7), d, c);
+        float4 o;
+        o.x = __fmul_rn(d, static_cast<float>(c[0]));
+        o.y = __fmul_rn(d, static_cast<float>(c[1]));
+        o.z = __fmul_rn(d, static_cast<float>(c[2]));
+        o.w = __fmul_rn(d, static_cast<float>(c[3]));
+        __stcs(y + t, o);
+    }
+}
+
 int sm_count()
 {
     int dev = 0, sms = 148;
@@ -212,6 +265,29 @@ extern "C" iqq_status iqq_dequant_q4_0(const void* blocks, float* y, int64_t nro
     const int grid = static_cast<int>(need < cap ? need : cap);
     dequant_q4_0_kernel<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint8_t*>(blocks), reinterpret_cast<float4*>(y), nquads);
+    return iqq::launch_status();
+}
+
+extern "C" iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, int64_t nrows,
+                                       int64_t n_per_row, void* stream)
+{
+    if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
+    if (bits == 4) return iqq_dequant_q4_0(blocks, y, nrows, n_per_row, stream);
+    if (!iqq::size_ok(nrows, n_per_row, 4)) return IQQ_ERR_SHAPE;
+    if (n_per_row % IQQ_Q4_0_BLOCK_VALUES != 0) return IQQ_ERR_SHAPE;
+    if (nrows == 0 || n_per_row == 0) return IQQ_OK;
+    if (blocks == nullptr || y == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(blocks, 2) || !iqq::aligned(y, 16)) return IQQ_ERR_ALIGN;
+    const int64_t nquads = nrows * n_per_row / 4;
+    const int64_t need = (nquads + kThreads - 1) / kThreads;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * IQQ_DQ_CTAS;
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    const uint8_t* bl = static_cast<const uint8_t*>(blocks);
+    float4* yy = reinterpret_cast<float4*>(y);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (bits == 5) dequant_qx_kernel<5><<<grid, kThreads, 0, st>>>(bl, yy, nquads);
+    else if (bits == 6) dequant_qx_kernel<6><<<grid, kThreads, 0, st>>>(bl, yy, nquads);
+    else dequant_qx_kernel<8><<<grid, kThreads, 0, st>>>(bl, yy, nquads);
     return iqq::launch_status();
 }
 

@@ -1,4 +1,4 @@
-// q4_0_w.cu -- imatrix-weighted Q4_0 quantization on sm_100a.
+// qx_0_w.cu -- imatrix-weighted Q4_0 (and Q5_0, Q6_0, Q8_0) quantization on sm_100a.
 //
 // Page "ik_llama.cpp 量化权重之谜：weight[j] = qw[j] * sqrtf(sigma2 +
 // xb[j]*xb[j])的由来与原理" (www.dpshk.com/news/4810665), §一: per row
@@ -14,6 +14,10 @@
 //   <= 5 Gauss-Seidel passes, a +-1 move accepted iff the score rises;
 //   final sums recomputed, d = sumlx/suml2 -> binary16 (RNE);
 //   block = d16 (LE) | qs[i] = (l[i]+8) | (l[i+16]+8) << 4.
+// The same search serves the family's other 32-value formats (§一 names
+// quantize_row_q5_0_impl, ..._q6_0_impl): nmax = 16, 32, 128, codes in
+// [-nmax, nmax-1], candidates c_k = (float)(nmax*(80+k))/80 (the Q4_0 set for
+// nmax = 8); the kernel is a template on the bit width.
 //
 // The work is ALU bound (about 150 binary32 operations per value against
 // 4.6 bytes of HBM traffic), so the design is about instruction count and
@@ -78,17 +82,32 @@ static_assert(kScratch + 2 * 32 * kRow1 <= kWarpFloats, "staging fits in the swe
 #define IQQ_Q4_MIN_CTAS 4  // resident CTAs per SM the register budget is sized for
 #endif
 
-// c_k = (float)(80 + k) / 10 for k = -9..9, each the IEEE quotient.
-__constant__ float c_cand[kCand] = {
-    71.0f / 10.0f, 72.0f / 10.0f, 73.0f / 10.0f, 74.0f / 10.0f, 75.0f / 10.0f,
-    76.0f / 10.0f, 77.0f / 10.0f, 78.0f / 10.0f, 79.0f / 10.0f, 80.0f / 10.0f,
-    81.0f / 10.0f, 82.0f / 10.0f, 83.0f / 10.0f, 84.0f / 10.0f, 85.0f / 10.0f,
-    86.0f / 10.0f, 87.0f / 10.0f, 88.0f / 10.0f, 89.0f / 10.0f};
+// Formats: bits -> nmax (codes in [-nmax, nmax-1]) and block bytes.
+template <int BITS> struct Fmt;
+template <> struct Fmt<4> { static constexpr int nmax = 8, bytes = 18, fi = 0; };
+template <> struct Fmt<5> { static constexpr int nmax = 16, bytes = 22, fi = 1; };
+template <> struct Fmt<6> { static constexpr int nmax = 32, bytes = 26, fi = 2; };
+template <> struct Fmt<8> { static constexpr int nmax = 128, bytes = 34, fi = 3; };
+
+// c_k = (float)(nmax * (80 + k)) / 80 for k = -9..9, each the IEEE quotient (for
+// nmax = 8 these are (80 + k)/10).
+#define IQQ_C(n, k) (static_cast<float>((n) * (80 + (k))) / 80.0f)
+#define IQQ_CROW(n)                                                                                   \
+    {IQQ_C(n, -9), IQQ_C(n, -8), IQQ_C(n, -7), IQQ_C(n, -6), IQQ_C(n, -5), IQQ_C(n, -4), IQQ_C(n, -3), \
+     IQQ_C(n, -2), IQQ_C(n, -1), IQQ_C(n, 0),  IQQ_C(n, 1),  IQQ_C(n, 2),  IQQ_C(n, 3),  IQQ_C(n, 4),  \
+     IQQ_C(n, 5),  IQQ_C(n, 6),  IQQ_C(n, 7),  IQQ_C(n, 8),  IQQ_C(n, 9)}
+__constant__ float c_cand_all[4][kCand] = {IQQ_CROW(8), IQQ_CROW(16), IQQ_CROW(32), IQQ_CROW(128)};
+#undef IQQ_CROW
+#undef IQQ_C
 
 // rint(v) for |v| < 2^22, half to even.
 __device__ __forceinline__ float rint_small(float v) { return __fsub_rn(__fadd_rn(v, kMagic), kMagic); }
 
-__device__ __forceinline__ float clamp_code(float r) { return fminf(fmaxf(r, -8.0f), 7.0f); }
+template <int NMAX>
+__device__ __forceinline__ float clamp_code(float r)
+{
+    return fminf(fmaxf(r, static_cast<float>(-NMAX)), static_cast<float>(NMAX - 1));
+}
 
 __device__ __forceinline__ double block_reduce_sum(double v, double* s_red)
 {
@@ -120,7 +139,7 @@ __device__ __forceinline__ void keep_best(float s, float t, int k, float& best, 
 // min(v + M, M + B) - M -- then the two sequential sums |sumlx| += |wx|*m and
 // suml2 += w*m*m.  |wx|, B, M + B and w stream from this thread's rows of the
 // warp's shared memory (LDS.128).
-template <int N>
+template <int BITS, int N>
 __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const float* __restrict__ my_w,
                                             const float* __restrict__ my_awx,
                                             const float* __restrict__ my_ub, float amax,
@@ -130,7 +149,7 @@ __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const
     float a[N], s[N], t[N];
 #pragma unroll
     for (int c = 0; c < N; ++c) {
-        a[c] = __fdiv_rn(c_cand[k0 + c], amax);  // |iscale_k|
+        a[c] = __fdiv_rn(c_cand_all[Fmt<BITS>::fi][k0 + c], amax);  // |iscale_k|
         s[c] = 0.0f;
         t[c] = 0.0f;
     }
@@ -171,6 +190,7 @@ __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const
 // move the sequential pass accepts first.  The state then advances and the scan
 // resumes after that element, so the sequence of accepted moves and every
 // rounding is that of the sequential Gauss-Seidel passes.
+template <int NMAX>
 __device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, float* sL, unsigned pending,
                                             float sumlx, float suml2, float score)
 {
@@ -196,7 +216,8 @@ __device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, fl
             const float ln = __fadd_rn(lj, sg);
             const float nlx = __fadd_rn(lx, __fmul_rn(sg, wxj));
             const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), l2);
-            bool ok = lane >= start && (g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f;
+            bool ok = lane >= start && (g > 0.0f || g < 0.0f) && ln >= static_cast<float>(-NMAX) &&
+                      ln <= static_cast<float>(NMAX - 1) && nl2 > 0.0f;
             float ns = 0.0f;
             if (ok) {
                 ns = __fdiv_rn(__fmul_rn(nlx, nlx), nl2);
@@ -229,8 +250,9 @@ __device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, fl
     }
 }
 
+template <int BITS>
 __global__ void __launch_bounds__(kThreads, IQQ_Q4_MIN_CTAS)
-q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
+qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
               int chunks_per_row, uint32_t* __restrict__ flags)
 {
@@ -246,6 +268,7 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
     float* const sL = warp_smem + kScratch + 32 * kRow1;
     float* const my_x = sX + lane * kRow1;
     float* const my_l = sL + lane * kRow1;
+    constexpr int NMAX = Fmt<BITS>::nmax;
     const int64_t nb = n_per_row / QK;
     const int64_t nwork = nrows * chunks_per_row;
 
@@ -356,15 +379,16 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
 #pragma unroll
             for (int j4 = 0; j4 < QK; j4 += 4) {
                 const float4 w4 = *reinterpret_cast<const float4*>(my_w + j4);
-                // |wx| and the clamp bound B: 8 when x_j has the sign of xmax (its code
-                // is <= 0, clamped at -8), 7 otherwise; also M + B for the adds form
+                // |wx| and the clamp bound B: nmax when x_j has the sign of xmax (its code
+                // is <= 0, clamped at -nmax), nmax - 1 otherwise
 #define IQQ_DIFF(j) ((__float_as_uint(xv[j]) ^ sxm) >> 31)
                 *reinterpret_cast<float4*>(my_awx + j4) =
                     make_float4(fabsf(__fmul_rn(w4.x, xv[j4])), fabsf(__fmul_rn(w4.y, xv[j4 + 1])),
                                 fabsf(__fmul_rn(w4.z, xv[j4 + 2])), fabsf(__fmul_rn(w4.w, xv[j4 + 3])));
+                constexpr float kB0 = static_cast<float>(NMAX), kB1 = static_cast<float>(NMAX - 1);
                 *reinterpret_cast<float4*>(my_ub + j4) =
-                    make_float4(IQQ_DIFF(j4) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 1) ? 7.0f : 8.0f,
-                                IQQ_DIFF(j4 + 2) ? 7.0f : 8.0f, IQQ_DIFF(j4 + 3) ? 7.0f : 8.0f);
+                    make_float4(IQQ_DIFF(j4) ? kB1 : kB0, IQQ_DIFF(j4 + 1) ? kB1 : kB0,
+                                IQQ_DIFF(j4 + 2) ? kB1 : kB0, IQQ_DIFF(j4 + 3) ? kB1 : kB0);
 #undef IQQ_DIFF
             }
             if (amax > 0.0f) {
@@ -372,9 +396,9 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 int k0 = 0;
 #pragma unroll 1
                 for (; k0 + N <= kCand; k0 += N)
-                    sweep_group<N>(k0, xv, my_w, my_awx, my_ub, amax, best, kbest);
+                    sweep_group<BITS, N>(k0, xv, my_w, my_awx, my_ub, amax, best, kbest);
 #pragma unroll 1
-                for (; k0 < kCand; ++k0) sweep_group<1>(k0, xv, my_w, my_awx, my_ub, amax, best, kbest);
+                for (; k0 < kCand; ++k0) sweep_group<BITS, 1>(k0, xv, my_w, my_awx, my_ub, amax, best, kbest);
             }
         }
         __syncwarp();  // the sweep area becomes the x / code staging area
@@ -389,11 +413,11 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
             if (amax > 0.0f) {
                 if (best == -INFINITY) {
                     // no candidate has positive weighted code energy: codes of k = 0, d = 1/iscale_0
-                    iscale = __fdiv_rn(-8.0f, xmax);
+                    iscale = __fdiv_rn(static_cast<float>(-NMAX), xmax);
                     dfb = __fdiv_rn(1.0f, iscale);
                     mode = 1;
                 } else {
-                    iscale = __fdiv_rn(-c_cand[kbest], xmax);
+                    iscale = __fdiv_rn(-c_cand_all[Fmt<BITS>::fi][kbest], xmax);
                     score = best;
                     mode = 2;
                 }
@@ -401,7 +425,7 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
 #pragma unroll 4
             for (int j = 0; j < QK; ++j) {
                 const float xj = my_x[j], wj = my_w[j];
-                const float l = clamp_code(rint_small(__fmul_rn(iscale, xj)));
+                const float l = clamp_code<NMAX>(rint_small(__fmul_rn(iscale, xj)));
                 my_l[j] = l;
                 sumlx = __fmaf_rn(__fmul_rn(wj, xj), l, sumlx);
                 suml2 = __fmaf_rn(wj, __fmul_rn(l, l), suml2);
@@ -425,7 +449,8 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 // then nlx^2/nl2 < score exactly and its rounded quotient cannot exceed score
                 const float thr = __fmul_rn(__fmul_rn(score, nl2), 0.99999976158142089844f);
                 const bool maybe = !(a2 <= thr && thr >= 1e-30f && thr <= 1e30f);
-                if (maybe && (g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f) {
+                if (maybe && (g > 0.0f || g < 0.0f) && ln >= static_cast<float>(-NMAX) &&
+                    ln <= static_cast<float>(NMAX - 1) && nl2 > 0.0f) {
                     const float ns = __fdiv_rn(a2, nl2);
                     if (ns > score) {
                         my_l[j] = ln;
@@ -442,13 +467,12 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
         const unsigned pending = __ballot_sync(kFull, changed);
         if (pending != 0u) {
             __syncwarp();
-            greedy_warp(sX, sW, sL, pending, sumlx, suml2, score);
+            greedy_warp<NMAX>(sX, sW, sL, pending, sumlx, suml2, score);
         }
         __syncwarp();
 
-        // final sums from the final codes, d, and the packed nibbles
+        // final sums from the final codes, d, and the packed block
         uint16_t d16 = 0;
-        uint32_t qs[4];  // 16 bytes: byte i = (l[i]+8) | (l[i+16]+8) << 4
         {
             float d = dfb;
             if (mode == 2) {
@@ -465,26 +489,43 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 d16 = __half_as_ushort(__float2half_rn(d));
                 if ((d16 & 0x7fffu) == 0x7c00u && isfinite(d)) bad |= IQQ_FLAG_SCALE_OVERFLOW;
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t word = 0u;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    // code + 8 from the float code: the low bits of (l + M + 8)
-                    const uint32_t lo = __float_as_uint(__fadd_rn(my_l[4 * i + k], kMagic + 8.0f)) & 0xfu;
-                    const uint32_t hi = __float_as_uint(__fadd_rn(my_l[4 * i + k + 16], kMagic + 8.0f)) & 0xfu;
-                    word |= (lo | (hi << 4)) << (8 * k);
-                }
-                qs[i] = word;
-            }
         }
         if (valid) {
-            uint16_t* o16 = reinterpret_cast<uint16_t*>(out + (row * nb + b) * IQQ_Q4_0_BLOCK_BYTES);
+            // biased code n = l + nmax: the low byte of (l + nmax + 1.5*2^23)
+            auto biased = [&](int j) -> uint32_t {
+                return __float_as_uint(__fadd_rn(my_l[j], kMagic + static_cast<float>(NMAX))) & 0xffu;
+            };
+            uint16_t* o16 = reinterpret_cast<uint16_t*>(out + (row * nb + b) * Fmt<BITS>::bytes);
             o16[0] = d16;
+            if (BITS == 8) {
+                // int8 codes: the low byte of (l + 1.5*2^23) is l in two's complement
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                o16[1 + 2 * i] = static_cast<uint16_t>(qs[i] & 0xffffu);
-                o16[2 + 2 * i] = static_cast<uint16_t>(qs[i] >> 16);
+                for (int i = 0; i < QK / 2; ++i) {
+                    const uint32_t lo = __float_as_uint(__fadd_rn(my_l[2 * i], kMagic)) & 0xffu;
+                    const uint32_t hi = __float_as_uint(__fadd_rn(my_l[2 * i + 1], kMagic)) & 0xffu;
+                    o16[1 + i] = static_cast<uint16_t>(lo | (hi << 8));
+                }
+            } else {
+                constexpr int kHighWords = BITS == 4 ? 0 : (BITS == 5 ? 2 : 4);  // 16-bit words of qh
+                if (BITS != 4) {
+                    uint32_t qh[2] = {0u, 0u};
+#pragma unroll
+                    for (int j = 0; j < QK; ++j) {
+                        const uint32_t n = biased(j);
+                        if (BITS == 5) qh[0] |= ((n >> 4) & 1u) << j;
+                        else qh[j >> 4] |= ((n >> 4) & 3u) << (2 * (j & 15));
+                    }
+#pragma unroll
+                    for (int i = 0; i < kHighWords; ++i)
+                        o16[1 + i] = static_cast<uint16_t>(qh[i >> 1] >> (16 * (i & 1)));
+                }
+#pragma unroll
+                for (int i = 0; i < QK / 4; ++i) {
+                    // bytes 2i, 2i+1 of qs: low nibbles of codes 2i, 2i+1 and 2i+16, 2i+17
+                    const uint32_t b0 = (biased(2 * i) & 15u) | ((biased(2 * i + 16) & 15u) << 4);
+                    const uint32_t b1 = (biased(2 * i + 1) & 15u) | ((biased(2 * i + 17) & 15u) << 4);
+                    o16[1 + kHighWords + i] = static_cast<uint16_t>(b0 | (b1 << 8));
+                }
             }
         }
         iqq::raise_flags(flags, bad);
@@ -494,20 +535,10 @@ q4_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
 
 constexpr size_t kDynSmem = sizeof(float) * kWarpFloats * kWarps;
 
-}  // namespace
-
-extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64_t nrows,
-                                          int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
-                                          uint32_t* d_flags, void* stream)
+template <int BITS>
+iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
+                     int64_t rows_per_qw, int weight_mode, uint32_t* d_flags, void* stream)
 {
-    if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
-    if (n_per_row % QK != 0) return IQQ_ERR_SHAPE;
-    if (weight_mode < 0 || weight_mode > 5) return IQQ_ERR_ARG;
-    if (nrows == 0 || n_per_row == 0) return IQQ_OK;
-    if (x == nullptr || out == nullptr) return IQQ_ERR_NULL;
-    if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||
-        (d_flags && !iqq::aligned(d_flags, 4)))
-        return IQQ_ERR_ALIGN;
     const int64_t nb = n_per_row / QK;
     const int64_t chunks = (nb + kThreads - 1) / kThreads;
     if (chunks > 0x7fffffff) return IQQ_ERR_SHAPE;
@@ -517,13 +548,50 @@ extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void*
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return iqq::launch_status();
     if (configured_device != dev) {
-        if (cudaFuncSetAttribute(q4_0_w_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(qx_0_w_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kDynSmem)) != cudaSuccess)
             return iqq::launch_status();
         configured_device = dev;
     }
-    q4_0_w_kernel<<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
+    qx_0_w_kernel<BITS><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
         x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode,
         static_cast<int>(chunks), d_flags);
     return iqq::launch_status();
+}
+
+iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int64_t nrows,
+                       int64_t n_per_row, int64_t rows_per_qw, int weight_mode, uint32_t* d_flags,
+                       void* stream)
+{
+    if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
+    if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
+    if (n_per_row % QK != 0) return IQQ_ERR_SHAPE;
+    if (weight_mode < 0 || weight_mode > 5) return IQQ_ERR_ARG;
+    if (nrows == 0 || n_per_row == 0) return IQQ_OK;
+    if (x == nullptr || out == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||
+        (d_flags && !iqq::aligned(d_flags, 4)))
+        return IQQ_ERR_ALIGN;
+    switch (bits) {
+    case 4: return launch_qx<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    case 5: return launch_qx<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    case 6: return launch_qx<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    default: return launch_qx<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    }
+}
+
+}  // namespace
+
+extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64_t nrows,
+                                          int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                                          uint32_t* d_flags, void* stream)
+{
+    return quantize_qx(4, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+}
+
+extern "C" iqq_status iqq_quantize_qx_0_w(int bits, const float* x, const float* qw, void* out,
+                                          int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                          int weight_mode, uint32_t* d_flags, void* stream)
+{
+    return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
 }

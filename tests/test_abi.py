@@ -25,7 +25,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("iqq_quantize_q4_0_w", "iqq_quantize_q8_k128", "iqq_dequant_q4_0",
-              "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string"):
+              "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string",
+              "iqq_quantize_qx_0_w", "iqq_dequant_qx_0"):
         assert n in names
 
 
@@ -70,6 +71,18 @@ def test_host_validation_without_gpu(lib):
     # enumerated argument
     assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 4, 32, 0, 6, None, None) == 5
     assert lib.iqq_quantize_q4_0_w(V(16), None, V(16), 4, 32, 0, -1, None, None) == 5
+    # the generic block formats: bits checked first, then as for Q4_0
+    for bits in (3, 7, 0, 16):
+        assert lib.iqq_quantize_qx_0_w(bits, V(16), None, V(16), 4, 32, 0, 0, None, None) == 5
+        assert lib.iqq_dequant_qx_0(bits, V(16), V(16), 1, 32, None) == 5
+    for bits in (4, 5, 6, 8):
+        assert lib.iqq_quantize_qx_0_w(bits, None, None, None, 4, 33, 0, 0, None, None) == 2
+        assert lib.iqq_quantize_qx_0_w(bits, None, None, None, 0, 64, 0, 0, None, None) == 0
+        assert lib.iqq_quantize_qx_0_w(bits, V(16), None, V(17), 4, 32, 0, 0, None, None) == 3
+        assert lib.iqq_quantize_qx_0_w(bits, V(16), None, V(16), 4, 32, 0, 6, None, None) == 5
+        assert lib.iqq_dequant_qx_0(bits, V(16), V(16), 2, 48, None) == 2
+        assert lib.iqq_dequant_qx_0(bits, None, V(16), 1, 32, None) == 1
+        assert lib.iqq_dequant_qx_0(bits, V(16), V(8), 1, 32, None) == 3
 
 
 def test_status_strings(lib):

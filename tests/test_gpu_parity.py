@@ -197,6 +197,49 @@ def test_q8_k128_shapes(iqq, rows, n):
     assert np.array_equal(g, o)
 
 
+# ------------------------------------------------------------------ Q5_0 / Q6_0 / Q8_0 weighted
+
+@pytest.mark.parametrize("bits", [5, 6, 8])
+@pytest.mark.parametrize("rows,n", [(256, 4096), (7, 4192), (3, 11008)])
+def test_qx_0_weighted_and_dequant(iqq, synth, bits, rows, n):
+    x = synth.weight_matrix(rows, n, seed=bits * 100 + rows).numpy()
+    qw = synth.imatrix(n, seed=bits + n).numpy()
+    xd, qd = torch.from_numpy(x).cuda(), torch.from_numpy(qw).cuda()
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = iqq.quantize_qx_0_w(bits, xd, qd, flags=flags)
+    y = iqq.dequant_qx_0(bits, g, rows, n)
+    torch.cuda.synchronize()
+    o, of = oracle.quantize_qx_0_w(bits, x, qw)
+    bb = oracle.qx_block_bytes(bits)
+    gb = g.cpu().numpy().reshape(-1, bb)
+    ob = o.reshape(-1, bb)
+    same = np.all(gb == ob, axis=1)
+    assert int(flags.item()) == of == 0
+    assert same.mean() >= 0.9999
+    # dequantization of the GPU's blocks is bit-exact against the oracle's decoder
+    assert np.array_equal(y.cpu().numpy(), oracle.dequant_qx_0(bits, g.cpu().numpy(), rows, n))
+    # any differing block: weighted error within 1e-5 of the oracle's
+    if not same.all():
+        yo = oracle.dequant_qx_0(bits, o, rows, n).reshape(-1, 32).astype(np.float64)
+        yg = y.cpu().numpy().reshape(-1, 32).astype(np.float64)
+        xb = x.reshape(-1, 32).astype(np.float64)
+        for i in np.nonzero(~same)[0]:
+            r = i // (n // 32)
+            w = oracle.block_weights(x[r, 32 * (i % (n // 32)):][:32], qw[32 * (i % (n // 32)):][:32],
+                                     oracle.row_sigma2(x[r]), 0).astype(np.float64)
+            eg, eo = np.sum(w * (xb[i] - yg[i]) ** 2), np.sum(w * (xb[i] - yo[i]) ** 2)
+            assert abs(eg - eo) <= 1e-5 * eo
+
+
+def test_qx_0_bits4_is_q4_0(iqq, synth):
+    x = synth.weight_matrix(64, 4096, seed=9, device="cuda")
+    q = synth.imatrix(4096, seed=10, device="cuda")
+    assert torch.equal(iqq.quantize_qx_0_w(4, x, q), iqq.quantize_q4_0_w(x, q))
+    with pytest.raises(iqq.IQQError, match="ARG"):
+        iqq._check("q", iqq._lib.iqq_quantize_qx_0_w(7, x.data_ptr(), None, x.data_ptr(), 64, 4096, 0, 0,
+                                                     None, None))
+
+
 # ------------------------------------------------------------------ Q8_1 (overflow contrast)
 
 def test_q8_1_bit_exact_and_overflow_count(iqq, synth):

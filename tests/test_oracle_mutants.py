@@ -15,16 +15,25 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 MUTANTS = {
     "nibble_order": ("blk[2 + i] = (uint8_t)((L[i] + 8) | ((L[i + 16] + 8) << 4));",
                      "blk[2 + i] = (uint8_t)((L[2*i] + 8) | ((L[2*i + 1] + 8) << 4));"),
-    "sigma2_dropped": ("float u = sigma2 + t;", "float u = t;"),
+    "sigma2_dropped": ("default: m = sqrtf(sigma2 + t); break;", "default: m = sqrtf(t); break;"),
     "greedy_direction": ("float s = g > 0.0f ? 1.0f : -1.0f;", "float s = g > 0.0f ? -1.0f : 1.0f;"),
     "iscale_sign": ("float iscale = -c / xmax;", "float iscale = c / xmax;"),
     "xmax_unsigned": ("if (a > amax) { amax = a; xmax = xb[j]; }",
                       "if (a > amax) { amax = a; xmax = a; }"),
     "ties_to_last_k": ("if (score > best) {", "if (score >= best) {"),
-    "symmetric_clamp": ("l[j] = fminf(fmaxf(r, -8.0f), 7.0f);", "l[j] = fminf(fmaxf(r, -7.0f), 7.0f);"),
+    "symmetric_clamp": ("const float lo = (float)(-nmax), hi = (float)(nmax - 1);\n    for (int j = 0; j < n; ++j) {\n        float v",
+                        "const float lo = (float)(1 - nmax), hi = (float)(nmax - 1);\n    for (int j = 0; j < n; ++j) {\n        float v"),
     "greedy_trial_term": ("float nl2 = fmaf(w[j], 2.0f * s * lbest[j] + 1.0f, suml2);",
                           "float nl2 = fmaf(w[j], 2.0f * s * lbest[j], suml2);"),
-    "q8_scale_128": ("float d = amax / 127.0f;", "float d = amax / 128.0f;"),
+    "q8_scale_128": ("float d = amax / 127.0f;\n        float id = amax > 0.0f ? 127.0f / amax : 0.0f;\n        int8_t q",
+                     "float d = amax / 128.0f;\n        float id = amax > 0.0f ? 127.0f / amax : 0.0f;\n        int8_t q"),
+    "q8_1_sum_unscaled": ("float sf = d * (float)sum;", "float sf = (float)sum;"),
+    "q5_0_high_bit_order": ("if (bits == 5) qh |= (uint64_t)((n >> 4) & 1u) << j;",
+                            "if (bits == 5) qh |= (uint64_t)((n >> 4) & 1u) << (31 - j);"),
+    "q6_0_high_bits_dropped": ("else qh |= (uint64_t)((n >> 4) & 3u) << (2 * j);",
+                               "else qh |= (uint64_t)((n >> 4) & 1u) << (2 * j);"),
+    "qx_candidate_step": ("float c = (float)(nmax * (80 + k)) / 80.0f;",
+                          "float c = (float)(nmax * (80 + 2 * k)) / 80.0f;"),
     "q8_truncation": ("float r = fminf(fmaxf(rintf(v), -127.0f), 127.0f);",
                       "float r = fminf(fmaxf(truncf(v), -127.0f), 127.0f);"),
     "rmse_unweighted": ("acc[0] += q * (ed * ed);", "acc[0] += (ed * ed);"),
@@ -32,7 +41,8 @@ MUTANTS = {
                        "if (rem > half) q += 1u;"),
 }
 
-PIN_FILES = ["test_oracle_q4_0.py", "test_oracle_q8.py", "test_oracle_dequant_rmse.py"]
+PIN_FILES = ["test_oracle_q4_0.py", "test_oracle_q8.py", "test_oracle_dequant_rmse.py",
+             "test_oracle_qx.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
