@@ -69,6 +69,8 @@ def lib():
         L.oracle_quantize_q8_1.argtypes = [_f32p, _u8p, _i64, _i64]
         L.oracle_quantize_q8_k128.restype = ctypes.c_int
         L.oracle_quantize_q8_k128.argtypes = [_f32p, _u8p, _i64, _i64, _u32p]
+        L.oracle_dot_q4_0_q8_k128.restype = ctypes.c_int
+        L.oracle_dot_q4_0_q8_k128.argtypes = [_u8p, _u8p, _f64p, _f64p, _i64, _i64, _i64]
         _LIB = L
     return _LIB
 
@@ -268,6 +270,22 @@ def decode_q8_k128(blocks, nrows: int, n_per_row: int):
     qs = b[:, :, 4:132].copy().view(np.int8).reshape(nrows, n_per_row)
     bs = b[:, :, 132:140].copy().view(np.int16).reshape(nrows, nb, 4)
     return d, qs, bs
+
+
+def dot_q4_0_q8_k128(w_blocks, a_blocks, n_out: int, k: int, n_tok: int):
+    """y[t, r] = dequant(W)[r] . dequant(A)[t] in binary64 (exact products, summed left
+    to right), and the sum of |products| beside it.  Returns (y, absum), both float64
+    [n_tok, n_out]."""
+    w = np.ascontiguousarray(w_blocks, dtype=np.uint8)
+    a = np.ascontiguousarray(a_blocks, dtype=np.uint8)
+    if w.size < n_out * (k // 32) * Q4_0_BYTES or a.size < n_tok * (k // 128) * Q8_K128_BYTES:
+        raise ValueError("dot_q4_0_q8_k128: buffers too small")
+    y = np.empty((n_tok, n_out), np.float64)
+    s = np.empty((n_tok, n_out), np.float64)
+    if lib().oracle_dot_q4_0_q8_k128(_ptr(w, _u8p), _ptr(a, _u8p), _ptr(y, _f64p), _ptr(s, _f64p),
+                                     n_out, k, n_tok) != 0:
+        raise ValueError("dot_q4_0_q8_k128: k must be a multiple of 128")
+    return y, s
 
 
 def decode_q4_0(blocks, nrows: int, n_per_row: int):

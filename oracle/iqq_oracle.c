@@ -611,6 +611,54 @@ int64_t oracle_quantize_q8_1(const float *x, uint8_t *out, int64_t nrows, int64_
     return overflow;
 }
 
+/* ------------------------------------------------------------------ */
+/* Q4_0 x Q8_K_128 dot product (matrix-vector form).                   */
+/* [Q8] 修复前的数值隐患 describes the consumer of the activation       */
+/* blocks: weight codes times int8 activation codes, block by block.    */
+/* The value computed is the plain definition -- the dot product of the */
+/* two dequantized vectors:                                             */
+/*   y[t][r] = sum_j  W~[r][j] * A~[t][j],                              */
+/*   W~ = fp16_to_float(d4) * (nibble - 8)     (exact in binary32),     */
+/*   A~ = d8 * q                               (exact in binary64).     */
+/* Each product W~ * A~ needs at most 11+4+24+8 = 47 significant bits,  */
+/* so it is exact in binary64; the K products are summed left to right  */
+/* in binary64 (error <= K * 2^-53 * sum |products|).  absum receives    */
+/* sum |W~ * A~| (the condition of the sum), and may be NULL.           */
+/* Layouts: w is n_out rows of k/32 Q4_0 blocks (18 B each); a is n_tok */
+/* rows of k/128 Q8_K_128 blocks (140 B each); y and absum are          */
+/* [n_tok][n_out].  k must be a multiple of 128.                        */
+/* ------------------------------------------------------------------ */
+int oracle_dot_q4_0_q8_k128(const uint8_t *w, const uint8_t *a, double *y, double *absum,
+                            int64_t n_out, int64_t k, int64_t n_tok)
+{
+    if (k % ORACLE_QK8 != 0 || n_out < 0 || k < 0 || n_tok < 0) return -1;
+    const int64_t nb4 = k / ORACLE_QK4_0, nb8 = k / ORACLE_QK8;
+    for (int64_t t = 0; t < n_tok; ++t) {
+        const uint8_t *ar = a + t * nb8 * ORACLE_Q8_BYTES;
+        for (int64_t r = 0; r < n_out; ++r) {
+            const uint8_t *wr = w + r * nb4 * ORACLE_Q4_0_BYTES;
+            double sum = 0.0, asum = 0.0;
+            for (int64_t j = 0; j < k; ++j) {
+                const uint8_t *wb = wr + (j / ORACLE_QK4_0) * ORACLE_Q4_0_BYTES;
+                const int i = (int)(j % ORACLE_QK4_0);
+                const int nib = i < 16 ? (wb[2 + i] & 0xf) : (wb[2 + i - 16] >> 4);
+                const double wv = (double)oracle_fp16_to_float((uint16_t)(wb[0] | (wb[1] << 8)))
+                                  * (double)(nib - 8);
+                const uint8_t *ab = ar + (j / ORACLE_QK8) * ORACLE_Q8_BYTES;
+                float d8;
+                memcpy(&d8, ab, sizeof d8);
+                const double av = (double)d8 * (double)(int8_t)ab[4 + j % ORACLE_QK8];
+                const double p = wv * av;
+                sum += p;
+                asum += fabs(p);
+            }
+            y[t * n_out + r] = sum;
+            if (absum) absum[t * n_out + r] = asum;
+        }
+    }
+    return 0;
+}
+
 /* Layout constants, for the test suite's self-description checks. */
 int oracle_q4_0_block_bytes(void) { return ORACLE_Q4_0_BYTES; }
 int oracle_q8_k128_block_bytes(void) { return ORACLE_Q8_BYTES; }

@@ -37,12 +37,17 @@ MUTANTS = {
     "q8_truncation": ("float r = fminf(fmaxf(rintf(v), -127.0f), 127.0f);",
                       "float r = fminf(fmaxf(truncf(v), -127.0f), 127.0f);"),
     "rmse_unweighted": ("acc[0] += q * (ed * ed);", "acc[0] += (ed * ed);"),
+    "dot_offset_7": ("* (double)(nib - 8);", "* (double)(nib - 7);"),
+    "dot_nibble_order": ("const int nib = i < 16 ? (wb[2 + i] & 0xf) : (wb[2 + i - 16] >> 4);",
+                         "const int nib = i < 16 ? (wb[2 + i] >> 4) : (wb[2 + i - 16] & 0xf);"),
+    "dot_activation_scale_dropped": ("const double av = (double)d8 * (double)(int8_t)ab[4 + j % ORACLE_QK8];",
+                                     "const double av = (double)(int8_t)ab[4 + j % ORACLE_QK8];"),
     "fp16_ties_down": ("if (rem > half || (rem == half && (q & 1u))) q += 1u;",
                        "if (rem > half) q += 1u;"),
 }
 
 PIN_FILES = ["test_oracle_q4_0.py", "test_oracle_q8.py", "test_oracle_dequant_rmse.py",
-             "test_oracle_qx.py"]
+             "test_oracle_qx.py", "test_oracle_dot.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
