@@ -56,6 +56,8 @@ typedef enum {
 #define IQQ_FLAG_NONFINITE_INPUT 1u /* NaN or Inf in x (or in qw)                    */
 #define IQQ_FLAG_NEG_QW 2u          /* an importance qw < 0                          */
 #define IQQ_FLAG_SCALE_OVERFLOW 4u  /* a finite Q4_0 scale rounded to +-Inf in fp16 */
+#define IQQ_FLAG_WAIT_TIMEOUT 8u    /* a staged copy did not arrive within the bounded
+                                       wait (about 2 s); the results are unspecified  */
 
 /* Block formats. */
 #define IQQ_Q4_0_BLOCK_VALUES 32
@@ -174,6 +176,32 @@ iqq_status iqq_dequant_q4_0(const void* blocks, float* y, int64_t nrows, int64_t
  */
 iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, int64_t nrows, int64_t n_per_row,
                             void* stream);
+
+/*
+ * iqq_gemv_q4_0_q8_k128 -- y[t][r] = dot(dequant(W row r), dequant(A row t)): Q4_0 weight
+ * rows times Q8_K_128 activation rows (a matrix-vector product per token).  [Q8]
+ * 修复前的数值隐患 describes the consumer of the activation blocks: unsigned weight codes
+ * times int8 activation codes, corrected by the block sum; 修复方案 makes that sum an
+ * unscaled int16 per 32 values, so the correction is exact.  Here, per 32-value block,
+ * isum = sum(u*q) - 8*bsum with u = l + 8 the stored nibble, and the block's term
+ * d8 * d4 * isum is formed exactly in binary64; the K/32 terms of a row are summed in
+ * binary64 in a fixed order and rounded once to binary32.  The result is reproducible and
+ * within (K/32 + 16) * 2^-53 * sum|terms| of the exact dot product before that rounding.
+ *
+ *  w_blocks  n_out rows of k/32 Q4_0 blocks (18 B, layout as iqq_quantize_q4_0_w),
+ *            16-byte aligned.
+ *  a_blocks  n_tok rows of k/128 Q8_K_128 blocks (140 B, layout as
+ *            iqq_quantize_q8_k128), 4-byte aligned.
+ *  y         float32 [n_tok][n_out], 4-byte aligned; fully overwritten.
+ *  k         values per row: a multiple of 128, at most IQQ_GEMV_MAX_K.  k == 0 writes
+ *            zeros (the empty dot product).
+ *  d_flags   optional; receives IQQ_FLAG_WAIT_TIMEOUT.
+ * Blocks whose binary16 scale is not finite give unspecified values in the rows that use
+ * them (iqq_quantize_q4_0_w flags such scales).
+ */
+#define IQQ_GEMV_MAX_K 65536
+iqq_status iqq_gemv_q4_0_q8_k128(const void* w_blocks, const void* a_blocks, float* y, int64_t n_out,
+                                 int64_t k, int64_t n_tok, uint32_t* d_flags, void* stream);
 
 /*
  * iqq_weighted_rmse -- round-trip error of Q4_0 blocks against the source,

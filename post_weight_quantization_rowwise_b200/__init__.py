@@ -48,6 +48,7 @@ def _load():
         "iqq_quantize_q8_1": [_vp, _vp, _i64, _i64, _vp, _vp, _vp],
         "iqq_quantize_qx_0_w": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_dequant_qx_0": [ctypes.c_int, _vp, _vp, _i64, _i64, _vp],
+        "iqq_gemv_q4_0_q8_k128": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -231,6 +232,25 @@ def iqq_dequant_q4_0(blocks, y, stream=None):
     return y
 
 
+def iqq_gemv_q4_0_q8_k128(w_blocks, a_blocks, y, k: int, flags=None, stream=None):
+    """y [n_tok, n_out] float32 = dequant(W) . dequant(A) per (token, row) for Q4_0 rows W
+    (n_out rows of k/32 blocks) and Q8_K_128 rows A (n_tok rows of k/128 blocks)."""
+    import torch
+    _need_cuda("w_blocks", w_blocks, torch.uint8)
+    _need_cuda("a_blocks", a_blocks, torch.uint8)
+    _need_cuda("y", y, torch.float32)
+    _need_cuda("flags", flags, torch.int32)
+    n_tok, n_out = _shape2(y)
+    if w_blocks.numel() < q4_0_nbytes(n_out, k):
+        raise ValueError("w_blocks is too small")
+    if a_blocks.numel() < q8_k128_nbytes(n_tok, k):
+        raise ValueError("a_blocks is too small")
+    _check("iqq_gemv_q4_0_q8_k128",
+           _lib.iqq_gemv_q4_0_q8_k128(_ptr(w_blocks), _ptr(a_blocks), _ptr(y), n_out, k, n_tok,
+                                      _ptr(flags), _stream(stream)))
+    return y
+
+
 def iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
     """Adds {sum qw e^2, sum qw, sum e^2} to acc[0:3] and maxes acc[3] with max|e| (float64, CUDA)."""
     import torch
@@ -287,6 +307,12 @@ def quantize_q8_1(x, overflow=None, flags=None, stream=None):
     nrows, n = _shape2(x)
     out = torch.empty((nrows, (n // 32) * 36), dtype=torch.uint8, device=x.device)
     return iqq_quantize_q8_1(x, out, overflow, flags, stream)
+
+
+def gemv_q4_0_q8_k128(w_blocks, a_blocks, n_out: int, k: int, n_tok: int, flags=None, stream=None):
+    import torch
+    y = torch.empty((n_tok, n_out), dtype=torch.float32, device=w_blocks.device)
+    return iqq_gemv_q4_0_q8_k128(w_blocks, a_blocks, y, k, flags, stream)
 
 
 def dequant_q4_0(blocks, nrows: int, n_per_row: int, stream=None):

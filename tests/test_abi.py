@@ -26,7 +26,7 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("iqq_quantize_q4_0_w", "iqq_quantize_q8_k128", "iqq_dequant_q4_0",
               "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string",
-              "iqq_quantize_qx_0_w", "iqq_dequant_qx_0"):
+              "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128"):
         assert n in names
 
 
@@ -83,6 +83,18 @@ def test_host_validation_without_gpu(lib):
         assert lib.iqq_dequant_qx_0(bits, V(16), V(16), 2, 48, None) == 2
         assert lib.iqq_dequant_qx_0(bits, None, V(16), 1, 32, None) == 1
         assert lib.iqq_dequant_qx_0(bits, V(16), V(8), 1, 32, None) == 3
+    # Q4_0 x Q8_K_128 matrix-vector product
+    G = lib.iqq_gemv_q4_0_q8_k128
+    assert G(V(16), V(16), V(16), 4, 96, 1, None, None) == 2          # k not a multiple of 128
+    assert G(V(16), V(16), V(16), 4, 65536 + 128, 1, None, None) == 2  # k above the maximum
+    assert G(V(16), V(16), V(16), -1, 128, 1, None, None) == 2
+    assert G(None, None, None, 0, 128, 1, None, None) == 0             # empty
+    assert G(None, None, None, 4, 128, 0, None, None) == 0
+    assert G(V(16), V(16), None, 4, 128, 1, None, None) == 1
+    assert G(None, V(16), V(16), 4, 128, 1, None, None) == 1
+    assert G(V(8), V(16), V(16), 4, 128, 1, None, None) == 3           # weights 16-byte aligned
+    assert G(V(16), V(18), V(16), 4, 128, 1, None, None) == 3
+    assert G(V(16), V(16), V(18), 4, 128, 1, None, None) == 3
 
 
 def test_status_strings(lib):
