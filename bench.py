@@ -236,6 +236,48 @@ def run_step(iqq, w: Workload, stream, ev=None):
     return 3 * len(w.tensors) + 1
 
 
+def run_gemv_phase(iqq, w: Workload, dev, reps: int = 5):
+    """One token through every quantized matrix of the layer set: y = W . a with the Q4_0
+    blocks of the step and a Q8_K_128 activation of each matrix's width (4096 or 11008).
+    The 224 launches are captured in one CUDA graph (the host-side cost of a launch exceeds
+    a 9 MB matrix's device time); replays are timed with CUDA events.  The 3.6 GB of blocks
+    exceed L2, so every replay streams them from HBM.  Returns (ms per pass, bytes)."""
+    import torch
+    from post_weight_quantization_rowwise_b200 import synth
+    acts = {}
+    for k in sorted({t.cols for t in w.tensors}):
+        a = synth.activations(1, k, seed=7 + k, device=dev)
+        acts[k] = iqq.quantize_q8_k128(a)
+    y = torch.empty(max(t.rows for t in w.tensors), dtype=torch.float32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+
+    def enqueue():
+        for t, b in zip(w.tensors, w.blocks):
+            iqq.iqq_gemv_q4_0_q8_k128(b, acts[t.cols], y[:t.rows].view(1, t.rows), t.cols, stream=s)
+
+    with torch.cuda.stream(s):
+        enqueue()  # outside the capture: fills the library's per-device launch caches
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        enqueue()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    with torch.cuda.stream(s):
+        for _ in range(reps):
+            g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = sum(t.rows * (t.cols // 32) * 18 + (t.cols // 128) * 140 + 4 * t.rows for t in w.tensors)
+    del g
+    return ms, nbytes
+
+
 def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
     """Same step through the public API from pinned host buffers: per tensor H2D of x,
     the three kernels, D2H of the blocks; D2H of the accumulator at the end."""
@@ -338,6 +380,10 @@ def main_ours(args):
     total_ms, phase = times[0], times[1:]
     acc = w.acc.cpu().tolist()
 
+    gemv = None
+    if not args.no_gemv:
+        gemv = run_gemv_phase(iqq, w, dev)
+
     e2e = None
     if rank == 0 and world == 1 and not args.no_e2e:
         e2e = run_e2e(iqq, w, dev, max(1, min(args.steps, 3)), args.e2e_layers)
@@ -394,6 +440,13 @@ def main_ours(args):
         "clocks": clk,
         "e2e": e2e,
     }
+    if gemv is not None:
+        gms, gbytes = gemv
+        ggbs = gbytes / (gms / 1e3) / 1e9
+        out["kernels"]["gemv_q4_0_q8_k128"] = {
+            "ms": round(gms, 4), "gb_s": round(ggbs, 1), "hbm_frac": round(ggbs / pk["hbm_gbs"], 4),
+            "tokens": 1, "launches": len(w.tensors), "timing": "one CUDA graph of the launches, "
+            "outside the step", "bytes": int(gbytes)}
     if cpu:
         out["cpu_baseline"] = {"value": round(cpu[0], 5), "unit": UNIT, "cores": cpu[1],
                                "kind": "oracle", "sample": cpu[2]}
@@ -442,6 +495,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-gemv", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -13,22 +13,23 @@
 //   isum  = dp4a over the nibbles - 8 * bsum                          int32, exact
 //   term  = (double)d8 * ((double)d4 * (double)isum)                  11+15+24 bits: exact
 //   y     = binary64 sum of the K/32 terms of the row, rounded once to binary32.
-// The sums run in a fixed order for a given (n_out, k): per lane over its pairs of blocks, a
-// warp butterfly, then the row's segment partials in order -- so results are reproducible
-// and within (K/32 + 16) * 2^-53 * sum|terms| of the exact dot before the final rounding.
+// (acc = fma(d8, d4 * isum, acc) is that exact product plus one rounding of the sum.)  The
+// sums run in a fixed order for a given k -- per lane over its pairs of blocks, then a warp
+// butterfly -- so results are reproducible and within (K/32 + 16) * 2^-53 * sum|terms| of
+// the exact dot product before the final rounding.
 //
-// Mapping (HBM-bound on the weight stream at small token counts):
-//  * The weights stream through shared memory in chunks of R whole rows (rows are
-//    contiguous, so a chunk is one contiguous byte range) with cp.async.bulk, completing on
-//    an mbarrier per stage; 2-4 stages are in flight per CTA.  The CTA is persistent over
-//    chunks c = blockIdx.x + i * gridDim.x.
-//  * The activations of the CTA's token tile (TT tokens) are staged once: int8 codes with a
-//    16-byte-chunk swizzle that makes the per-lane 128-bit loads conflict-free, the binary32
-//    scales and the int16 block sums.
-//  * A warp owns one (row, segment) task per chunk; a lane takes a pair of blocks (64 values,
-//    36 bytes read as nine 32-bit words -- conflict-free because 9 is odd).
-//  * Every wait on an mbarrier is bounded by a clock limit; on expiry the CTA raises
-//    IQQ_FLAG_WAIT_TIMEOUT, drains its copies in flight (again bounded) and returns.
+// Mapping (HBM-bound on the weight stream at small token counts): every warp owns whole
+// weight rows (rows gw, gw + GW, ... for global warp gw of GW) and streams each row through
+// its own shared-memory stages in units of up to 64 pairs of blocks (2304 bytes), copied
+// with cp.async.bulk and completing on the warp's own mbarriers; lane 0 keeps D units in
+// flight.  A lane takes up to two pairs of blocks per unit (36 bytes each, read as nine
+// 32-bit words: conflict-free because 9 is odd).  Partial sums stay in registers across the
+// units of a row; one butterfly per row.  The CTA synchronizes once, after staging the token
+// tile's activations (int8 codes with a 16-byte-chunk swizzle that keeps the per-lane
+// 128-bit loads conflict-free, the binary32 scales and the int16 block sums).
+//
+// Every wait on an mbarrier is bounded by a clock limit; on expiry the warp raises
+// IQQ_FLAG_WAIT_TIMEOUT, drains its copies in flight (again bounded) and returns.
 #include <cuda_fp16.h>
 
 #include <atomic>
@@ -37,13 +38,14 @@
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kMaxStages = 4;
-constexpr int kChunkTarget = 32 * 1024;
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kUnitPairs = 64;                    // pairs of blocks per streamed unit
+constexpr int kUnitBytes = kUnitPairs * 36 + 16;  // + room for the 8-byte start offset
 constexpr int kSmemMax = 227 * 1024;
 constexpr int kSmemPerSm = 228 * 1024;
-constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at the maximum SM clock
+constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the maximum SM clock
+constexpr uint32_t kSuspendHintNs = 100000;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p)
 {
@@ -66,10 +68,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0u;
 }
@@ -108,193 +110,238 @@ struct Params {
     uint32_t* flags;
     int64_t n_out;
     int64_t n_tok;
+    int64_t wbytes;    // n_out * rowbytes
     int k;
-    int rowbytes;     // (k / 32) * 18
-    int rows;         // R, rows per chunk
-    int seg;          // segments per row (R * seg == kWarps)
-    int pps;          // pairs of blocks per segment
-    int stages;
-    int64_t nchunks;
-    int act_q8_bytes;  // per token, k
-    int chunk_bytes;   // R * rowbytes rounded up to 16
-    int off_d8, off_bs, off_stage, off_part, off_bar;  // shared-memory layout
+    int rowbytes;      // (k / 32) * 18
+    int nseg;          // units per row
+    int stages;        // D, units in flight per warp
+    int act_q8_bytes;  // per token: k rounded up to 16
+    int off_d8, off_bs, off_stage, off_bar;  // shared-memory layout
 };
 
 // Byte offset of logical int8 index j of a token row in the swizzled layout: 16-byte chunk
-// c = j / 16 of pair p = c / 4 is stored at chunk 4p + ((c % 4) ^ ((p >> 1) & 3)).
-__host__ __device__ __forceinline__ int q8_swizzle(int j)
+// c = j / 16 of pair p = c / 4 is stored at chunk 4p + ((c % 4) ^ ((p >> 1) & 3)), so the
+// lanes of a quarter warp (consecutive pairs) hit distinct bank groups.
+__device__ __forceinline__ int q8_swizzle(int j)
 {
     const int c = j >> 4, p = c >> 2;
     return (((p << 2) | ((c & 3) ^ ((p >> 1) & 3))) << 4) | (j & 15);
 }
 
-__device__ __forceinline__ void issue_chunk(const Params& P, uint8_t* stage, uint64_t* bar, int64_t c)
+// Issues unit (row, seg) into a stage.  The copy starts at the 16-byte boundary at or below
+// the unit's first byte (rows start 8 bytes past one when k % 256 == 128), so the unit's
+// pairs begin at stage offset (start & 15).
+__device__ __forceinline__ void issue_unit(const Params& P, uint8_t* stage, uint64_t* bar, int64_t row, int seg)
 {
-    const int64_t row0 = c * P.rows;
-    const int64_t nr = P.n_out - row0 < P.rows ? P.n_out - row0 : P.rows;
-    const uint32_t bytes = static_cast<uint32_t>(nr * P.rowbytes);
-    const uint32_t body = bytes & ~15u;
-    const uint8_t* src = P.w + row0 * P.rowbytes;
-    if (bytes != body) {
-        // last chunk of a matrix whose byte size is 8 mod 16: the final 8 bytes by a plain
-        // load (8-byte aligned: body is a multiple of 16 from a 16-byte aligned start)
-        *reinterpret_cast<uint2*>(stage + body) = __ldg(reinterpret_cast<const uint2*>(src + body));
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const int p0 = seg * kUnitPairs;
+    const int np = (P.k >> 6) - p0 < kUnitPairs ? (P.k >> 6) - p0 : kUnitPairs;
+    const int64_t start = row * P.rowbytes + 36LL * p0;
+    const int64_t src = start & ~15LL;
+    const uint32_t total = static_cast<uint32_t>(start - src) + 36u * np;
+    uint32_t bulk = total & ~15u;
+    if (bulk != total) {
+        if (src + bulk + 16 <= P.wbytes) {
+            bulk += 16;  // over-read up to 12 bytes that still lie inside the weights
+        } else {
+            // the end of the weights: the last 4-12 bytes by plain loads (4-byte aligned)
+            for (uint32_t o = bulk; o < total; o += 4)
+                *reinterpret_cast<uint32_t*>(stage + o) = __ldg(reinterpret_cast<const uint32_t*>(P.w + src + o));
+        }
     }
-    mbar_arrive_expect_tx(bar, body);
-    bulk_copy_g2s(stage, src, body, bar);
+    // order this thread's generic-proxy accesses to the stage before the async copy into it
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(bar, bulk);
+    bulk_copy_g2s(stage, P.w + src, bulk, bar);
+}
+
+__device__ __forceinline__ double half_bits_to_double(unsigned short h)
+{
+    double d;
+    asm("cvt.f64.f16 %0, %1;" : "=d"(d) : "h"(h));
+    return d;
+}
+
+// One pair of blocks (nine words): block a (bytes 0..17) then block b (18..35).  qs holds
+// the 16 code bytes of each block, 4-byte aligned (block a's are shifted into place); byte
+// i of a block's codes has value i in its low nibble and value i + 16 in its high nibble.
+struct PairW {
+    uint32_t qs[8];
+    double d4a, d4b;
+};
+
+__device__ __forceinline__ void load_pair(const uint32_t* w9, PairW& q)
+{
+    uint32_t w[9];
+#pragma unroll
+    for (int i = 0; i < 9; ++i) w[i] = w9[i];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        q.qs[m] = __funnelshift_r(w[m], w[m + 1], 16);
+        q.qs[4 + m] = w[5 + m];
+    }
+    q.d4a = half_bits_to_double(static_cast<unsigned short>(w[0] & 0xffffu));
+    q.d4b = half_bits_to_double(static_cast<unsigned short>(w[4] >> 16));
+}
+
+// acc += the two block terms of pair p for one token.
+__device__ __forceinline__ void pair_token(const PairW& q, const uint8_t* q8t, const int16_t* bst,
+                                           const float* d8t, int p, int sw, double& acc)
+{
+    const uint8_t* qrow = q8t + (p << 6);
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(qrow + ((j ^ sw) << 4));
+    constexpr uint32_t L = 0x0F0F0F0Fu, H = 0xF0F0F0F0u;  // high nibbles kept in place: x16
+    int la = 0, ha = 0, lb = 0, hb = 0;
+    la = dp4a_us(q.qs[0] & L, v[0].x, la); la = dp4a_us(q.qs[1] & L, v[0].y, la);
+    la = dp4a_us(q.qs[2] & L, v[0].z, la); la = dp4a_us(q.qs[3] & L, v[0].w, la);
+    ha = dp4a_us(q.qs[0] & H, v[1].x, ha); ha = dp4a_us(q.qs[1] & H, v[1].y, ha);
+    ha = dp4a_us(q.qs[2] & H, v[1].z, ha); ha = dp4a_us(q.qs[3] & H, v[1].w, ha);
+    lb = dp4a_us(q.qs[4] & L, v[2].x, lb); lb = dp4a_us(q.qs[5] & L, v[2].y, lb);
+    lb = dp4a_us(q.qs[6] & L, v[2].z, lb); lb = dp4a_us(q.qs[7] & L, v[2].w, lb);
+    hb = dp4a_us(q.qs[4] & H, v[3].x, hb); hb = dp4a_us(q.qs[5] & H, v[3].y, hb);
+    hb = dp4a_us(q.qs[6] & H, v[3].z, hb); hb = dp4a_us(q.qs[7] & H, v[3].w, hb);
+    const uint32_t bsw = *reinterpret_cast<const uint32_t*>(bst + 2 * p);
+    // the high-nibble products carry a factor 16, so the shift is exact
+    const int ia = la + (ha >> 4) - 8 * static_cast<int>(static_cast<int16_t>(bsw & 0xffffu));
+    const int ib = lb + (hb >> 4) - 8 * static_cast<int>(static_cast<int16_t>(bsw >> 16));
+    const double d8 = static_cast<double>(d8t[p >> 1]);
+    acc = fma(d8, q.d4a * static_cast<double>(ia), acc);
+    acc = fma(d8, q.d4b * static_cast<double>(ib), acc);
 }
 
 template <int TT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, TT <= 2 ? 2 : 1)
 gemv_q4_0_q8_k128_kernel(const Params P)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* q8s = smem;                                              // [TT][k] swizzled
-    float* d8s = reinterpret_cast<float*>(smem + P.off_d8);           // [TT][k/128]
-    int16_t* bss = reinterpret_cast<int16_t*>(smem + P.off_bs);       // [TT][k/32]
-    uint8_t* stages = smem + P.off_stage;                             // [stages][chunk_bytes]
-    double* part = reinterpret_cast<double*>(smem + P.off_part);      // [2][kWarps][TT]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar);   // [stages]
+    uint8_t* q8s = smem;                                         // [TT][k] swizzled
+    float* d8s = reinterpret_cast<float*>(smem + P.off_d8);      // [TT][k/128]
+    int16_t* bss = reinterpret_cast<int16_t*>(smem + P.off_bs);  // [TT][k/32]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t* stages = smem + P.off_stage + warp * P.stages * kUnitBytes;               // this warp's
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar) + warp * P.stages;  // this warp's
+
     const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * TT;
     const int nt = static_cast<int>(P.n_tok - tok0 < TT ? P.n_tok - tok0 : TT);
-    const int k = P.k, nb8 = k >> 7, nb4 = k >> 5;
+    const int k = P.k, nb8 = k >> 7, nb4 = k >> 5, npairs = k >> 6;
 
-    if (tid == 0) {
-        for (int s = 0; s < P.stages; ++s) mbar_init(&bars[s], 1u);
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    const int64_t GW = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int D = P.stages, nseg = P.nseg;
+
+    // issue pointer: the next unit (irow, iseg) to copy
+    int64_t irow = gw;
+    int iseg = 0;
+    if (lane == 0) {
+        for (int s = 0; s < D; ++s) mbar_init(&bars[s], 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    __syncthreads();
-    if (tid == 0) {
-        for (int s = 0; s < P.stages; ++s) {
-            const int64_t c = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
-            if (c < P.nchunks) issue_chunk(P, stages + s * P.chunk_bytes, &bars[s], c);
+    for (int s = 0; s < D && irow < P.n_out; ++s) {
+        if (lane == 0) issue_unit(P, stages + s * kUnitBytes, &bars[s], irow, iseg);
+        if (++iseg == nseg) {
+            iseg = 0;
+            irow += GW;
         }
     }
 
-    // Stage the token tile's activations (35 words per 140-byte block) while the first
-    // weight chunks are in flight.
-    {
-        const int words = nt * nb8 * 35;
-        for (int i = tid; i < words; i += kThreads) {
-            const int t = i / (nb8 * 35), rem = i - t * (nb8 * 35);
-            const int g = rem / 35, wi = rem - g * 35;
-            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(
-                P.a + ((tok0 + t) * nb8 + g) * 140 + 4 * wi));
-            if (wi == 0) {
-                d8s[t * nb8 + g] = __uint_as_float(v);
-            } else if (wi <= 32) {
-                *reinterpret_cast<uint32_t*>(q8s + t * P.act_q8_bytes + q8_swizzle(128 * g + 4 * (wi - 1))) = v;
-            } else {
-                *reinterpret_cast<uint32_t*>(bss + t * nb4 + 4 * g + 2 * (wi - 33)) = v;
-            }
+    // Stage the token tile's activations while the first units are in flight: one warp per
+    // 140-byte block, lane i copying code word i.
+    for (int b = warp; b < nt * nb8; b += kWarps) {
+        const int t = b / nb8, g = b - t * nb8;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(P.a + ((tok0 + t) * nb8 + g) * 140);
+        const uint32_t v = __ldg(src + 1 + lane);
+        *reinterpret_cast<uint32_t*>(q8s + t * P.act_q8_bytes + q8_swizzle(128 * g + 4 * lane)) = v;
+        if (lane < 3) {
+            const uint32_t e = __ldg(src + (lane == 0 ? 0 : 32 + lane));
+            if (lane == 0) d8s[t * nb8 + g] = __uint_as_float(e);
+            else *reinterpret_cast<uint32_t*>(bss + t * nb4 + 4 * g + 2 * (lane - 1)) = e;
         }
     }
-    __syncthreads();
+    __syncthreads();  // the only CTA-wide barrier
 
-    const int P2 = k >> 6;  // pairs of blocks per row
-    int64_t it = 0;
+    // units start on 64-pair boundaries, so a lane's pairs p0 + lane and p0 + lane + 32 share
+    // the swizzle phase (p >> 1) & 3 = (lane >> 1) & 3
+    const int sw = (lane >> 1) & 3;
+    double acc[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] = 0.0;
+    // consume pointer: unit (row, seg) in stage s, phase parity ph
+    int64_t row = gw;
+    int seg = 0, s = 0;
+    uint32_t ph = 0;
     bool aborted = false;
-    for (int64_t c = blockIdx.x; c < P.nchunks; c += gridDim.x, ++it) {
-        const int s = static_cast<int>(it % P.stages);
-        const uint32_t parity = static_cast<uint32_t>((it / P.stages) & 1);
-        const bool timed_out = !mbar_wait(&bars[s], parity);
-        const uint8_t* stage = stages + s * P.chunk_bytes;
-        const int64_t row0 = c * P.rows;
-        double* pw = part + (it & 1) * (kWarps * TT);
+    while (row < P.n_out) {
+        const bool timed_out = !mbar_wait(&bars[s], ph);
+        if (__any_sync(0xffffffffu, timed_out)) {
+            aborted = true;
+            break;
+        }
+        const int p0 = seg * kUnitPairs;
+        const int np = npairs - p0 < kUnitPairs ? npairs - p0 : kUnitPairs;
+        const int64_t start = row * P.rowbytes + 36LL * p0;
+        const uint32_t* w9 = reinterpret_cast<const uint32_t*>(stages + s * kUnitBytes + (start & 15));
 
-        // one (row, segment) task per warp
-        const int rho = warp / P.seg, sigma = warp - rho * P.seg;
-        double acc[TT];
-#pragma unroll
-        for (int t = 0; t < TT; ++t) acc[t] = 0.0;
-        if (row0 + rho < P.n_out) {
-            const int pb = sigma * P.pps;
-            const int pe = pb + P.pps < P2 ? pb + P.pps : P2;
-            const uint32_t* rw = reinterpret_cast<const uint32_t*>(stage + rho * P.rowbytes);
-            for (int p = pb + lane; p < pe; p += 32) {
-                uint32_t w[9];
-#pragma unroll
-                for (int i = 0; i < 9; ++i) w[i] = rw[9 * p + i];
-                const float d4a = __half2float(__ushort_as_half(static_cast<unsigned short>(w[0] & 0xffffu)));
-                const float d4b = __half2float(__ushort_as_half(static_cast<unsigned short>(w[4] >> 16)));
-                uint32_t lo[8], hi[8];  // nibbles of block a (0..3) and block b (4..7)
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const uint32_t qa = __funnelshift_r(w[m], w[m + 1], 16);
-                    lo[m] = qa & 0x0F0F0F0Fu;
-                    hi[m] = (qa >> 4) & 0x0F0F0F0Fu;
-                    lo[4 + m] = w[5 + m] & 0x0F0F0F0Fu;
-                    hi[4 + m] = (w[5 + m] >> 4) & 0x0F0F0F0Fu;
-                }
-                const int sw = (p >> 1) & 3;
-#pragma unroll
-                for (int t = 0; t < TT; ++t) {
-                    if (t < nt) {
-                        const uint8_t* qrow = q8s + t * P.act_q8_bytes + (p << 6);
-                        uint4 q[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) q[j] = *reinterpret_cast<const uint4*>(qrow + ((j ^ sw) << 4));
-                        // block a: values 0..15 <- q[0], q[1]; values 16..31 <- q[2], q[3]
-                        int sa = 0, sb = 0;
-                        sa = dp4a_us(lo[0], q[0].x, sa); sa = dp4a_us(lo[1], q[0].y, sa);
-                        sa = dp4a_us(lo[2], q[0].z, sa); sa = dp4a_us(lo[3], q[0].w, sa);
-                        sa = dp4a_us(hi[0], q[1].x, sa); sa = dp4a_us(hi[1], q[1].y, sa);
-                        sa = dp4a_us(hi[2], q[1].z, sa); sa = dp4a_us(hi[3], q[1].w, sa);
-                        sb = dp4a_us(lo[4], q[2].x, sb); sb = dp4a_us(lo[5], q[2].y, sb);
-                        sb = dp4a_us(lo[6], q[2].z, sb); sb = dp4a_us(lo[7], q[2].w, sb);
-                        sb = dp4a_us(hi[4], q[3].x, sb); sb = dp4a_us(hi[5], q[3].y, sb);
-                        sb = dp4a_us(hi[6], q[3].z, sb); sb = dp4a_us(hi[7], q[3].w, sb);
-                        const uint32_t bsw = *reinterpret_cast<const uint32_t*>(bss + t * nb4 + 2 * p);
-                        const int ia = sa - 8 * static_cast<int>(static_cast<int16_t>(bsw & 0xffffu));
-                        const int ib = sb - 8 * static_cast<int>(static_cast<int16_t>(bsw >> 16));
-                        const double d8 = static_cast<double>(d8s[t * nb8 + (p >> 1)]);
-                        acc[t] += d8 * (static_cast<double>(d4a) * static_cast<double>(ia));
-                        acc[t] += d8 * (static_cast<double>(d4b) * static_cast<double>(ib));
-                    }
-                }
+        PairW q0, q1;
+        const bool has0 = lane < np, has1 = lane + 32 < np;
+        if (has0) load_pair(w9 + 9 * lane, q0);
+        if (has1) load_pair(w9 + 9 * (lane + 32), q1);
+        __syncwarp();
+        // every lane holds its words: refill the stage with the next unit to copy
+        if (irow < P.n_out) {
+            if (lane == 0) issue_unit(P, stages + s * kUnitBytes, &bars[s], irow, iseg);
+            if (++iseg == nseg) {
+                iseg = 0;
+                irow += GW;
             }
         }
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-        }
-        if (lane == 0) {
-#pragma unroll
-            for (int t = 0; t < TT; ++t) pw[warp * TT + t] = acc[t];
-        }
-        if (__syncthreads_or(timed_out)) {  // uniform across the CTA
-            aborted = true;
-            break;
-        }
-        // refill the stage just consumed (every thread has passed its reads)
-        if (tid == 0) {
-            const int64_t cn = c + static_cast<int64_t>(P.stages) * gridDim.x;
-            if (cn < P.nchunks) issue_chunk(P, stages + s * P.chunk_bytes, &bars[s], cn);
-        }
-        // finalize: row partials summed over segments in order
-        if (tid < P.rows * nt) {
-            const int r = tid / nt, t = tid - r * nt;
-            if (row0 + r < P.n_out) {
-                double v = 0.0;
-                for (int sg = 0; sg < P.seg; ++sg) v += pw[(r * P.seg + sg) * TT + t];
-                P.y[(tok0 + t) * P.n_out + row0 + r] = static_cast<float>(v);
+            if (t < nt) {
+                const uint8_t* q8t = q8s + t * P.act_q8_bytes;
+                const int16_t* bst = bss + t * nb4;
+                const float* d8t = d8s + t * nb8;
+                if (has0) pair_token(q0, q8t, bst, d8t, p0 + lane, sw, acc[t]);
+                if (has1) pair_token(q1, q8t, bst, d8t, p0 + lane + 32, sw, acc[t]);
             }
+        }
+        if (++seg == nseg) {  // the row is complete
+#pragma unroll
+            for (int t = 0; t < TT; ++t) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < TT; ++t)
+                    if (t < nt) P.y[(tok0 + t) * P.n_out + row] = static_cast<float>(acc[t]);
+            }
+#pragma unroll
+            for (int t = 0; t < TT; ++t) acc[t] = 0.0;
+            seg = 0;
+            row += GW;
+        }
+        if (++s == D) {
+            s = 0;
+            ph ^= 1u;
         }
     }
 
-    if (aborted && tid == 0) {
+    if (aborted && lane == 0) {
+        // a wait ran out: report, then wait (bounded) for this warp's copies in flight, which
+        // are the units from (row, seg) up to the issue pointer
         iqq::raise_flags(P.flags, IQQ_FLAG_WAIT_TIMEOUT);
-        // drain: wait (bounded) for every copy this CTA issued and did not consume
-        int64_t j = it;
-        for (int64_t c = blockIdx.x + it * static_cast<int64_t>(gridDim.x); c < P.nchunks && j < it + P.stages;
-             c += gridDim.x, ++j) {
-            const int s = static_cast<int>(j % P.stages);
-            (void)mbar_wait(&bars[s], static_cast<uint32_t>((j / P.stages) & 1));
+        for (int j = 0; j < D && (row < irow || (row == irow && seg < iseg)); ++j) {
+            (void)mbar_wait(&bars[s], ph);
+            if (++seg == nseg) {
+                seg = 0;
+                row += GW;
+            }
+            if (++s == D) {
+                s = 0;
+                ph ^= 1u;
+            }
         }
     }
 }
@@ -303,7 +350,7 @@ gemv_q4_0_q8_k128_kernel(const Params P)
 // time in these queries than a small matrix takes on the GPU).
 struct DeviceCache {
     std::atomic<int> sms{0};
-    std::atomic<int> smem_set[4] = {{0}, {0}, {0}, {0}};  // largest dynamic smem opted in, per TT
+    std::atomic<int> smem_set[4] = {{0}, {0}, {0}, {0}};  // dynamic smem opted in, per TT
     std::atomic<int> regs[4] = {{0}, {0}, {0}, {0}};      // registers per thread, per TT
 };
 constexpr int kMaxDevices = 64;
@@ -327,66 +374,96 @@ int sm_count_gemv(int dev)
     return sms;
 }
 
+constexpr int tt_slot(int tt) { return tt == 1 ? 0 : (tt == 2 ? 1 : (tt == 4 ? 2 : 3)); }
+
 int align16(int v) { return (v + 15) & ~15; }
 
-// Shared-memory plan for a token tile of tt tokens; false if it does not fit.
-bool make_plan(Params& P, int tt)
+int smem_bytes(const Params& P) { return P.off_bar + kWarps * P.stages * 8; }
+
+// Shared-memory layout for a token tile of tt tokens and d units in flight per warp.
+void make_plan(Params& P, int tt, int d)
 {
     const int k = P.k;
     P.rowbytes = (k / 32) * 18;
-    const bool row16 = (P.rowbytes % 16) == 0;
-    int R = 8;
-    while (R > 1 && R * P.rowbytes > kChunkTarget) R >>= 1;
-    if (!row16 && R < 2) R = 2;  // chunks must start on 16-byte boundaries
-    P.rows = R;
-    P.seg = kWarps / R;
-    const int pairs = k / 64;
-    P.pps = (pairs + P.seg - 1) / P.seg;
-    P.nchunks = (P.n_out + R - 1) / R;
+    P.nseg = (k / 64 + kUnitPairs - 1) / kUnitPairs;
+    P.stages = d;
     P.act_q8_bytes = align16(k);
     P.off_d8 = tt * P.act_q8_bytes;
     P.off_bs = align16(P.off_d8 + tt * (k / 128) * 4);
-    P.off_part = align16(P.off_bs + tt * (k / 32) * 2);
-    P.off_bar = P.off_part + 2 * kWarps * tt * 8;
-    P.off_stage = align16(P.off_bar + kMaxStages * 8);
-    P.chunk_bytes = align16(R * P.rowbytes);
-    const int room = kSmemMax - P.off_stage;
-    int st = room / P.chunk_bytes;
-    if (st > kMaxStages) st = kMaxStages;
-    if (st < 2) return false;
-    P.stages = st;
+    P.off_stage = align16(P.off_bs + tt * (k / 32) * 2);
+    P.off_bar = P.off_stage + kWarps * d * kUnitBytes;
+}
+
+// Resident CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA) and 64 K registers
+// (allocated per warp in units of 256).
+int ctas_per_sm(int smem, int regs)
+{
+    int occ = kSmemPerSm / (smem + 1024);
+    const int regs_cta = ((regs * 32 + 255) / 256) * 256 * kWarps;
+    if (65536 / regs_cta < occ) occ = 65536 / regs_cta;
+    return occ;
+}
+
+template <int TT>
+int kernel_regs(int dev)
+{
+    std::atomic<int>& cached = g_cache[dev].regs[tt_slot(TT)];
+    int regs = cached.load(std::memory_order_relaxed);
+    if (regs == 0) {
+        cudaFuncAttributes fa{};
+        regs = 64;
+        if (cudaFuncGetAttributes(&fa, gemv_q4_0_q8_k128_kernel<TT>) == cudaSuccess && fa.numRegs > 0)
+            regs = fa.numRegs;
+        cached.store(regs, std::memory_order_relaxed);
+    }
+    return regs;
+}
+
+// Chooses D in 2..4: the most units in flight per SM among the layouts that fit, and at
+// equal flight the layout with more resident warps (measured on B200: 32 warps x 2 units
+// beat 16 warps x 4 units, the per-unit arithmetic needing the extra warps to hide its
+// latency).
+template <int TT>
+bool plan_tt(Params& P, int dev, int& ctas)
+{
+    const int regs = kernel_regs<TT>(dev);
+    int best_d = 0, best_flight = 0, best_ctas = 0;
+    for (int d = 2; d <= 4; ++d) {
+        make_plan(P, TT, d);
+        const int smem = smem_bytes(P);
+        if (smem > kSmemMax) break;
+        const int c = ctas_per_sm(smem, regs);
+        if (c < 1) break;
+        if (c * d > best_flight) {
+            best_flight = c * d;
+            best_d = d;
+            best_ctas = c;
+        }
+    }
+    if (best_d == 0) return false;
+    make_plan(P, TT, best_d);
+    ctas = best_ctas;
     return true;
 }
 
 template <int TT>
-iqq_status launch_tt(Params& P, cudaStream_t st)
+iqq_status plan_and_launch(Params& P, cudaStream_t st, bool& fits)
 {
-    constexpr int slot = TT == 1 ? 0 : (TT == 2 ? 1 : (TT == 4 ? 2 : 3));
-    const int smem = P.off_stage + P.stages * P.chunk_bytes;
-    auto kern = gemv_q4_0_q8_k128_kernel<TT>;
     const int dev = current_device();
-    std::atomic<int>& opted = g_cache[dev].smem_set[slot];
+    int ctas = 0;
+    fits = plan_tt<TT>(P, dev, ctas);
+    if (!fits) return IQQ_OK;
+    const int smem = smem_bytes(P);
+    auto kern = gemv_q4_0_q8_k128_kernel<TT>;
+    std::atomic<int>& opted = g_cache[dev].smem_set[tt_slot(TT)];
     if (opted.load(std::memory_order_relaxed) < smem) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
             return iqq::launch_status();
         opted.store(kSmemMax, std::memory_order_relaxed);
     }
-    int regs = g_cache[dev].regs[slot].load(std::memory_order_relaxed);
-    if (regs == 0) {
-        cudaFuncAttributes fa{};
-        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return iqq::launch_status();
-        regs = fa.numRegs > 0 ? fa.numRegs : 255;
-        g_cache[dev].regs[slot].store(regs, std::memory_order_relaxed);
-    }
-    // resident CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA) and 64 K
-    // registers (allocated per warp in units of 256)
-    int occ = kSmemPerSm / (smem + 1024);
-    const int regs_cta = ((regs * 32 + 255) / 256) * 256 * kWarps;
-    if (65536 / regs_cta < occ) occ = 65536 / regs_cta;
-    if (occ < 1) occ = 1;
-    if (occ > 4) occ = 4;
-    const int64_t cap = static_cast<int64_t>(sm_count_gemv(dev)) * occ;
-    const int gx = static_cast<int>(P.nchunks < cap ? P.nchunks : cap);
+    const int64_t need = (P.n_out + kWarps - 1) / kWarps;
+    const int64_t cap = static_cast<int64_t>(sm_count_gemv(dev)) * ctas;
+    const int gx = static_cast<int>(need < cap ? need : cap);
     const int64_t gy = (P.n_tok + TT - 1) / TT;
     if (gy > 65535) return IQQ_ERR_SHAPE;
     kern<<<dim3(gx, static_cast<unsigned>(gy)), kThreads, smem, st>>>(P);
@@ -423,15 +500,21 @@ extern "C" iqq_status iqq_gemv_q4_0_q8_k128(const void* w_blocks, const void* a_
     P.n_out = n_out;
     P.n_tok = n_tok;
     P.k = static_cast<int>(k);
-    int tt = n_tok >= 8 ? 8 : (n_tok >= 4 ? (n_tok == 4 ? 4 : 8) : (n_tok == 3 ? 4 : static_cast<int>(n_tok)));
-    while (!make_plan(P, tt)) {
+    P.wbytes = n_out * ((k / 32) * 18);
+    // token tile: the smallest of 1, 2, 4, 8 covering n_tok (8 beyond), halved while the
+    // activations do not fit beside the weight stages
+    int tt = n_tok >= 5 ? 8 : (n_tok >= 3 ? 4 : static_cast<int>(n_tok));
+    for (;;) {
+        bool fits = false;
+        iqq_status s = IQQ_OK;
+        switch (tt) {
+        case 1: s = plan_and_launch<1>(P, st, fits); break;
+        case 2: s = plan_and_launch<2>(P, st, fits); break;
+        case 4: s = plan_and_launch<4>(P, st, fits); break;
+        default: s = plan_and_launch<8>(P, st, fits); break;
+        }
+        if (fits || s != IQQ_OK) return s;
         if (tt == 1) return IQQ_ERR_SHAPE;
         tt >>= 1;
-    }
-    switch (tt) {
-    case 1: return launch_tt<1>(P, st);
-    case 2: return launch_tt<2>(P, st);
-    case 4: return launch_tt<4>(P, st);
-    default: return launch_tt<8>(P, st);
     }
 }
