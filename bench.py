@@ -484,6 +484,27 @@ def main_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def profile_case(name: str):
+    """Small fixed cases for ncu captures (one GPU, a few launches, tens of MB)."""
+    import torch
+    import post_weight_quantization_rowwise_b200 as iqq
+    if name != "gemv_11008x4096":
+        raise SystemExit(f"unknown profile case {name}")
+    torch.manual_seed(0)
+    n_out, k = 11008, 4096
+    w = torch.randint(0, 256, (n_out * (k // 32) * 18,), dtype=torch.uint8, device="cuda")
+    w.view(-1, 18)[:, 1] &= 0x3B  # finite binary16 scales
+    a1 = iqq.quantize_q8_k128(torch.randn(1, k, device="cuda"))
+    a8 = iqq.quantize_q8_k128(torch.randn(8, k, device="cuda"))
+    y1 = torch.empty(1, n_out, device="cuda")
+    y8 = torch.empty(8, n_out, device="cuda")
+    for _ in range(4):
+        iqq.iqq_gemv_q4_0_q8_k128(w, a1, y1, k)
+    iqq.iqq_gemv_q4_0_q8_k128(w, a8, y8, k)
+    torch.cuda.synchronize()
+    print("ok", float(y1.abs().sum()), float(y8.abs().sum()))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,7 +517,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--profile-case", default=None, help="run one small ncu case and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
