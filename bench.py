@@ -278,6 +278,94 @@ def run_gemv_phase(iqq, w: Workload, dev, reps: int = 5):
     return ms, nbytes
 
 
+def _timed(fn, reps: int = 3):
+    """Device ms per call of fn (one untimed call first), CUDA events on the current stream."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
+    """The other formats, importance forms and the Q8_1 contrast, each measured once:
+      formats      Q4_0/Q5_0/Q6_0/Q8_0 weighted quantization, dequantization and weighted RMSE
+                   of the 8192^2 tensor of the scaling sweep (256 MB, beyond L2);
+      weight_modes the six importance forms on the same tensor (Q4_0);
+      sweep_ab     weight = qw against qw*sqrt(sigma2 + x^2) on every scaling-sweep tensor;
+      q8_1         Q8_1 against Q8_K_128 on the 4096x7168 activations with spikes."""
+    import torch
+    from post_weight_quantization_rowwise_b200 import synth
+    out = {}
+    sweep = synth.scaling_sweep()
+    t = sweep[1]
+    x, qw = t.weights(device=dev), t.qw(device=dev)
+    n = x.numel()
+    ops = Q4_0_OPS_BASE + Q4_0_OPS_PER_PASS * p_mean
+    fm = {}
+    for bits in (4, 5, 6, 8):
+        blocks = torch.empty(t.rows * (t.cols // 32) * iqq.QX_0_BLOCK_BYTES[bits], dtype=torch.uint8, device=dev)
+        y = torch.empty_like(x)
+        qms = _timed(lambda: iqq.iqq_quantize_qx_0_w(bits, x, qw, blocks))
+        dms = _timed(lambda: iqq.iqq_dequant_qx_0(bits, blocks, y))
+        acc = iqq.weighted_rmse_qx(bits, x, blocks, qw)
+        rms = _timed(lambda: iqq.iqq_weighted_rmse_qx(bits, x, blocks, qw, acc.zero_()))
+        a = acc.cpu().tolist()
+        dbytes = n * (4 + iqq.QX_0_BLOCK_BYTES[bits] / 32)
+        fm[f"q{bits}_0"] = {"quantize_gelem_s": round(n / qms / 1e6, 3),
+                            "quantize_frac": round(n * ops / (qms / 1e3) / 1e12 / peak_ops, 4),
+                            "dequant_gb_s": round(dbytes / dms / 1e6, 1),
+                            "dequant_hbm_frac": round(dbytes / dms / 1e6 / hbm_gbs, 4),
+                            "rmse_gb_s": round(dbytes / rms / 1e6, 1),
+                            "wrmse": math.sqrt(a[0] / a[1])}
+        del blocks, y
+    out["formats"] = {"tensor": t.name, "values": n, **fm}
+    blocks = torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8, device=dev)
+    wm = {}
+    for mode in range(6):
+        qms = _timed(lambda: iqq.iqq_quantize_q4_0_w(x, qw, blocks, 0, mode))
+        acc = iqq.weighted_rmse(x, blocks, qw)
+        a = acc.cpu().tolist()
+        wm[str(mode)] = {"gelem_s": round(n / qms / 1e6, 3), "wrmse": math.sqrt(a[0] / a[1])}
+    out["weight_modes"] = {"tensor": t.name, "modes": "0 qw*sqrt(s2+x2), 1 qw, 2 qw*x2, 3 qw*|x|, "
+                           "4 qw*(s2+x2), 5 qw*(sqrt(s2)+|x|)", **wm}
+    del x, qw, blocks
+    ab = {}
+    for tt in sweep:
+        x, qw = tt.weights(device=dev), tt.qw(device=dev)
+        blocks = torch.empty(tt.rows * (tt.cols // 32) * 18, dtype=torch.uint8, device=dev)
+        row = {}
+        for mode, name in ((1, "qw"), (0, "qw_sqrt_s2_x2")):
+            qms = _timed(lambda: iqq.iqq_quantize_q4_0_w(x, qw, blocks, 0, mode), reps=2)
+            a = iqq.weighted_rmse(x, blocks, qw).cpu().tolist()
+            row[name] = {"gelem_s": round(x.numel() / qms / 1e6, 3), "wrmse": math.sqrt(a[0] / a[1])}
+        ab[tt.name] = row
+        del x, qw, blocks
+    out["sweep_ab"] = ab
+    act = synth.activation_batch_4096x7168(device=dev)
+    q81 = torch.empty(act.numel() // 32 * 36, dtype=torch.uint8, device=dev)
+    q8k = torch.empty(act.numel() // 128 * 140, dtype=torch.uint8, device=dev)
+    over = torch.zeros(1, dtype=torch.int64, device=dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    iqq.iqq_quantize_q8_1(act, q81, over)
+    iqq.iqq_quantize_q8_k128(act, q8k, flags)
+    torch.cuda.synchronize()
+    n_over = int(over.item())
+    m1 = _timed(lambda: iqq.iqq_quantize_q8_1(act, q81))
+    mk = _timed(lambda: iqq.iqq_quantize_q8_k128(act, q8k))
+    na = act.numel()
+    out["q8_1"] = {"values": na, "blocks": na // 32, "overflowed_blocks": n_over,
+                   "q8_k128_nonfinite_flag": int(flags.item()),
+                   "q8_1_gb_s": round(na * (4 + 36 / 32) / m1 / 1e6, 1),
+                   "q8_k128_gb_s": round(na * (4 + 140 / 128) / mk / 1e6, 1)}
+    return out
+
+
 def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
     """Same step through the public API from pinned host buffers: per tensor H2D of x,
     the three kernels, D2H of the blocks; D2H of the accumulator at the end."""
@@ -383,6 +471,11 @@ def main_ours(args):
     gemv = None
     if not args.no_gemv:
         gemv = run_gemv_phase(iqq, w, dev)
+    extras = None
+    if rank == 0 and not args.no_extras:
+        pk0 = peaks()
+        extras = run_extras(iqq, dev, cpu[3] if cpu else 1.1,
+                            B200_SMS * FP32_LANES_PER_SM * pk0["sm_max_mhz"] * 1e6 / 1e12, pk0["hbm_gbs"])
 
     e2e = None
     if rank == 0 and world == 1 and not args.no_e2e:
@@ -440,6 +533,8 @@ def main_ours(args):
         "clocks": clk,
         "e2e": e2e,
     }
+    if extras is not None:
+        out["extras"] = extras
     if gemv is not None:
         gms, gbytes = gemv
         ggbs = gbytes / (gms / 1e3) / 1e9
@@ -517,6 +612,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--profile-case", default=None, help="run one small ncu case and exit")
     args = ap.parse_args()
     if args.profile_case:

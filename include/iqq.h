@@ -178,6 +178,15 @@ iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, int64_t nrow
                             void* stream);
 
 /*
+ * iqq_weighted_rmse_qx -- iqq_weighted_rmse for blocks of any of the 32-value formats
+ * written by iqq_quantize_qx_0_w (bits 4, 5, 6, 8; y = fp16(d) * code as
+ * iqq_dequant_qx_0).  Same arguments, accumulator and errors; bits outside {4, 5, 6, 8}
+ * return IQQ_ERR_ARG.
+ */
+iqq_status iqq_weighted_rmse_qx(int bits, const float* x, const void* blocks, const float* qw, int64_t nrows,
+                                int64_t n_per_row, int64_t rows_per_qw, double* d_acc, void* stream);
+
+/*
  * iqq_gemv_q4_0_q8_k128 -- y[t][r] = dot(dequant(W row r), dequant(A row t)): Q4_0 weight
  * rows times Q8_K_128 activation rows (a matrix-vector product per token).  [Q8]
  * 修复前的数值隐患 describes the consumer of the activation blocks: unsigned weight codes

@@ -225,6 +225,20 @@ def weighted_rmse(x, blocks, qw=None, rows_per_qw: int = 0, acc=None):
     return acc
 
 
+def weighted_rmse_qx(bits: int, x, blocks, qw=None, rows_per_qw: int = 0, acc=None):
+    """weighted_rmse for Q4_0/Q5_0/Q6_0/Q8_0 blocks (bits 4/5/6/8)."""
+    x = _f32(x)
+    nrows, n = x.shape
+    blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
+    qw = None if qw is None else _f32(qw)
+    acc = np.zeros(4, np.float64) if acc is None else acc
+    rc = lib().oracle_weighted_rmse_qx(bits, _ptr(x, _f32p), _ptr(blocks, _u8p), _ptr(qw, _f32p), nrows,
+                                       n, rows_per_qw, _ptr(acc, _f64p))
+    if rc != 0:
+        raise ValueError("oracle_weighted_rmse_qx: bad bits or shape")
+    return acc
+
+
 def quantize_q8_k128(x):
     """Quantize a [nrows, n_per_row] float32 matrix; returns (blocks uint8 [nrows, nb*140], flags)."""
     x = _f32(x)

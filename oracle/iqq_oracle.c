@@ -494,20 +494,21 @@ int oracle_dequant_q4_0(const uint8_t *blocks, float *y, int64_t nrows, int64_t 
 /* rounded once to binary32, and the sums are binary64:                 */
 /*   acc[0] += qw*e*e, acc[1] += qw, acc[2] += e*e, acc[3] = max |e|.   */
 /* acc accumulates (the caller zeroes it); wrmse = sqrt(acc0/acc1),     */
-/* rmse = sqrt(acc2/(nrows*n_per_row)).                                 */
-int oracle_weighted_rmse(const float *x, const uint8_t *blocks, const float *qw,
-                         int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, double *acc)
+/* rmse = sqrt(acc2/(nrows*n_per_row)).  Any of the 32-value formats    */
+/* (bits 4, 5, 6, 8), y = fp16(d) * code as oracle_dequant_qx_0.        */
+int oracle_weighted_rmse_qx(int bits, const float *x, const uint8_t *blocks, const float *qw,
+                            int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, double *acc)
 {
-    if (n_per_row % ORACLE_QK4_0 != 0) return -1;
-    const int64_t nb = n_per_row / ORACLE_QK4_0;
+    const int bb = oracle_qx_block_bytes(bits);
+    if (bb < 0 || n_per_row % 32 != 0) return -1;
+    const int64_t nb = n_per_row / 32;
     for (int64_t r = 0; r < nrows; ++r) {
         const float *qr = qw ? qw + (rows_per_qw > 0 ? r / rows_per_qw : 0) * n_per_row : NULL;
         for (int64_t b = 0; b < nb; ++b) {
-            const uint8_t *blk = blocks + (r * nb + b) * ORACLE_Q4_0_BYTES;
+            const uint8_t *blk = blocks + (r * nb + b) * bb;
             float d = oracle_fp16_to_float((uint16_t)(blk[0] | (blk[1] << 8)));
             for (int i = 0; i < 32; ++i) {
-                int nib = i < 16 ? (blk[2 + i] & 0xf) : (blk[2 + i - 16] >> 4);
-                float y = d * (float)(nib - 8);
+                float y = d * (float)unpack_code(bits, blk, i);
                 int64_t j = b * 32 + i;
                 float e = x[r * n_per_row + j] - y;
                 double ed = (double)e;
@@ -520,6 +521,13 @@ int oracle_weighted_rmse(const float *x, const uint8_t *blocks, const float *qw,
         }
     }
     return 0;
+}
+
+/* The Q4_0 form (18-byte blocks). */
+int oracle_weighted_rmse(const float *x, const uint8_t *blocks, const float *qw,
+                         int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, double *acc)
+{
+    return oracle_weighted_rmse_qx(4, x, blocks, qw, nrows, n_per_row, rows_per_qw, acc);
 }
 
 /* ------------------------------------------------------------------ */

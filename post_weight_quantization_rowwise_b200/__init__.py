@@ -49,6 +49,7 @@ def _load():
         "iqq_quantize_qx_0_w": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_dequant_qx_0": [ctypes.c_int, _vp, _vp, _i64, _i64, _vp],
         "iqq_gemv_q4_0_q8_k128": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+        "iqq_weighted_rmse_qx": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -267,6 +268,24 @@ def iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
     return acc
 
 
+def iqq_weighted_rmse_qx(bits, x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
+    """iqq_weighted_rmse for Q4_0/Q5_0/Q6_0/Q8_0 blocks (bits 4/5/6/8)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("blocks", blocks, torch.uint8)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("acc", acc, torch.float64)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits] or acc.numel() < 4:
+        raise ValueError("blocks or acc is too small")
+    _check("iqq_weighted_rmse_qx",
+           _lib.iqq_weighted_rmse_qx(bits, _ptr(x), _ptr(blocks), _ptr(qw), nrows, n, rows_per_qw, _ptr(acc),
+                                     _stream(stream)))
+    return acc
+
+
 # ----------------------------------------------------------------------------
 # conveniences
 # ----------------------------------------------------------------------------
@@ -319,6 +338,13 @@ def dequant_q4_0(blocks, nrows: int, n_per_row: int, stream=None):
     import torch
     y = torch.empty((nrows, n_per_row), dtype=torch.float32, device=blocks.device)
     return iqq_dequant_q4_0(blocks, y, stream)
+
+
+def weighted_rmse_qx(bits, x, blocks, qw=None, rows_per_qw: int = 0, stream=None):
+    """Returns the float64 accumulator [sum qw e^2, sum qw, sum e^2, max|e|] as a CUDA tensor."""
+    import torch
+    acc = torch.zeros(4, dtype=torch.float64, device=x.device)
+    return iqq_weighted_rmse_qx(bits, x, blocks, qw, acc, rows_per_qw, stream)
 
 
 def weighted_rmse(x, blocks, qw=None, rows_per_qw: int = 0, stream=None):

@@ -97,98 +97,6 @@ dequant_q4_0_kernel(const uint8_t* __restrict__ blocks, float4* __restrict__ y, 
 }
 
 // Adds the squared errors of one row's quad to the per-column accumulators.
-__device__ __forceinline__ void rmse_quad(const float4 xv, const Quad q, double (&col)[4], float& emax)
-{
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float xk = k == 0 ? xv.x : k == 1 ? xv.y : k == 2 ? xv.z : xv.w;
-        const float e = __fsub_rn(xk, __fmul_rn(q.d, code_value(q.nib4, k)));
-        emax = fmaxf(emax, fabsf(e));
-        const double ed = static_cast<double>(e);
-        col[k] = fma(ed, ed, col[k]);
-    }
-}
-
-// Rows [blockIdx.y*rows_per_cta, ...) x column quad blockIdx.x*kThreads + threadIdx.x.
-// Per column the thread keeps sum_r e^2 (binary64) and multiplies by qw once per
-// imatrix row, so qw is read and converted once per row segment, not per value.
-__global__ void __launch_bounds__(kThreads)
-weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ blocks,
-                     const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
-                     int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc)
-{
-    const int64_t nq = n_per_row / 4;
-    const int64_t nb = n_per_row / IQQ_Q4_0_BLOCK_VALUES;
-    const int64_t cq = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
-    const int64_t r1 = min(nrows, r0 + rows_per_cta);
-
-    double sw = 0.0, sq = 0.0, se = 0.0;
-    float emax = 0.0f;
-    if (cq < nq) {
-        const int64_t b = cq >> 3;
-        const int qd = static_cast<int>(cq & 7);
-        for (int64_t s0 = r0; s0 < r1;) {
-            // a segment of rows sharing one imatrix row
-            const int64_t qrow = rows_per_qw > 0 ? s0 / rows_per_qw : 0;
-            const int64_t s1 = rows_per_qw > 0 ? min(r1, (qrow + 1) * rows_per_qw) : r1;
-            double col[4] = {0.0, 0.0, 0.0, 0.0};
-            int64_t r = s0;
-            for (; r + kRowUnroll <= s1; r += kRowUnroll) {
-                float4 xv[kRowUnroll];
-                Quad q[kRowUnroll];
-#pragma unroll
-                for (int u = 0; u < kRowUnroll; ++u) {
-                    xv[u] = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + (r + u) * n_per_row) + cq);
-                    q[u] = load_quad(blocks + ((r + u) * nb + b) * IQQ_Q4_0_BLOCK_BYTES, qd);
-                }
-#pragma unroll
-                for (int u = 0; u < kRowUnroll; ++u) rmse_quad(xv[u], q[u], col, emax);
-            }
-            for (; r < s1; ++r) {
-                const float4 xv = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + r * n_per_row) + cq);
-                rmse_quad(xv, load_quad(blocks + (r * nb + b) * IQQ_Q4_0_BLOCK_BYTES, qd), col, emax);
-            }
-            float4 w = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
-            if (qw != nullptr) w = __ldg(reinterpret_cast<const float4*>(qw + qrow * n_per_row) + cq);
-            const double nr = static_cast<double>(s1 - s0);
-            sw = fma(static_cast<double>(w.x), col[0], sw);
-            sw = fma(static_cast<double>(w.y), col[1], sw);
-            sw = fma(static_cast<double>(w.z), col[2], sw);
-            sw = fma(static_cast<double>(w.w), col[3], sw);
-            se += (col[0] + col[1]) + (col[2] + col[3]);
-            sq = fma(static_cast<double>(w.x) + static_cast<double>(w.y) + static_cast<double>(w.z) +
-                         static_cast<double>(w.w), nr, sq);
-            s0 = s1;
-        }
-    }
-
-    // CTA reduction, then one atomic per quantity per CTA
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        sw += __shfl_xor_sync(0xffffffffu, sw, o);
-        sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        se += __shfl_xor_sync(0xffffffffu, se, o);
-        emax = fmaxf(emax, __shfl_xor_sync(0xffffffffu, emax, o));
-    }
-    __shared__ double s_w[kThreads / 32], s_q[kThreads / 32], s_e[kThreads / 32];
-    __shared__ float s_m[kThreads / 32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) { s_w[warp] = sw; s_q[warp] = sq; s_e[warp] = se; s_m[warp] = emax; }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double a = 0.0, bq = 0.0, c = 0.0;
-        float m = 0.0f;
-        for (int w = 0; w < kThreads / 32; ++w) { a += s_w[w]; bq += s_q[w]; c += s_e[w]; m = fmaxf(m, s_m[w]); }
-        atomicAdd(acc + 0, a);
-        atomicAdd(acc + 1, bq);
-        atomicAdd(acc + 2, c);
-        // non-negative binary64 values order like their bit patterns
-        atomicMax(reinterpret_cast<unsigned long long*>(acc + 3),
-                  static_cast<unsigned long long>(__double_as_longlong(static_cast<double>(m))));
-    }
-}
-
 // Q5_0 / Q6_0 / Q8_0 (layouts in iqq.h): the four codes of quad qd (values 4qd..4qd+3).
 template <int BITS>
 __device__ __forceinline__ void load_quad_qx(const uint8_t* blk, int qd, float& d, int (&c)[4])
@@ -242,6 +150,123 @@ dequant_qx_kernel(const uint8_t* __restrict__ blocks, float4* __restrict__ y, in
     }
 }
 
+// The scale and the four signed codes of quad qd of a block of any 32-value format.
+struct QuadC {
+    float d;
+    int c[4];
+};
+
+template <int BITS>
+__device__ __forceinline__ QuadC load_codes(const uint8_t* blk, int qd)
+{
+    QuadC q;
+    if (BITS == 4) {
+        const Quad n = load_quad(blk, qd);
+        q.d = n.d;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q.c[k] = static_cast<int>((n.nib4 >> (4 * k)) & 0xfu) - 8;
+    } else {
+        load_quad_qx<BITS>(blk, qd, q.d, q.c);
+    }
+    return q;
+}
+
+template <int BITS>
+__host__ __device__ constexpr int block_bytes() { return BITS == 4 ? 18 : (BITS == 5 ? 22 : (BITS == 6 ? 26 : 34)); }
+
+__device__ __forceinline__ void rmse_quad(const float4 xv, const QuadC q, double (&col)[4], float& emax)
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float xk = k == 0 ? xv.x : k == 1 ? xv.y : k == 2 ? xv.z : xv.w;
+        const float e = __fsub_rn(xk, __fmul_rn(q.d, static_cast<float>(q.c[k])));
+        emax = fmaxf(emax, fabsf(e));
+        const double ed = static_cast<double>(e);
+        col[k] = fma(ed, ed, col[k]);
+    }
+}
+
+// Rows [blockIdx.y*rows_per_cta, ...) x column quad blockIdx.x*kThreads + threadIdx.x.
+// Per column the thread keeps sum_r e^2 (binary64) and multiplies by qw once per
+// imatrix row, so qw is read and converted once per row segment, not per value.
+template <int BITS>
+__global__ void __launch_bounds__(kThreads)
+weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ blocks,
+                     const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
+                     int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc)
+{
+    const int64_t nq = n_per_row / 4;
+    const int64_t nb = n_per_row / IQQ_Q4_0_BLOCK_VALUES;
+    const int64_t cq = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
+    const int64_t r1 = min(nrows, r0 + rows_per_cta);
+
+    double sw = 0.0, sq = 0.0, se = 0.0;
+    float emax = 0.0f;
+    if (cq < nq) {
+        const int64_t b = cq >> 3;
+        const int qd = static_cast<int>(cq & 7);
+        for (int64_t s0 = r0; s0 < r1;) {
+            // a segment of rows sharing one imatrix row
+            const int64_t qrow = rows_per_qw > 0 ? s0 / rows_per_qw : 0;
+            const int64_t s1 = rows_per_qw > 0 ? min(r1, (qrow + 1) * rows_per_qw) : r1;
+            double col[4] = {0.0, 0.0, 0.0, 0.0};
+            int64_t r = s0;
+            for (; r + kRowUnroll <= s1; r += kRowUnroll) {
+                float4 xv[kRowUnroll];
+                QuadC q[kRowUnroll];
+#pragma unroll
+                for (int u = 0; u < kRowUnroll; ++u) {
+                    xv[u] = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + (r + u) * n_per_row) + cq);
+                    q[u] = load_codes<BITS>(blocks + ((r + u) * nb + b) * block_bytes<BITS>(), qd);
+                }
+#pragma unroll
+                for (int u = 0; u < kRowUnroll; ++u) rmse_quad(xv[u], q[u], col, emax);
+            }
+            for (; r < s1; ++r) {
+                const float4 xv = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + r * n_per_row) + cq);
+                rmse_quad(xv, load_codes<BITS>(blocks + (r * nb + b) * block_bytes<BITS>(), qd), col, emax);
+            }
+            float4 w = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            if (qw != nullptr) w = __ldg(reinterpret_cast<const float4*>(qw + qrow * n_per_row) + cq);
+            const double nr = static_cast<double>(s1 - s0);
+            sw = fma(static_cast<double>(w.x), col[0], sw);
+            sw = fma(static_cast<double>(w.y), col[1], sw);
+            sw = fma(static_cast<double>(w.z), col[2], sw);
+            sw = fma(static_cast<double>(w.w), col[3], sw);
+            se += (col[0] + col[1]) + (col[2] + col[3]);
+            sq = fma(static_cast<double>(w.x) + static_cast<double>(w.y) + static_cast<double>(w.z) +
+                         static_cast<double>(w.w), nr, sq);
+            s0 = s1;
+        }
+    }
+
+    // CTA reduction, then one atomic per quantity per CTA
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sw += __shfl_xor_sync(0xffffffffu, sw, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        se += __shfl_xor_sync(0xffffffffu, se, o);
+        emax = fmaxf(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+    }
+    __shared__ double s_w[kThreads / 32], s_q[kThreads / 32], s_e[kThreads / 32];
+    __shared__ float s_m[kThreads / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) { s_w[warp] = sw; s_q[warp] = sq; s_e[warp] = se; s_m[warp] = emax; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double a = 0.0, bq = 0.0, c = 0.0;
+        float m = 0.0f;
+        for (int w = 0; w < kThreads / 32; ++w) { a += s_w[w]; bq += s_q[w]; c += s_e[w]; m = fmaxf(m, s_m[w]); }
+        atomicAdd(acc + 0, a);
+        atomicAdd(acc + 1, bq);
+        atomicAdd(acc + 2, c);
+        // non-negative binary64 values order like their bit patterns
+        atomicMax(reinterpret_cast<unsigned long long*>(acc + 3),
+                  static_cast<unsigned long long>(__double_as_longlong(static_cast<double>(m))));
+    }
+}
+
 int sm_count()
 {
     int dev = 0, sms = 148;
@@ -291,9 +316,11 @@ extern "C" iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, i
     return iqq::launch_status();
 }
 
-extern "C" iqq_status iqq_weighted_rmse(const float* x, const void* blocks, const float* qw,
-                                        int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
-                                        double* d_acc, void* stream)
+namespace {
+
+template <int BITS>
+iqq_status rmse_launch(const float* x, const void* blocks, const float* qw, int64_t nrows, int64_t n_per_row,
+                       int64_t rows_per_qw, double* d_acc, void* stream)
 {
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
     if (n_per_row % IQQ_Q4_0_BLOCK_VALUES != 0) return IQQ_ERR_SHAPE;
@@ -313,8 +340,30 @@ extern "C" iqq_status iqq_weighted_rmse(const float* x, const void* blocks, cons
     gy = (nrows + rpc - 1) / rpc;
     if (gx > 0x7fffffff || gy > 65535) return IQQ_ERR_SHAPE;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-    weighted_rmse_kernel<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+    weighted_rmse_kernel<BITS><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         x, static_cast<const uint8_t*>(blocks), qw, nrows, n_per_row, rows_per_qw,
         static_cast<int>(rpc), d_acc);
     return iqq::launch_status();
+}
+
+}  // namespace
+
+extern "C" iqq_status iqq_weighted_rmse(const float* x, const void* blocks, const float* qw,
+                                        int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                        double* d_acc, void* stream)
+{
+    return rmse_launch<4>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+}
+
+extern "C" iqq_status iqq_weighted_rmse_qx(int bits, const float* x, const void* blocks, const float* qw,
+                                           int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                           double* d_acc, void* stream)
+{
+    switch (bits) {
+    case 4: return rmse_launch<4>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+    case 5: return rmse_launch<5>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+    case 6: return rmse_launch<6>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+    case 8: return rmse_launch<8>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+    default: return IQQ_ERR_ARG;
+    }
 }

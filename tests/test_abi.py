@@ -26,7 +26,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("iqq_quantize_q4_0_w", "iqq_quantize_q8_k128", "iqq_dequant_q4_0",
               "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string",
-              "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128"):
+              "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128",
+              "iqq_weighted_rmse_qx"):
         assert n in names
 
 
@@ -83,6 +84,12 @@ def test_host_validation_without_gpu(lib):
         assert lib.iqq_dequant_qx_0(bits, V(16), V(16), 2, 48, None) == 2
         assert lib.iqq_dequant_qx_0(bits, None, V(16), 1, 32, None) == 1
         assert lib.iqq_dequant_qx_0(bits, V(16), V(8), 1, 32, None) == 3
+    for bits in (3, 7):
+        assert lib.iqq_weighted_rmse_qx(bits, V(16), V(16), None, 1, 32, 0, V(16), None) == 5
+    for bits in (4, 5, 6, 8):
+        assert lib.iqq_weighted_rmse_qx(bits, V(16), V(16), None, 2, 48, 0, V(16), None) == 2
+        assert lib.iqq_weighted_rmse_qx(bits, V(16), V(16), None, 1, 32, 0, V(4), None) == 3
+        assert lib.iqq_weighted_rmse_qx(bits, None, None, None, 0, 32, 0, None, None) == 0
     # Q4_0 x Q8_K_128 matrix-vector product
     G = lib.iqq_gemv_q4_0_q8_k128
     assert G(V(16), V(16), V(16), 4, 96, 1, None, None) == 2          # k not a multiple of 128

@@ -218,6 +218,12 @@ def test_qx_0_weighted_and_dequant(iqq, synth, bits, rows, n):
     assert same.mean() >= 0.9999
     # dequantization of the GPU's blocks is bit-exact against the oracle's decoder
     assert np.array_equal(y.cpu().numpy(), oracle.dequant_qx_0(bits, g.cpu().numpy(), rows, n))
+    # the weighted RMSE of the GPU's blocks against the oracle's reduction of the same blocks
+    acc = iqq.weighted_rmse_qx(bits, xd, g, qd)
+    torch.cuda.synchronize()
+    ref = oracle.weighted_rmse_qx(bits, x, g.cpu().numpy(), qw)
+    a = acc.cpu().numpy()
+    assert np.allclose(a[:3], ref[:3], rtol=1e-9, atol=0) and a[3] == ref[3]
     # any differing block: weighted error within 1e-5 of the oracle's
     if not same.all():
         yo = oracle.dequant_qx_0(bits, o, rows, n).reshape(-1, 32).astype(np.float64)

@@ -24,6 +24,8 @@ def _pack(bits, d, codes, orc):
     if bits == 8:
         return bytes(head + [c & 0xFF for c in codes])
     n = [c + nmax for c in codes]
+    if bits == 4:
+        return bytes(head + [n[i] | (n[i + 16] << 4) for i in range(16)])
     if bits == 5:
         qh = sum(((v >> 4) & 1) << j for j, v in enumerate(n))
         hb = qh.to_bytes(4, "little")
@@ -155,3 +157,29 @@ def test_more_bits_less_error(orc):
         y = orc.dequant_qx_0(bits, out, 32, 512)
         errs.append(float(np.sum(qw * (x - y).astype(np.float64) ** 2)))
     assert errs[0] > errs[1] > errs[2] > errs[3]
+
+
+def test_weighted_rmse_closed_form(orc):
+    """Hand-built blocks of every format with x = y + delta, delta exactly representable:
+    the accumulator equals the exact sums of qw e^2, qw, e^2 and max |e|; bits = 4 is the
+    separately pinned Q4_0 reduction."""
+    from fractions import Fraction
+    rng = np.random.default_rng(60)
+    for bits in (4, 5, 6, 8):
+        nmax = orc.NMAX[bits]
+        d0 = 2.0 ** -5
+        codes = rng.integers(-nmax, nmax, (3, 32))
+        blk = np.stack([np.frombuffer(_pack(bits, d0, c.tolist(), orc), np.uint8) for c in codes])
+        delta = (rng.integers(-64, 65, (3, 32)) * 2.0 ** -12).astype(np.float32)
+        x = (codes * np.float32(d0)).astype(np.float32) + delta     # exact in binary32
+        qw = (rng.integers(1, 9, 32) * 0.25).astype(np.float32)
+        acc = orc.weighted_rmse_qx(bits, x.reshape(1, 96), blk.reshape(1, -1), np.tile(qw, 3))
+        e = [Fraction(float(v)) for v in delta.reshape(-1)]
+        q = [Fraction(float(v)) for v in np.tile(qw, 3)]
+        assert Fraction(acc[0]) == sum(qi * ei * ei for qi, ei in zip(q, e))
+        assert Fraction(acc[1]) == sum(q)
+        assert Fraction(acc[2]) == sum(ei * ei for ei in e)
+        assert acc[3] == float(np.abs(delta).max())
+        if bits == 4:
+            ref = orc.weighted_rmse(x.reshape(1, 96), blk.reshape(1, -1), np.tile(qw, 3))
+            assert np.array_equal(acc, ref)
