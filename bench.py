@@ -339,13 +339,19 @@ def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
     for tt in sweep:
         x, qw = tt.weights(device=dev), tt.qw(device=dev)
         blocks = torch.empty(tt.rows * (tt.cols // 32) * 18, dtype=torch.uint8, device=dev)
-        row = {}
+        nws = iqq.qx_0_w_workspace_bytes(tt.rows, tt.cols)
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+        row = {"workspace_bytes": nws}
         for mode, name in ((1, "qw"), (0, "qw_sqrt_s2_x2")):
-            qms = _timed(lambda: iqq.iqq_quantize_q4_0_w(x, qw, blocks, 0, mode), reps=2)
+            qms = _timed(lambda: iqq.iqq_quantize_qx_0_w_ws(4, x, qw, blocks, ws, 0, mode), reps=2)
             a = iqq.weighted_rmse(x, blocks, qw).cpu().tolist()
             row[name] = {"gelem_s": round(x.numel() / qms / 1e6, 3), "wrmse": math.sqrt(a[0] / a[1])}
+        if nws:
+            # the same tensor without the workspace (the fused per-CTA row reduction)
+            qms = _timed(lambda: iqq.iqq_quantize_q4_0_w(x, qw, blocks, 0, 0), reps=2)
+            row["qw_sqrt_s2_x2_fused"] = {"gelem_s": round(x.numel() / qms / 1e6, 3)}
         ab[tt.name] = row
-        del x, qw, blocks
+        del x, qw, blocks, ws
     out["sweep_ab"] = ab
     act = synth.activation_batch_4096x7168(device=dev)
     q81 = torch.empty(act.numel() // 32 * 36, dtype=torch.uint8, device=dev)

@@ -36,6 +36,7 @@
 #ifndef IQQ_H
 #define IQQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -119,6 +120,39 @@ iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64
 iqq_status iqq_quantize_qx_0_w(int bits, const float* x, const float* qw, void* out, int64_t nrows,
                                int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
                                uint32_t* d_flags, void* stream);
+
+/*
+ * iqq_quantize_qx_0_w_ws -- iqq_quantize_qx_0_w with a caller-owned device workspace for
+ * wide rows.  A row spanning at least 4 CTAs of the quantizer (n_per_row > 12288) has its
+ * sigma2 computed once by a separate per-row pass into the workspace (nrows floats),
+ * instead of once per CTA of the row; the binary64 sum of exact squares and its rounding are
+ * those of iqq_quantize_qx_0_w (only the summation order can differ, as there), and the
+ * pass reports IQQ_FLAG_NONFINITE_INPUT.  Narrower rows need no workspace and take the
+ * fused path.
+ *  workspace        device memory of at least iqq_quantize_qx_0_w_workspace_bytes(nrows,
+ *                   n_per_row) bytes, 16-byte aligned; may be NULL when that size is 0.
+ *                   Overwritten; free for reuse once the stream has passed the call.
+ *  workspace_bytes  its size.  Too small: IQQ_ERR_SHAPE; NULL when needed: IQQ_ERR_NULL.
+ * Other arguments and errors as for iqq_quantize_qx_0_w.
+ */
+size_t iqq_quantize_qx_0_w_workspace_bytes(int64_t nrows, int64_t n_per_row);
+iqq_status iqq_quantize_qx_0_w_ws(int bits, const float* x, const float* qw, void* out, int64_t nrows,
+                                  int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
+                                  size_t workspace_bytes, uint32_t* d_flags, void* stream);
+
+/*
+ * iqq_quantize_qx_0_w_static -- iqq_quantize_qx_0_w_ws without a caller workspace: the
+ * per-row sigma2 of wide rows goes to a library-owned device array of IQQ_STATIC_WS_ROWS
+ * floats (a file-scope __device__ variable, one per device; nothing is allocated), and
+ * tensors with more rows are processed in batches of that many rows.  Results are
+ * identical to iqq_quantize_qx_0_w_ws.  The array is shared by every call on a device, so
+ * calls must be ordered (one stream, or synchronized); concurrent calls on different
+ * streams of one device are not supported.  Arguments and errors as iqq_quantize_qx_0_w.
+ */
+#define IQQ_STATIC_WS_ROWS 16384
+iqq_status iqq_quantize_qx_0_w_static(int bits, const float* x, const float* qw, void* out, int64_t nrows,
+                                      int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                                      uint32_t* d_flags, void* stream);
 
 /*
  * iqq_quantize_q8_k128 -- Q8_K_128 activation quantization, [Q8] 修复方案:

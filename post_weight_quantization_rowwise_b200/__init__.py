@@ -50,6 +50,9 @@ def _load():
         "iqq_dequant_qx_0": [ctypes.c_int, _vp, _vp, _i64, _i64, _vp],
         "iqq_gemv_q4_0_q8_k128": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
         "iqq_weighted_rmse_qx": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+        "iqq_quantize_qx_0_w_ws": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
+                                   ctypes.c_size_t, _vp, _vp],
+        "iqq_quantize_qx_0_w_static": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -62,6 +65,8 @@ def _load():
     lib.iqq_last_cuda_error.restype = ctypes.c_int
     lib.iqq_version.argtypes = []
     lib.iqq_version.restype = ctypes.c_char_p
+    lib.iqq_quantize_qx_0_w_workspace_bytes.restype = ctypes.c_size_t
+    lib.iqq_quantize_qx_0_w_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
     return lib
 
 
@@ -190,6 +195,33 @@ def iqq_dequant_qx_0(bits, blocks, y, stream=None):
     return y
 
 
+def qx_0_w_workspace_bytes(nrows: int, n_per_row: int) -> int:
+    """Device workspace iqq_quantize_qx_0_w_ws needs (0: none)."""
+    return int(_lib.iqq_quantize_qx_0_w_workspace_bytes(nrows, n_per_row))
+
+
+def iqq_quantize_qx_0_w_ws(bits, x, qw, out, workspace, rows_per_qw: int = 0, weight_mode: int = 0,
+                           flags=None, stream=None):
+    """iqq_quantize_qx_0_w with a device workspace (uint8 tensor of at least
+    qx_0_w_workspace_bytes bytes, or None when that is 0) for rows spanning many CTAs."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("workspace", workspace, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
+        raise ValueError("out is too small")
+    nbytes = 0 if workspace is None else workspace.numel()
+    _check("iqq_quantize_qx_0_w_ws",
+           _lib.iqq_quantize_qx_0_w_ws(bits, _ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw, weight_mode,
+                                       _ptr(workspace), nbytes, _ptr(flags), _stream(stream)))
+    return out
+
+
 def iqq_quantize_q8_k128(x, out, flags=None, stream=None):
     """Q8_K_128 blocks of x [nrows, n_per_row] float32 into out (uint8, q8_k128_nbytes)."""
     import torch
@@ -313,6 +345,36 @@ def quantize_qx_0_w(bits, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0
     nrows, n = _shape2(x)
     out = torch.empty((nrows, (n // 32) * QX_0_BLOCK_BYTES[bits]), dtype=torch.uint8, device=x.device)
     return iqq_quantize_qx_0_w(bits, x, qw, out, rows_per_qw, weight_mode, flags, stream)
+
+
+def iqq_quantize_qx_0_w_static(bits, x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,
+                               stream=None):
+    """iqq_quantize_qx_0_w_ws with the library's own static workspace (allocates nothing)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
+        raise ValueError("out is too small")
+    _check("iqq_quantize_qx_0_w_static",
+           _lib.iqq_quantize_qx_0_w_static(bits, _ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw,
+                                           weight_mode, _ptr(flags), _stream(stream)))
+    return out
+
+
+def quantize_qx_0_w_ws(bits, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,
+                       stream=None):
+    """quantize_qx_0_w through the workspace entry point (the workspace is allocated here)."""
+    import torch
+    nrows, n = _shape2(x)
+    out = torch.empty((nrows, (n // 32) * QX_0_BLOCK_BYTES[bits]), dtype=torch.uint8, device=x.device)
+    nb = qx_0_w_workspace_bytes(nrows, n)
+    ws = torch.empty(nb, dtype=torch.uint8, device=x.device) if nb else None
+    return iqq_quantize_qx_0_w_ws(bits, x, qw, out, ws, rows_per_qw, weight_mode, flags, stream)
 
 
 def dequant_qx_0(bits, blocks, nrows: int, n_per_row: int, stream=None):

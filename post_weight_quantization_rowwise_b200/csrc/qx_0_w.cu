@@ -254,7 +254,7 @@ template <int BITS>
 __global__ void __launch_bounds__(kThreads, IQQ_Q4_MIN_CTAS)
 qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
-              int chunks_per_row, uint32_t* __restrict__ flags)
+              int chunks_per_row, const float* __restrict__ row_sigma2, uint32_t* __restrict__ flags)
 {
     extern __shared__ float smem[];
     __shared__ double s_red[kWarps];
@@ -308,24 +308,30 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
             for (int i = 0; i < QK / 4; ++i) q4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
 
-        // sigma2: binary64 sum of exact squares over the whole row
-        double acc = 0.0;
-        float nf = 0.0f;
-        const float4* xr4 = reinterpret_cast<const float4*>(xr);
-        for (int64_t i = threadIdx.x; i < n_per_row / 4; i += kThreads) {
-            const float4 v = __ldg(xr4 + i);
-            acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
-            acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
-            acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
-            acc = fma(static_cast<double>(v.w), static_cast<double>(v.w), acc);
-            nf = __fmaf_rn(v.x, 0.0f, nf);  // becomes NaN on any Inf/NaN
-            nf = __fmaf_rn(v.y, 0.0f, nf);
-            nf = __fmaf_rn(v.z, 0.0f, nf);
-            nf = __fmaf_rn(v.w, 0.0f, nf);
+        // sigma2: binary64 sum of exact squares over the whole row -- reduced here, or
+        // read from the per-row pass (which also reports non-finite x)
+        float sigma2;
+        if (row_sigma2 != nullptr) {
+            sigma2 = __ldg(row_sigma2 + row);
+        } else {
+            double acc = 0.0;
+            float nf = 0.0f;
+            const float4* xr4 = reinterpret_cast<const float4*>(xr);
+            for (int64_t i = threadIdx.x; i < n_per_row / 4; i += kThreads) {
+                const float4 v = __ldg(xr4 + i);
+                acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
+                acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
+                acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
+                acc = fma(static_cast<double>(v.w), static_cast<double>(v.w), acc);
+                nf = __fmaf_rn(v.x, 0.0f, nf);  // becomes NaN on any Inf/NaN
+                nf = __fmaf_rn(v.y, 0.0f, nf);
+                nf = __fmaf_rn(v.z, 0.0f, nf);
+                nf = __fmaf_rn(v.w, 0.0f, nf);
+            }
+            if (chunk == 0 && nf != nf) bad |= IQQ_FLAG_NONFINITE_INPUT;
+            const double sum = block_reduce_sum(acc, s_red);
+            sigma2 = static_cast<float>(sum / static_cast<double>(n_per_row));
         }
-        if (chunk == 0 && nf != nf) bad |= IQQ_FLAG_NONFINITE_INPUT;
-        const double sum = block_reduce_sum(acc, s_red);
-        const float sigma2 = static_cast<float>(sum / static_cast<double>(n_per_row));
 
         if (valid && qr != nullptr && (rows_per_qw > 0 ? row % rows_per_qw == 0 : row == 0)) {
             float qmin = q4[0].x, qnf = 0.0f;
@@ -535,9 +541,70 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
 
 constexpr size_t kDynSmem = sizeof(float) * kWarpFloats * kWarps;
 
+// Rows spanning at least this many CTAs take sigma2 from a separate per-row pass when the
+// caller provides a workspace: below it the fused reduction's re-reads of the row (from L2,
+// once per chunk) cost less than a second pass over the tensor.
+#ifndef IQQ_PREPASS_CHUNKS
+#define IQQ_PREPASS_CHUNKS 4
+#endif
+constexpr int64_t kPrepassChunks = IQQ_PREPASS_CHUNKS;
+constexpr int kPrepassThreads = 256;
+
+// sigma2 of each row (the same binary64 sum of exact squares and rounding as the fused
+// reduction), one CTA per row, and the non-finite check of x.
+__global__ void __launch_bounds__(kPrepassThreads)
+row_sigma2_kernel(const float* __restrict__ x, int64_t nrows, int64_t n_per_row, float* __restrict__ out,
+                  uint32_t* __restrict__ flags)
+{
+    __shared__ double s_red[kPrepassThreads / 32];
+    for (int64_t row = blockIdx.x; row < nrows; row += gridDim.x) {
+        const float4* xr4 = reinterpret_cast<const float4*>(x + row * n_per_row);
+        double acc = 0.0;
+        float nf = 0.0f;
+        for (int64_t i = threadIdx.x; i < n_per_row / 4; i += kPrepassThreads) {
+            const float4 v = iqq::ld_stream_f4(xr4 + i);
+            acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
+            acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
+            acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
+            acc = fma(static_cast<double>(v.w), static_cast<double>(v.w), acc);
+            nf = __fmaf_rn(v.x, 0.0f, nf);
+            nf = __fmaf_rn(v.y, 0.0f, nf);
+            nf = __fmaf_rn(v.z, 0.0f, nf);
+            nf = __fmaf_rn(v.w, 0.0f, nf);
+        }
+        iqq::raise_flags(flags, nf != nf ? IQQ_FLAG_NONFINITE_INPUT : 0u);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        if (lane == 0) s_red[warp] = acc;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t = 0.0;
+#pragma unroll
+            for (int w = 0; w < kPrepassThreads / 32; ++w) t += s_red[w];
+            out[row] = static_cast<float>(t / static_cast<double>(n_per_row));
+        }
+        __syncthreads();
+    }
+}
+
+int64_t chunks_of(int64_t n_per_row) { return (n_per_row / QK + kThreads - 1) / kThreads; }
+
+// Library-owned sigma2 rows for iqq_quantize_qx_0_w_static (one copy per device; calls that
+// use it are ordered by their stream, so concurrent calls on different streams must not
+// share a device).
+static __device__ __align__(256) float g_static_sigma2[IQQ_STATIC_WS_ROWS];
+
+int64_t workspace_bytes_for(int64_t nrows, int64_t n_per_row)
+{
+    if (nrows <= 0 || n_per_row <= 0 || chunks_of(n_per_row) < kPrepassChunks) return 0;
+    return (nrows * 4 + 255) / 256 * 256;
+}
+
 template <int BITS>
 iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
-                     int64_t rows_per_qw, int weight_mode, uint32_t* d_flags, void* stream)
+                     int64_t rows_per_qw, int weight_mode, const float* row_sigma2, uint32_t* d_flags,
+                     void* stream)
 {
     const int64_t nb = n_per_row / QK;
     const int64_t chunks = (nb + kThreads - 1) / kThreads;
@@ -555,13 +622,15 @@ iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, 
     }
     qx_0_w_kernel<BITS><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
         x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode,
-        static_cast<int>(chunks), d_flags);
+        static_cast<int>(chunks), row_sigma2, d_flags);
     return iqq::launch_status();
 }
 
+// workspace == nullptr: the fused reduction.  Otherwise it holds at least
+// workspace_bytes_for(nrows, n_per_row) bytes (checked by the caller).
 iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int64_t nrows,
-                       int64_t n_per_row, int64_t rows_per_qw, int weight_mode, uint32_t* d_flags,
-                       void* stream)
+                       int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
+                       uint32_t* d_flags, void* stream)
 {
     if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
@@ -572,11 +641,21 @@ iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int
     if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||
         (d_flags && !iqq::aligned(d_flags, 4)))
         return IQQ_ERR_ALIGN;
+    const float* rs = nullptr;
+    if (workspace != nullptr && workspace_bytes_for(nrows, n_per_row) > 0) {
+        float* ws = static_cast<float*>(workspace);
+        const int64_t g = nrows < 0x7fffffff ? nrows : 0x7fffffff;
+        row_sigma2_kernel<<<static_cast<int>(g), kPrepassThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+            x, nrows, n_per_row, ws, d_flags);
+        const iqq_status st = iqq::launch_status();
+        if (st != IQQ_OK) return st;
+        rs = ws;
+    }
     switch (bits) {
-    case 4: return launch_qx<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
-    case 5: return launch_qx<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
-    case 6: return launch_qx<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
-    default: return launch_qx<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    case 4: return launch_qx<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
+    case 5: return launch_qx<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
+    case 6: return launch_qx<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
+    default: return launch_qx<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
     }
 }
 
@@ -586,12 +665,81 @@ extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void*
                                           int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
                                           uint32_t* d_flags, void* stream)
 {
-    return quantize_qx(4, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    return quantize_qx(4, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, nullptr, d_flags, stream);
 }
 
 extern "C" iqq_status iqq_quantize_qx_0_w(int bits, const float* x, const float* qw, void* out,
                                           int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
                                           int weight_mode, uint32_t* d_flags, void* stream)
 {
-    return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, d_flags, stream);
+    return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, nullptr, d_flags, stream);
+}
+
+extern "C" iqq_status iqq_quantize_qx_0_w_static(int bits, const float* x, const float* qw, void* out,
+                                                 int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                                 int weight_mode, uint32_t* d_flags, void* stream)
+{
+    if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
+    if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0 || n_per_row % QK != 0) return IQQ_ERR_SHAPE;
+    if (workspace_bytes_for(nrows, n_per_row) == 0)  // no per-row pass: the fused path
+        return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, nullptr, d_flags,
+                           stream);
+    if (weight_mode < 0 || weight_mode > 5) return IQQ_ERR_ARG;
+    if (x == nullptr || out == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||
+        (d_flags && !iqq::aligned(d_flags, 4)))
+        return IQQ_ERR_ALIGN;  // every host check before the first CUDA call
+    void* ws = nullptr;
+    if (cudaGetSymbolAddress(&ws, g_static_sigma2) != cudaSuccess) return iqq::launch_status();
+    // row batches that fit the static rows; each batch is a tensor of its own rows (the
+    // imatrix row of a batch row follows from its global index)
+    const int64_t bb = bits == 4 ? Fmt<4>::bytes : bits == 5 ? Fmt<5>::bytes : bits == 6 ? Fmt<6>::bytes : Fmt<8>::bytes;
+    for (int64_t r0 = 0; r0 < nrows; r0 += IQQ_STATIC_WS_ROWS) {
+        const int64_t nr = nrows - r0 < IQQ_STATIC_WS_ROWS ? nrows - r0 : IQQ_STATIC_WS_ROWS;
+        const float* qb = qw;
+        if (qw != nullptr && rows_per_qw > 0) {
+            // a batch starts on an imatrix-row boundary only if IQQ_STATIC_WS_ROWS is a
+            // multiple of rows_per_qw; otherwise quantize the batch row by imatrix segment
+            if (IQQ_STATIC_WS_ROWS % rows_per_qw != 0) {
+                for (int64_t s0 = r0; s0 < r0 + nr;) {
+                    const int64_t q = s0 / rows_per_qw;
+                    const int64_t s1 = (q + 1) * rows_per_qw < r0 + nr ? (q + 1) * rows_per_qw : r0 + nr;
+                    const iqq_status st = quantize_qx(bits, x + s0 * n_per_row, qw + q * n_per_row,
+                                                      static_cast<uint8_t*>(out) + s0 * (n_per_row / QK) * bb,
+                                                      s1 - s0, n_per_row, 0, weight_mode, ws, d_flags, stream);
+                    if (st != IQQ_OK) return st;
+                    s0 = s1;
+                }
+                continue;
+            }
+            qb = qw + (r0 / rows_per_qw) * n_per_row;
+        }
+        const iqq_status st = quantize_qx(bits, x + r0 * n_per_row, qb,
+                                          static_cast<uint8_t*>(out) + r0 * (n_per_row / QK) * bb, nr, n_per_row,
+                                          rows_per_qw, weight_mode, ws, d_flags, stream);
+        if (st != IQQ_OK) return st;
+    }
+    return IQQ_OK;
+}
+
+extern "C" size_t iqq_quantize_qx_0_w_workspace_bytes(int64_t nrows, int64_t n_per_row)
+{
+    return static_cast<size_t>(workspace_bytes_for(nrows, n_per_row));
+}
+
+extern "C" iqq_status iqq_quantize_qx_0_w_ws(int bits, const float* x, const float* qw, void* out,
+                                             int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                             int weight_mode, void* workspace, size_t workspace_bytes,
+                                             uint32_t* d_flags, void* stream)
+{
+    if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
+    if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0 || n_per_row % QK != 0) return IQQ_ERR_SHAPE;
+    const int64_t need = workspace_bytes_for(nrows, n_per_row);
+    if (need > 0) {
+        if (workspace == nullptr) return IQQ_ERR_NULL;
+        if (workspace_bytes < static_cast<size_t>(need)) return IQQ_ERR_SHAPE;
+        if (!iqq::aligned(workspace, 16)) return IQQ_ERR_ALIGN;
+    }
+    return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode,
+                       need > 0 ? workspace : nullptr, d_flags, stream);
 }

@@ -27,7 +27,8 @@ def test_header_declares_the_boundary():
     for n in ("iqq_quantize_q4_0_w", "iqq_quantize_q8_k128", "iqq_dequant_q4_0",
               "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string",
               "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128",
-              "iqq_weighted_rmse_qx"):
+              "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
+              "iqq_quantize_qx_0_w_static"):
         assert n in names
 
 
@@ -90,6 +91,27 @@ def test_host_validation_without_gpu(lib):
         assert lib.iqq_weighted_rmse_qx(bits, V(16), V(16), None, 2, 48, 0, V(16), None) == 2
         assert lib.iqq_weighted_rmse_qx(bits, V(16), V(16), None, 1, 32, 0, V(4), None) == 3
         assert lib.iqq_weighted_rmse_qx(bits, None, None, None, 0, 32, 0, None, None) == 0
+    # workspace variant: size rule, and the workspace checks
+    WB = lib.iqq_quantize_qx_0_w_workspace_bytes
+    WB.restype = ctypes.c_size_t
+    WB.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    assert WB(10, 4096) == 0 and WB(10, 12288) == 0       # 3 CTAs per row: fused
+    assert WB(10, 12320) == 256 and WB(100, 53248) == 512  # 4 and 13 CTAs per row
+    assert WB(0, 53248) == 0
+    Q = lib.iqq_quantize_qx_0_w_ws
+    assert Q(4, V(16), None, V(16), 2, 53248, 0, 0, None, 0, None, None) == 1
+    assert Q(4, V(16), None, V(16), 2, 53248, 0, 0, V(16), 8, None, None) == 2
+    assert Q(4, V(16), None, V(16), 2, 53248, 0, 0, V(8), 256, None, None) == 3
+    assert Q(7, V(16), None, V(16), 2, 53248, 0, 0, V(16), 256, None, None) == 5
+    assert Q(4, V(16), None, V(16), 2, 4096, 0, 9, None, 0, None, None) == 5  # no workspace needed
+    assert Q(4, None, None, None, 0, 4096, 0, 0, None, 0, None, None) == 0
+    S = lib.iqq_quantize_qx_0_w_static
+    assert S(3, V(16), None, V(16), 2, 53248, 0, 0, None, None) == 5
+    assert S(4, V(16), None, V(16), 2, 53248 + 16, 0, 0, None, None) == 2
+    assert S(4, None, None, V(16), 2, 53248, 0, 0, None, None) == 1
+    assert S(4, V(16), None, V(16), 2, 53248, 0, 7, None, None) == 5
+    assert S(4, V(8), None, V(16), 2, 53248, 0, 0, None, None) == 3
+    assert S(4, None, None, None, 0, 53248, 0, 0, None, None) == 0
     # Q4_0 x Q8_K_128 matrix-vector product
     G = lib.iqq_gemv_q4_0_q8_k128
     assert G(V(16), V(16), V(16), 4, 96, 1, None, None) == 2          # k not a multiple of 128

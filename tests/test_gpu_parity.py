@@ -237,6 +237,55 @@ def test_qx_0_weighted_and_dequant(iqq, synth, bits, rows, n):
             assert abs(eg - eo) <= 1e-5 * eo
 
 
+def _compare_qx(bits, x, qw, g, o, rows, n, min_exact=0.9999):
+    bb = oracle.qx_block_bytes(bits)
+    gb = g.reshape(-1, bb)
+    ob = o.reshape(-1, bb)
+    same = np.all(gb == ob, axis=1)
+    assert same.mean() >= min_exact, same.mean()
+    if not same.all():
+        yo = oracle.dequant_qx_0(bits, o, rows, n).reshape(-1, 32).astype(np.float64)
+        yg = oracle.dequant_qx_0(bits, g, rows, n).reshape(-1, 32).astype(np.float64)
+        xb = x.reshape(-1, 32).astype(np.float64)
+        for i in np.nonzero(~same)[0]:
+            r, c = divmod(int(i), n // 32)
+            w = oracle.block_weights(x[r, 32 * c:32 * c + 32], qw[32 * c:32 * c + 32],
+                                     oracle.row_sigma2(x[r]), 0).astype(np.float64)
+            eg, eo = np.sum(w * (xb[i] - yg[i]) ** 2), np.sum(w * (xb[i] - yo[i]) ** 2)
+            assert abs(eg - eo) <= 1e-5 * eo
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("rows,n", [(3, 53248), (5, 16416), (2, 12320)])
+def test_qx_0_workspace_wide_rows(iqq, synth, bits, rows, n):
+    """Rows spanning 4 or more CTAs: sigma2 from the per-row pass into the workspace."""
+    assert iqq.qx_0_w_workspace_bytes(rows, n) > 0
+    x = synth.weight_matrix(rows, n, seed=rows + n + bits).numpy()
+    qw = synth.imatrix(n, seed=n + 1).numpy()
+    xd, qd = torch.from_numpy(x).cuda(), torch.from_numpy(qw).cuda()
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g_ws = iqq.quantize_qx_0_w_ws(bits, xd, qd, flags=flags)
+    g_fused = iqq.quantize_qx_0_w(bits, xd, qd)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    o, _ = oracle.quantize_qx_0_w(bits, x, qw)
+    _compare_qx(bits, x, qw, g_ws.cpu().numpy(), o, rows, n)
+    assert np.mean(np.all(g_ws.cpu().numpy().reshape(-1, oracle.qx_block_bytes(bits)) ==
+                          g_fused.cpu().numpy().reshape(-1, oracle.qx_block_bytes(bits)), axis=1)) >= 0.9999
+
+
+def test_qx_0_workspace_flags_nonfinite(iqq, synth):
+    x = synth.weight_matrix(2, 53248, seed=1)
+    x[1, 40000] = float("inf")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = iqq.quantize_qx_0_w_ws(4, x.cuda(), None, flags=flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) & 1
+    # the finite row is unaffected
+    o, _ = oracle.quantize_qx_0_w(4, x[:1].numpy(), None)
+    assert np.mean(np.all(g.cpu().numpy()[:1].reshape(-1, 18) == o.reshape(-1, 18), axis=1)) >= 0.9999
+
+
 def test_qx_0_bits4_is_q4_0(iqq, synth):
     x = synth.weight_matrix(64, 4096, seed=9, device="cuda")
     q = synth.imatrix(4096, seed=10, device="cuda")
