@@ -275,7 +275,21 @@ def run_gemv_phase(iqq, w: Workload, dev, reps: int = 5):
     ms = e0.elapsed_time(e1) / reps
     nbytes = sum(t.rows * (t.cols // 32) * 18 + (t.cols // 128) * 140 + 4 * t.rows for t in w.tensors)
     del g
-    return ms, nbytes
+    # one large matrix (the widest scaling-sweep tensor, 490 MB of blocks): the kernel's
+    # streaming rate once launch and ramp no longer matter
+    big = synth.scaling_sweep()[3]
+    xb = big.weights(device=dev)
+    bb = iqq.quantize_q4_0_w(xb, big.qw(device=dev))
+    del xb
+    large = {}
+    for tok in (1, 8):
+        ab = iqq.quantize_q8_k128(synth.activations(tok, big.cols, seed=9, device=dev))
+        yb = torch.empty(tok, big.rows, dtype=torch.float32, device=dev)
+        lms = _timed(lambda: iqq.iqq_gemv_q4_0_q8_k128(bb, ab, yb, big.cols), reps=5)
+        lbytes = big.rows * (big.cols // 32) * 18 + tok * (big.cols // 128) * 140 + 4 * tok * big.rows
+        large[f"tokens_{tok}"] = {"ms": round(lms, 4), "bytes": int(lbytes), "gb_s": round(lbytes / lms / 1e6, 1)}
+    del bb
+    return ms, nbytes, {"matrix": f"{big.rows}x{big.cols}", **large}
 
 
 def _timed(fn, reps: int = 3):
@@ -542,12 +556,15 @@ def main_ours(args):
     if extras is not None:
         out["extras"] = extras
     if gemv is not None:
-        gms, gbytes = gemv
+        gms, gbytes, glarge = gemv
         ggbs = gbytes / (gms / 1e3) / 1e9
+        for v in glarge.values():
+            if isinstance(v, dict):
+                v["hbm_frac"] = round(v["gb_s"] / pk["hbm_gbs"], 4)
         out["kernels"]["gemv_q4_0_q8_k128"] = {
             "ms": round(gms, 4), "gb_s": round(ggbs, 1), "hbm_frac": round(ggbs / pk["hbm_gbs"], 4),
             "tokens": 1, "launches": len(w.tensors), "timing": "one CUDA graph of the launches, "
-            "outside the step", "bytes": int(gbytes)}
+            "outside the step", "bytes": int(gbytes), "large_matrix": glarge}
     if cpu:
         out["cpu_baseline"] = {"value": round(cpu[0], 5), "unit": UNIT, "cores": cpu[1],
                                "kind": "oracle", "sample": cpu[2]}

@@ -46,6 +46,9 @@ constexpr int kSmemMax = 227 * 1024;
 constexpr int kSmemPerSm = 228 * 1024;
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the maximum SM clock
 constexpr uint32_t kSuspendHintNs = 100000;
+#ifndef IQQ_GEMV_PDL
+#define IQQ_GEMV_PDL 1  // launch with programmatic stream serialization
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p)
 {
@@ -230,6 +233,13 @@ gemv_q4_0_q8_k128_kernel(const Params P)
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
     const int64_t GW = static_cast<int64_t>(gridDim.x) * kWarps;
     const int D = P.stages, nseg = P.nseg;
+
+    // Programmatic dependent launch: let the next kernel of the stream be scheduled as this
+    // grid's CTAs retire, and wait for the previous kernel (completion and memory flush)
+    // before the first access to global memory.  Both are no-ops without the launch
+    // attribute.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // issue pointer: the next unit (irow, iseg) to copy
     int64_t irow = gw;
@@ -466,7 +476,17 @@ iqq_status plan_and_launch(Params& P, cudaStream_t st, bool& fits)
     const int gx = static_cast<int>(need < cap ? need : cap);
     const int64_t gy = (P.n_tok + TT - 1) / TT;
     if (gy > 65535) return IQQ_ERR_SHAPE;
-    kern<<<dim3(gx, static_cast<unsigned>(gy)), kThreads, smem, st>>>(P);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gx, static_cast<unsigned>(gy));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = IQQ_GEMV_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, P) != cudaSuccess) return iqq::launch_status();
     return iqq::launch_status();
 }
 
