@@ -247,6 +247,29 @@ iqq_status iqq_gemv_q4_0_q8_k128(const void* w_blocks, const void* a_blocks, flo
                                  int64_t k, int64_t n_tok, uint32_t* d_flags, void* stream);
 
 /*
+ * iqq_gemv_q4_0_q8_k128_batch -- iqq_gemv_q4_0_q8_k128 for a list of independent problems
+ * (for example every weight matrix of a model for one decode step) in as few launches as
+ * possible: up to 64 problems per launch, the launch's CTAs apportioned to its problems by
+ * their weight bytes.  Each problem's result is exactly that of iqq_gemv_q4_0_q8_k128
+ * (the per-row summation order does not depend on the launch).
+ *  problems  HOST array of count descriptors, read during the call and not kept; every
+ *            field as for iqq_gemv_q4_0_q8_k128.  The outputs y must not overlap any
+ *            problem's inputs or other outputs.
+ * All problems are checked before anything is enqueued; the first failing check's status
+ * is returned.
+ */
+typedef struct iqq_gemv_problem {
+    const void* w_blocks;
+    const void* a_blocks;
+    float* y;
+    int64_t n_out;
+    int64_t k;
+    int64_t n_tok;
+} iqq_gemv_problem;
+iqq_status iqq_gemv_q4_0_q8_k128_batch(const iqq_gemv_problem* problems, int64_t count, uint32_t* d_flags,
+                                       void* stream);
+
+/*
  * iqq_weighted_rmse -- round-trip error of Q4_0 blocks against the source,
  * weighted by the imatrix ([SVD] §3.2 rmse and maxerr; the weights are qw
  * alone, not the quantizer weights).  With e = x - dequant(blocks) rounded to

@@ -49,6 +49,7 @@ def _load():
         "iqq_quantize_qx_0_w": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_dequant_qx_0": [ctypes.c_int, _vp, _vp, _i64, _i64, _vp],
         "iqq_gemv_q4_0_q8_k128": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+        "iqq_gemv_q4_0_q8_k128_batch": [_vp, _i64, _vp, _vp],
         "iqq_weighted_rmse_qx": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
         "iqq_quantize_qx_0_w_ws": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
                                    ctypes.c_size_t, _vp, _vp],
@@ -282,6 +283,37 @@ def iqq_gemv_q4_0_q8_k128(w_blocks, a_blocks, y, k: int, flags=None, stream=None
            _lib.iqq_gemv_q4_0_q8_k128(_ptr(w_blocks), _ptr(a_blocks), _ptr(y), n_out, k, n_tok,
                                       _ptr(flags), _stream(stream)))
     return y
+
+
+class GemvProblem(ctypes.Structure):
+    """iqq_gemv_problem."""
+    _fields_ = [("w_blocks", ctypes.c_void_p), ("a_blocks", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("n_out", ctypes.c_int64), ("k", ctypes.c_int64), ("n_tok", ctypes.c_int64)]
+
+
+def gemv_problems(items):
+    """A ctypes array of iqq_gemv_problem from (w_blocks, a_blocks, y, k) tuples of CUDA
+    tensors (y [n_tok, n_out]); the tensors must outlive every call that uses the array."""
+    import torch
+    arr = (GemvProblem * len(items))()
+    for i, (w, a, y, k) in enumerate(items):
+        _need_cuda("w_blocks", w, torch.uint8)
+        _need_cuda("a_blocks", a, torch.uint8)
+        _need_cuda("y", y, torch.float32)
+        n_tok, n_out = _shape2(y)
+        if w.numel() < q4_0_nbytes(n_out, k) or a.numel() < q8_k128_nbytes(n_tok, k):
+            raise ValueError(f"problem {i}: blocks too small")
+        arr[i] = GemvProblem(w.data_ptr(), a.data_ptr(), y.data_ptr(), n_out, k, n_tok)
+    return arr
+
+
+def iqq_gemv_q4_0_q8_k128_batch(problems, flags=None, stream=None):
+    """Runs every problem of a gemv_problems() array."""
+    import torch
+    _need_cuda("flags", flags, torch.int32)
+    _check("iqq_gemv_q4_0_q8_k128_batch",
+           _lib.iqq_gemv_q4_0_q8_k128_batch(ctypes.cast(problems, ctypes.c_void_p), len(problems), _ptr(flags),
+                                            _stream(stream)))
 
 
 def iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):

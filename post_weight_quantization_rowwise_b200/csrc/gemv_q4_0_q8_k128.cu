@@ -18,15 +18,17 @@
 // butterfly -- so results are reproducible and within (K/32 + 16) * 2^-53 * sum|terms| of
 // the exact dot product before the final rounding.
 //
-// Mapping (HBM-bound on the weight stream at small token counts): every warp owns whole
-// weight rows (rows gw, gw + GW, ... for global warp gw of GW) and streams each row through
-// its own shared-memory stages in units of up to 64 pairs of blocks (2304 bytes), copied
-// with cp.async.bulk and completing on the warp's own mbarriers; lane 0 keeps D units in
-// flight.  A lane takes up to two pairs of blocks per unit (36 bytes each, read as nine
-// 32-bit words: conflict-free because 9 is odd).  Partial sums stay in registers across the
-// units of a row; one butterfly per row.  The CTA synchronizes once, after staging the token
-// tile's activations (int8 codes with a 16-byte-chunk swizzle that keeps the per-lane
-// 128-bit loads conflict-free, the binary32 scales and the int16 block sums).
+// Mapping (HBM-bound on the weight stream at small token counts): a launch serves up to 64
+// problems (matrices); its CTAs are apportioned to them by weight bytes and each CTA owns a
+// contiguous range of one problem's rows.  Every warp of the CTA takes rows r_begin + warp,
+// + 16, ... and streams each row through its own shared-memory stages in units of up to 64
+// pairs of blocks (2304 bytes), copied with cp.async.bulk and completing on the warp's own
+// mbarriers; lane 0 keeps D units in flight.  A lane takes up to two pairs of blocks per
+// unit (36 bytes each, read as nine 32-bit words: conflict-free because 9 is odd).  Partial
+// sums stay in registers across the units of a row; one butterfly per row.  The CTA
+// synchronizes once, after staging its problem's activations for its token tile (int8 codes
+// with a 16-byte-chunk swizzle that keeps the per-lane 128-bit loads conflict-free, the
+// binary32 scales and the int16 block sums).
 //
 // Every wait on an mbarrier is bounded by a clock limit; on expiry the warp raises
 // IQQ_FLAG_WAIT_TIMEOUT, drains its copies in flight (again bounded) and returns.
@@ -106,20 +108,33 @@ __device__ __forceinline__ int dp4a_us(uint32_t u, uint32_t s, int c)
     return r;
 }
 
-struct Params {
+// One matrix-vector problem of a launch (the ABI's iqq_gemv_problem, validated).
+struct Problem {
     const uint8_t* w;
     const uint8_t* a;
     float* y;
-    uint32_t* flags;
     int64_t n_out;
-    int64_t n_tok;
-    int64_t wbytes;    // n_out * rowbytes
-    int k;
-    int rowbytes;      // (k / 32) * 18
-    int nseg;          // units per row
-    int stages;        // D, units in flight per warp
-    int act_q8_bytes;  // per token: k rounded up to 16
-    int off_d8, off_bs, off_stage, off_bar;  // shared-memory layout
+    int32_t k;
+    int32_t n_tok;
+};
+
+constexpr int kMaxBatch = 64;  // problems per launch (kernel parameters stay under 4 KB)
+
+struct Params {
+    Problem prob[kMaxBatch];
+    int cta_begin[kMaxBatch + 1];  // CTAs [cta_begin[p], cta_begin[p + 1]) serve problem p
+    int count;
+    int stages;                    // D, units in flight per warp
+    int off_stage, off_bar;        // shared-memory layout; activations below off_stage
+    uint32_t* flags;
+};
+static_assert(sizeof(Params) <= 4096, "kernel parameters");
+
+// What a CTA needs of its problem.
+struct View {
+    const uint8_t* w;
+    int64_t wbytes;  // n_out * rowbytes
+    int k, rowbytes, nseg;
 };
 
 // Byte offset of logical int8 index j of a token row in the swizzled layout: 16-byte chunk
@@ -134,7 +149,7 @@ __device__ __forceinline__ int q8_swizzle(int j)
 // Issues unit (row, seg) into a stage.  The copy starts at the 16-byte boundary at or below
 // the unit's first byte (rows start 8 bytes past one when k % 256 == 128), so the unit's
 // pairs begin at stage offset (start & 15).
-__device__ __forceinline__ void issue_unit(const Params& P, uint8_t* stage, uint64_t* bar, int64_t row, int seg)
+__device__ __forceinline__ void issue_unit(const View& P, uint8_t* stage, uint64_t* bar, int64_t row, int seg)
 {
     const int p0 = seg * kUnitPairs;
     const int np = (P.k >> 6) - p0 < kUnitPairs ? (P.k >> 6) - p0 : kUnitPairs;
@@ -214,25 +229,36 @@ __device__ __forceinline__ void pair_token(const PairW& q, const uint8_t* q8t, c
 }
 
 template <int TT>
-__global__ void __launch_bounds__(kThreads, TT <= 2 ? 2 : 1)
-gemv_q4_0_q8_k128_kernel(const Params P)
+__global__ void __launch_bounds__(kThreads, TT == 1 ? 2 : 1)
+gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* q8s = smem;                                         // [TT][k] swizzled
-    float* d8s = reinterpret_cast<float*>(smem + P.off_d8);      // [TT][k/128]
-    int16_t* bss = reinterpret_cast<int16_t*>(smem + P.off_bs);  // [TT][k/32]
-
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // this CTA's problem and its contiguous share of the problem's rows
+    int pi = 0;
+    while (pi + 1 < P.count && P.cta_begin[pi + 1] <= static_cast<int>(blockIdx.x)) ++pi;
+    const Problem& pr = P.prob[pi];
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * TT;
+    if (tok0 >= pr.n_tok) return;  // a token tile another problem needs
+    const int lc = static_cast<int>(blockIdx.x) - P.cta_begin[pi];
+    const int nc = P.cta_begin[pi + 1] - P.cta_begin[pi];
+    const int64_t r_begin = pr.n_out * lc / nc, r_end = pr.n_out * (lc + 1) / nc;
+    const int nt = static_cast<int>(pr.n_tok - tok0 < TT ? pr.n_tok - tok0 : TT);
+    const int k = pr.k, nb8 = k >> 7, nb4 = k >> 5, npairs = k >> 6;
+    View V;
+    V.w = pr.w;
+    V.k = k;
+    V.rowbytes = (k >> 5) * 18;
+    V.wbytes = pr.n_out * V.rowbytes;
+    V.nseg = (npairs + kUnitPairs - 1) / kUnitPairs;
+    const int act_q8_bytes = (k + 15) & ~15;
+    uint8_t* q8s = smem;                                                                  // [TT][k]
+    float* d8s = reinterpret_cast<float*>(smem + TT * act_q8_bytes);                      // [TT][k/128]
+    int16_t* bss = reinterpret_cast<int16_t*>(smem + ((TT * act_q8_bytes + TT * nb8 * 4 + 15) & ~15));
     uint8_t* stages = smem + P.off_stage + warp * P.stages * kUnitBytes;               // this warp's
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar) + warp * P.stages;  // this warp's
-
-    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * TT;
-    const int nt = static_cast<int>(P.n_tok - tok0 < TT ? P.n_tok - tok0 : TT);
-    const int k = P.k, nb8 = k >> 7, nb4 = k >> 5, npairs = k >> 6;
-
-    const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-    const int64_t GW = static_cast<int64_t>(gridDim.x) * kWarps;
-    const int D = P.stages, nseg = P.nseg;
+    const int D = P.stages, nseg = V.nseg;
 
     // Programmatic dependent launch: let the next kernel of the stream be scheduled as this
     // grid's CTAs retire, and wait for the previous kernel (completion and memory flush)
@@ -242,17 +268,17 @@ gemv_q4_0_q8_k128_kernel(const Params P)
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // issue pointer: the next unit (irow, iseg) to copy
-    int64_t irow = gw;
+    int64_t irow = r_begin + warp;
     int iseg = 0;
     if (lane == 0) {
         for (int s = 0; s < D; ++s) mbar_init(&bars[s], 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int s = 0; s < D && irow < P.n_out; ++s) {
-        if (lane == 0) issue_unit(P, stages + s * kUnitBytes, &bars[s], irow, iseg);
+    for (int s = 0; s < D && irow < r_end; ++s) {
+        if (lane == 0) issue_unit(V, stages + s * kUnitBytes, &bars[s], irow, iseg);
         if (++iseg == nseg) {
             iseg = 0;
-            irow += GW;
+            irow += kWarps;
         }
     }
 
@@ -260,9 +286,9 @@ gemv_q4_0_q8_k128_kernel(const Params P)
     // 140-byte block, lane i copying code word i.
     for (int b = warp; b < nt * nb8; b += kWarps) {
         const int t = b / nb8, g = b - t * nb8;
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(P.a + ((tok0 + t) * nb8 + g) * 140);
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(pr.a + ((tok0 + t) * nb8 + g) * 140);
         const uint32_t v = __ldg(src + 1 + lane);
-        *reinterpret_cast<uint32_t*>(q8s + t * P.act_q8_bytes + q8_swizzle(128 * g + 4 * lane)) = v;
+        *reinterpret_cast<uint32_t*>(q8s + t * act_q8_bytes + q8_swizzle(128 * g + 4 * lane)) = v;
         if (lane < 3) {
             const uint32_t e = __ldg(src + (lane == 0 ? 0 : 32 + lane));
             if (lane == 0) d8s[t * nb8 + g] = __uint_as_float(e);
@@ -278,11 +304,11 @@ gemv_q4_0_q8_k128_kernel(const Params P)
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.0;
     // consume pointer: unit (row, seg) in stage s, phase parity ph
-    int64_t row = gw;
+    int64_t row = r_begin + warp;
     int seg = 0, s = 0;
     uint32_t ph = 0;
     bool aborted = false;
-    while (row < P.n_out) {
+    while (row < r_end) {
         const bool timed_out = !mbar_wait(&bars[s], ph);
         if (__any_sync(0xffffffffu, timed_out)) {
             aborted = true;
@@ -290,7 +316,7 @@ gemv_q4_0_q8_k128_kernel(const Params P)
         }
         const int p0 = seg * kUnitPairs;
         const int np = npairs - p0 < kUnitPairs ? npairs - p0 : kUnitPairs;
-        const int64_t start = row * P.rowbytes + 36LL * p0;
+        const int64_t start = row * V.rowbytes + 36LL * p0;
         const uint32_t* w9 = reinterpret_cast<const uint32_t*>(stages + s * kUnitBytes + (start & 15));
 
         PairW q0, q1;
@@ -299,17 +325,17 @@ gemv_q4_0_q8_k128_kernel(const Params P)
         if (has1) load_pair(w9 + 9 * (lane + 32), q1);
         __syncwarp();
         // every lane holds its words: refill the stage with the next unit to copy
-        if (irow < P.n_out) {
-            if (lane == 0) issue_unit(P, stages + s * kUnitBytes, &bars[s], irow, iseg);
+        if (irow < r_end) {
+            if (lane == 0) issue_unit(V, stages + s * kUnitBytes, &bars[s], irow, iseg);
             if (++iseg == nseg) {
                 iseg = 0;
-                irow += GW;
+                irow += kWarps;
             }
         }
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
             if (t < nt) {
-                const uint8_t* q8t = q8s + t * P.act_q8_bytes;
+                const uint8_t* q8t = q8s + t * act_q8_bytes;
                 const int16_t* bst = bss + t * nb4;
                 const float* d8t = d8s + t * nb8;
                 if (has0) pair_token(q0, q8t, bst, d8t, p0 + lane, sw, acc[t]);
@@ -325,12 +351,12 @@ gemv_q4_0_q8_k128_kernel(const Params P)
             if (lane == 0) {
 #pragma unroll
                 for (int t = 0; t < TT; ++t)
-                    if (t < nt) P.y[(tok0 + t) * P.n_out + row] = static_cast<float>(acc[t]);
+                    if (t < nt) pr.y[(tok0 + t) * pr.n_out + row] = static_cast<float>(acc[t]);
             }
 #pragma unroll
             for (int t = 0; t < TT; ++t) acc[t] = 0.0;
             seg = 0;
-            row += GW;
+            row += kWarps;
         }
         if (++s == D) {
             s = 0;
@@ -346,7 +372,7 @@ gemv_q4_0_q8_k128_kernel(const Params P)
             (void)mbar_wait(&bars[s], ph);
             if (++seg == nseg) {
                 seg = 0;
-                row += GW;
+                row += kWarps;
             }
             if (++s == D) {
                 s = 0;
@@ -388,21 +414,18 @@ constexpr int tt_slot(int tt) { return tt == 1 ? 0 : (tt == 2 ? 1 : (tt == 4 ? 2
 
 int align16(int v) { return (v + 15) & ~15; }
 
-int smem_bytes(const Params& P) { return P.off_bar + kWarps * P.stages * 8; }
+// Shared-memory layout of a launch: activations of tt tokens for the largest k, then d
+// units per warp, then the warps' mbarriers.
+int act_bytes(int tt, int k) { return align16(align16(tt * align16(k) + tt * (k / 128) * 4) + tt * (k / 32) * 2); }
 
-// Shared-memory layout for a token tile of tt tokens and d units in flight per warp.
-void make_plan(Params& P, int tt, int d)
+void make_plan(Params& P, int tt, int kmax, int d)
 {
-    const int k = P.k;
-    P.rowbytes = (k / 32) * 18;
-    P.nseg = (k / 64 + kUnitPairs - 1) / kUnitPairs;
     P.stages = d;
-    P.act_q8_bytes = align16(k);
-    P.off_d8 = tt * P.act_q8_bytes;
-    P.off_bs = align16(P.off_d8 + tt * (k / 128) * 4);
-    P.off_stage = align16(P.off_bs + tt * (k / 32) * 2);
+    P.off_stage = act_bytes(tt, kmax);
     P.off_bar = P.off_stage + kWarps * d * kUnitBytes;
 }
+
+int smem_bytes(const Params& P) { return P.off_bar + kWarps * P.stages * 8; }
 
 // Resident CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA) and 64 K registers
 // (allocated per warp in units of 256).
@@ -434,12 +457,12 @@ int kernel_regs(int dev)
 // beat 16 warps x 4 units, the per-unit arithmetic needing the extra warps to hide its
 // latency).
 template <int TT>
-bool plan_tt(Params& P, int dev, int& ctas)
+bool plan_tt(Params& P, int kmax, int dev, int& ctas)
 {
     const int regs = kernel_regs<TT>(dev);
     int best_d = 0, best_flight = 0, best_ctas = 0;
     for (int d = 2; d <= 4; ++d) {
-        make_plan(P, TT, d);
+        make_plan(P, TT, kmax, d);
         const int smem = smem_bytes(P);
         if (smem > kSmemMax) break;
         const int c = ctas_per_sm(smem, regs);
@@ -451,17 +474,19 @@ bool plan_tt(Params& P, int dev, int& ctas)
         }
     }
     if (best_d == 0) return false;
-    make_plan(P, TT, best_d);
+    make_plan(P, TT, kmax, best_d);
     ctas = best_ctas;
     return true;
 }
 
+// Launches P.count (<= kMaxBatch) problems: CTAs apportioned to the problems by their
+// weight bytes (at least one each, at most one per 16 rows), the token tiles on grid y.
 template <int TT>
-iqq_status plan_and_launch(Params& P, cudaStream_t st, bool& fits)
+iqq_status launch_tt(Params& P, int kmax, int64_t max_tok, cudaStream_t st, bool& fits)
 {
     const int dev = current_device();
     int ctas = 0;
-    fits = plan_tt<TT>(P, dev, ctas);
+    fits = plan_tt<TT>(P, kmax, dev, ctas);
     if (!fits) return IQQ_OK;
     const int smem = smem_bytes(P);
     auto kern = gemv_q4_0_q8_k128_kernel<TT>;
@@ -471,13 +496,24 @@ iqq_status plan_and_launch(Params& P, cudaStream_t st, bool& fits)
             return iqq::launch_status();
         opted.store(kSmemMax, std::memory_order_relaxed);
     }
-    const int64_t need = (P.n_out + kWarps - 1) / kWarps;
-    const int64_t cap = static_cast<int64_t>(sm_count_gemv(dev)) * ctas;
-    const int gx = static_cast<int>(need < cap ? need : cap);
-    const int64_t gy = (P.n_tok + TT - 1) / TT;
+    const int64_t target = static_cast<int64_t>(sm_count_gemv(dev)) * ctas;
+    double total = 0.0;
+    for (int i = 0; i < P.count; ++i) total += static_cast<double>(P.prob[i].n_out) * (P.prob[i].k / 32) * 18;
+    int c0 = 0;
+    for (int i = 0; i < P.count; ++i) {
+        const double bytes = static_cast<double>(P.prob[i].n_out) * (P.prob[i].k / 32) * 18;
+        int64_t n = static_cast<int64_t>(static_cast<double>(target) * bytes / total + 0.5);
+        const int64_t most = (P.prob[i].n_out + kWarps - 1) / kWarps;
+        if (n > most) n = most;
+        if (n < 1) n = 1;
+        P.cta_begin[i] = c0;
+        c0 += static_cast<int>(n);
+    }
+    P.cta_begin[P.count] = c0;
+    const int64_t gy = (max_tok + TT - 1) / TT;
     if (gy > 65535) return IQQ_ERR_SHAPE;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(gx, static_cast<unsigned>(gy));
+    cfg.gridDim = dim3(static_cast<unsigned>(c0), static_cast<unsigned>(gy));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = st;
@@ -490,51 +526,101 @@ iqq_status plan_and_launch(Params& P, cudaStream_t st, bool& fits)
     return iqq::launch_status();
 }
 
+// Host checks of one problem, before anything is enqueued.
+iqq_status check_problem(const iqq_gemv_problem& q)
+{
+    if (q.n_out < 0 || q.k < 0 || q.n_tok < 0 || q.k % 128 != 0 || q.k > IQQ_GEMV_MAX_K) return IQQ_ERR_SHAPE;
+    if (!iqq::size_ok(q.n_out, q.k, 1) || !iqq::size_ok(q.n_tok, q.k, 2) || !iqq::size_ok(q.n_tok, q.n_out, 4))
+        return IQQ_ERR_SHAPE;
+    if (q.n_out == 0 || q.n_tok == 0) return IQQ_OK;
+    if (q.y == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(q.y, 4)) return IQQ_ERR_ALIGN;
+    if (q.k == 0) return IQQ_OK;
+    if (q.w_blocks == nullptr || q.a_blocks == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(q.w_blocks, 16) || !iqq::aligned(q.a_blocks, 4)) return IQQ_ERR_ALIGN;
+    return IQQ_OK;
+}
+
+iqq_status gemv_batch(const iqq_gemv_problem* probs, int64_t count, uint32_t* d_flags, cudaStream_t st)
+{
+    if (count < 0) return IQQ_ERR_SHAPE;
+    if (count > 0 && probs == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(d_flags, 4)) return IQQ_ERR_ALIGN;
+    for (int64_t i = 0; i < count; ++i) {
+        const iqq_status c = check_problem(probs[i]);
+        if (c != IQQ_OK) return c;
+    }
+    Params P{};
+    P.flags = d_flags;
+    int kmax = 0;
+    int64_t max_tok = 0;
+    auto flush = [&]() -> iqq_status {
+        if (P.count == 0) return IQQ_OK;
+        // token tile: the smallest of 1, 2, 4, 8 covering the largest n_tok (8 beyond),
+        // halved while the activations do not fit beside the weight stages
+        int tt = max_tok >= 5 ? 8 : (max_tok >= 3 ? 4 : static_cast<int>(max_tok));
+        iqq_status s = IQQ_OK;
+        for (;;) {
+            bool fits = false;
+            switch (tt) {
+            case 1: s = launch_tt<1>(P, kmax, max_tok, st, fits); break;
+            case 2: s = launch_tt<2>(P, kmax, max_tok, st, fits); break;
+            case 4: s = launch_tt<4>(P, kmax, max_tok, st, fits); break;
+            default: s = launch_tt<8>(P, kmax, max_tok, st, fits); break;
+            }
+            if (fits || s != IQQ_OK) break;
+            if (tt == 1) return IQQ_ERR_SHAPE;
+            tt >>= 1;
+        }
+        P.count = 0;
+        kmax = 0;
+        max_tok = 0;
+        return s;
+    };
+    for (int64_t i = 0; i < count; ++i) {
+        const iqq_gemv_problem& q = probs[i];
+        if (q.n_out == 0 || q.n_tok == 0) continue;
+        if (q.k == 0) {
+            // the dot product of empty vectors
+            if (cudaMemsetAsync(q.y, 0, static_cast<size_t>(q.n_tok * q.n_out) * sizeof(float), st) != cudaSuccess)
+                return iqq::launch_status();
+            continue;
+        }
+        Problem& pr = P.prob[P.count++];
+        pr.w = static_cast<const uint8_t*>(q.w_blocks);
+        pr.a = static_cast<const uint8_t*>(q.a_blocks);
+        pr.y = q.y;
+        pr.n_out = q.n_out;
+        pr.k = static_cast<int32_t>(q.k);
+        pr.n_tok = static_cast<int32_t>(q.n_tok);
+        if (pr.k > kmax) kmax = pr.k;
+        if (q.n_tok > max_tok) max_tok = q.n_tok;
+        if (P.count == kMaxBatch) {
+            const iqq_status s = flush();
+            if (s != IQQ_OK) return s;
+        }
+    }
+    return flush();
+}
+
 }  // namespace
 
 extern "C" iqq_status iqq_gemv_q4_0_q8_k128(const void* w_blocks, const void* a_blocks, float* y,
                                             int64_t n_out, int64_t k, int64_t n_tok, uint32_t* d_flags,
                                             void* stream)
 {
-    if (n_out < 0 || k < 0 || n_tok < 0 || k % 128 != 0 || k > IQQ_GEMV_MAX_K) return IQQ_ERR_SHAPE;
-    if (!iqq::size_ok(n_out, k, 1) || !iqq::size_ok(n_tok, k, 2) || !iqq::size_ok(n_tok, n_out, 4))
-        return IQQ_ERR_SHAPE;
-    if (n_out == 0 || n_tok == 0) return IQQ_OK;
-    if (y == nullptr) return IQQ_ERR_NULL;
-    if (!iqq::aligned(y, 4) || !iqq::aligned(d_flags, 4)) return IQQ_ERR_ALIGN;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (k == 0) {
-        // the dot product of empty vectors
-        if (cudaMemsetAsync(y, 0, static_cast<size_t>(n_tok * n_out) * sizeof(float), st) != cudaSuccess)
-            return iqq::launch_status();
-        return IQQ_OK;
-    }
-    if (w_blocks == nullptr || a_blocks == nullptr) return IQQ_ERR_NULL;
-    if (!iqq::aligned(w_blocks, 16) || !iqq::aligned(a_blocks, 4)) return IQQ_ERR_ALIGN;
+    iqq_gemv_problem q;
+    q.w_blocks = w_blocks;
+    q.a_blocks = a_blocks;
+    q.y = y;
+    q.n_out = n_out;
+    q.k = k;
+    q.n_tok = n_tok;
+    return gemv_batch(&q, 1, d_flags, static_cast<cudaStream_t>(stream));
+}
 
-    Params P{};
-    P.w = static_cast<const uint8_t*>(w_blocks);
-    P.a = static_cast<const uint8_t*>(a_blocks);
-    P.y = y;
-    P.flags = d_flags;
-    P.n_out = n_out;
-    P.n_tok = n_tok;
-    P.k = static_cast<int>(k);
-    P.wbytes = n_out * ((k / 32) * 18);
-    // token tile: the smallest of 1, 2, 4, 8 covering n_tok (8 beyond), halved while the
-    // activations do not fit beside the weight stages
-    int tt = n_tok >= 5 ? 8 : (n_tok >= 3 ? 4 : static_cast<int>(n_tok));
-    for (;;) {
-        bool fits = false;
-        iqq_status s = IQQ_OK;
-        switch (tt) {
-        case 1: s = plan_and_launch<1>(P, st, fits); break;
-        case 2: s = plan_and_launch<2>(P, st, fits); break;
-        case 4: s = plan_and_launch<4>(P, st, fits); break;
-        default: s = plan_and_launch<8>(P, st, fits); break;
-        }
-        if (fits || s != IQQ_OK) return s;
-        if (tt == 1) return IQQ_ERR_SHAPE;
-        tt >>= 1;
-    }
+extern "C" iqq_status iqq_gemv_q4_0_q8_k128_batch(const iqq_gemv_problem* problems, int64_t count,
+                                                  uint32_t* d_flags, void* stream)
+{
+    return gemv_batch(problems, count, d_flags, static_cast<cudaStream_t>(stream));
 }

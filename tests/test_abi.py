@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
               "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string",
               "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128",
               "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
-              "iqq_quantize_qx_0_w_static"):
+              "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch"):
         assert n in names
 
 
@@ -112,6 +112,20 @@ def test_host_validation_without_gpu(lib):
     assert S(4, V(16), None, V(16), 2, 53248, 0, 7, None, None) == 5
     assert S(4, V(8), None, V(16), 2, 53248, 0, 0, None, None) == 3
     assert S(4, None, None, None, 0, 53248, 0, 0, None, None) == 0
+    # the batched product: checks of every problem before anything is enqueued
+    import post_weight_quantization_rowwise_b200 as m
+    B = lib.iqq_gemv_q4_0_q8_k128_batch
+    ok = m.GemvProblem(16, 16, 16, 4, 128, 1)
+    bad = m.GemvProblem(16, 16, 16, 4, 96, 1)
+    arr = (m.GemvProblem * 3)(ok, bad, ok)
+    assert B(ctypes.cast(arr, V), 3, None, None) == 2
+    assert B(None, 2, None, None) == 1
+    assert B(ctypes.cast(arr, V), -1, None, None) == 2
+    assert B(None, 0, None, None) == 0
+    empty = (m.GemvProblem * 2)(m.GemvProblem(0, 0, 0, 0, 128, 1), m.GemvProblem(16, 16, 16, 4, 128, 0))
+    assert B(ctypes.cast(empty, V), 2, None, None) == 0
+    unaligned = (m.GemvProblem * 1)(m.GemvProblem(8, 16, 16, 4, 128, 1))
+    assert B(ctypes.cast(unaligned, V), 1, None, None) == 3
     # Q4_0 x Q8_K_128 matrix-vector product
     G = lib.iqq_gemv_q4_0_q8_k128
     assert G(V(16), V(16), V(16), 4, 96, 1, None, None) == 2          # k not a multiple of 128

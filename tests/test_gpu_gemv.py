@@ -121,3 +121,34 @@ def test_gemv_reproducible_and_empty(iqq, synth):
     iqq.iqq_gemv_q4_0_q8_k128(w, a, y0, 0)
     torch.cuda.synchronize()
     assert torch.count_nonzero(y0).item() == 0
+
+
+def test_gemv_batch_matches_single_calls(iqq, synth):
+    """A list of problems of different shapes, token counts and widths (incl. empty and
+    k == 0 ones, and more than one launch's worth): every output equals the single call's
+    bit for bit and lies within the bound of the oracle's value."""
+    rng = np.random.default_rng(40)
+    shapes = [(64, 4096, 1), (37, 11008, 3), (5, 128, 1), (130, 4224, 5), (1, 256, 9), (0, 512, 2),
+              (7, 0, 2), (300, 1024, 1)] + [(3 + i % 5, 128 * (1 + i % 4), 1 + i % 3) for i in range(66)]
+    items, singles, refs = [], [], []
+    for i, (n_out, k, n_tok) in enumerate(shapes):
+        w = torch.from_numpy(_random_q4_0(rng, max(n_out, 1), max(k, 128))).cuda()
+        a = torch.from_numpy(_activations(synth, n_tok, max(k, 128), seed=i)).cuda()
+        y = torch.full((n_tok, n_out), float("nan"), device="cuda")
+        items.append((w, a, y, k))
+        singles.append(iqq.gemv_q4_0_q8_k128(w, a, n_out, k, n_tok) if n_out and n_tok else None)
+        refs.append((w, a, n_out, k, n_tok))
+    probs = iqq.gemv_problems(items)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    iqq.iqq_gemv_q4_0_q8_k128_batch(probs, flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    for (w, a, y, k), single, (_, _, n_out, _, n_tok) in zip(items, singles, refs):
+        if single is None:
+            continue
+        assert torch.equal(y, single)
+        if k == 0:
+            assert torch.count_nonzero(y).item() == 0
+            continue
+        yo, s = oracle.dot_q4_0_q8_k128(w.cpu().numpy(), a.cpu().numpy(), n_out, k, n_tok)
+        _check(y.cpu().numpy(), yo, s, k)
