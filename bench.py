@@ -39,15 +39,19 @@ WORKLOAD = "llama2-7b layer set x32 (q4_0 imatrix + dequant + wrmse) + q8_k128 4
 #   Q8_K_128: 4 + 140/128 bytes per value; dequant: 18/32 + 4; wrmse: 4 + 18/32 (+ qw from L2).
 Q4_0_OPS_BASE = 145.0
 Q4_0_OPS_PER_PASS = 8.0
+# the round trip accumulated by the same kernel: y = d*l, e = x - y, e^2, qw*e^2 + sum,
+# sum qw, sum e^2, max |e|
+Q4_0_RMSE_OPS = 7.0
 Q8_BYTES_PER_VALUE = 4.0 + 140.0 / 128.0
 DEQ_BYTES_PER_VALUE = 18.0 / 32.0 + 4.0
+DEQ_RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0 + 4.0  # read x and the blocks, write y
 RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
-# kernel (4096x4096 launch: 67.187 MB read + 2.091 MB written for 16,777,216 values); set
+# kernel (4096x4096 launch: 67.196 MB read + 1.494 MB written for 16,777,216 values); set
 # to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = 4.1293
+Q4_0_DRAM_BYTES_PER_VALUE = 4.0942
 
 
 def peaks():
@@ -213,7 +217,10 @@ class Workload:
 
 
 def run_step(iqq, w: Workload, stream, ev=None):
-    """Enqueues one step.  ev: optional list of 5 events bracketing the 4 phases."""
+    """Enqueues one step.  ev: optional list of 4 events bracketing the 3 phases: the
+    weighted Q4_0 quantization of every tensor; the dequantization of every tensor with
+    its round-trip weighted error accumulated in the same pass; Q8_K_128 of the
+    activations."""
     import torch
     if ev is not None:
         ev[0].record(stream)
@@ -221,19 +228,15 @@ def run_step(iqq, w: Workload, stream, ev=None):
         iqq.iqq_quantize_q4_0_w(x, qw, b, stream=stream)
     if ev is not None:
         ev[1].record(stream)
-    for t, b in zip(w.tensors, w.blocks):
-        iqq.iqq_dequant_q4_0(b, w.y[:t.numel].view(t.rows, t.cols), stream=stream)
+    w.acc.zero_()
+    for t, x, qw, b in zip(w.tensors, w.x, w.qw, w.blocks):
+        iqq.iqq_dequant_rmse_qx(4, x, b, qw, w.y[:t.numel].view(t.rows, t.cols), w.acc, stream=stream)
     if ev is not None:
         ev[2].record(stream)
-    w.acc.zero_()
-    for x, qw, b in zip(w.x, w.qw, w.blocks):
-        iqq.iqq_weighted_rmse(x, b, qw, w.acc, stream=stream)
-    if ev is not None:
-        ev[3].record(stream)
     iqq.iqq_quantize_q8_k128(w.act, w.q8, stream=stream)
     if ev is not None:
-        ev[4].record(stream)
-    return 3 * len(w.tensors) + 1
+        ev[3].record(stream)
+    return 2 * len(w.tensors) + 1
 
 
 def run_gemv_phase(iqq, w: Workload, dev, reps: int = 5):
@@ -420,8 +423,8 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
             xv.copy_(host_x[i], non_blocking=True)
             qd[:t.cols].copy_(host_qw[i], non_blocking=True)
             iqq.iqq_quantize_q4_0_w(xv, qd[:t.cols], w.blocks[i], stream=stream)
-            iqq.iqq_dequant_q4_0(w.blocks[i], w.y[:t.numel].view(t.rows, t.cols), stream=stream)
-            iqq.iqq_weighted_rmse(xv, w.blocks[i], qd[:t.cols], w.acc, stream=stream)
+            iqq.iqq_dequant_rmse_qx(4, xv, w.blocks[i], qd[:t.cols], w.y[:t.numel].view(t.rows, t.cols), w.acc,
+                                    stream=stream)
             host_b[i].copy_(w.blocks[i], non_blocking=True)
         w.act.copy_(host_act, non_blocking=True)
         iqq.iqq_quantize_q8_k128(w.act, w.q8, stream=stream)
@@ -467,7 +470,7 @@ def main_ours(args):
         run_step(iqq, w, stream)
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(1.0)  # nvidia-smi's first sample arrives after start-up
@@ -480,11 +483,11 @@ def main_ours(args):
         launches += run_step(iqq, w, stream, ev[s])
     torch.cuda.synchronize()
     clk = clocks.stop()
-    phase = [0.0] * 4
+    phase = [0.0] * 3
     for s in range(args.steps):
-        for p in range(4):
+        for p in range(3):
             phase[p] += ev[s][p].elapsed_time(ev[s][p + 1])
-    total_ms = ev[0][0].elapsed_time(ev[-1][4])
+    total_ms = ev[0][0].elapsed_time(ev[-1][3])
     from post_weight_quantization_rowwise_b200 import replicas
     times = replicas.max_over_ranks([total_ms] + phase, device=dev)  # the slowest rank
     if world > 1:
@@ -521,9 +524,8 @@ def main_ours(args):
     ops_per_value = Q4_0_OPS_BASE + Q4_0_OPS_PER_PASS * p_mean
     achieved = w.q4_elems * ops_per_value / (q4_ms / 1e3) / 1e12          # Tops/s
     peak_ops = B200_SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
-    deq_gbs = w.q4_elems * DEQ_BYTES_PER_VALUE / (phase[1] / K / 1e3) / 1e9
-    rmse_gbs = w.q4_elems * RMSE_BYTES_PER_VALUE / (phase[2] / K / 1e3) / 1e9
-    q8_gbs = w.q8_elems * Q8_BYTES_PER_VALUE / (phase[3] / K / 1e3) / 1e9
+    drm_gbs = w.q4_elems * DEQ_RMSE_BYTES_PER_VALUE / (phase[1] / K / 1e3) / 1e9
+    q8_gbs = w.q8_elems * Q8_BYTES_PER_VALUE / (phase[2] / K / 1e3) / 1e9
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -532,7 +534,8 @@ def main_ours(args):
         "config": {"workload": WORKLOAD, "layers": args.layers, "tensors": n_q4,
                    "q4_0_values": w.q4_elems, "q8_k128_values": w.q8_elems,
                    "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (replicas)"},
-        "roofline": {"bound": "alu", "kernel": "qx_0_w_kernel<4>", "achieved": round(achieved, 3),
+        "roofline": {"bound": "alu", "kernel": "qx_0_w_kernel<4>",
+                     "achieved": round(achieved, 3),
                      "peak": round(peak_ops, 3), "unit": "Tops/s",
                      "frac": round(achieved / peak_ops, 4),
                      "traffic": (None if Q4_0_DRAM_BYTES_PER_VALUE is None else
@@ -544,14 +547,15 @@ def main_ours(args):
                                    f"{pk['sm_max_mhz']:.0f} MHz ({pk['source']} max clock)"},
         "kernels": {
             "q4_0_w": {"ms": round(q4_ms, 4), "gelem_s": round(w.q4_elems / (q4_ms / 1e3) / 1e9, 3)},
-            "dequant_q4_0": {"ms": round(phase[1] / K, 4), "gb_s": round(deq_gbs, 1),
-                             "hbm_frac": round(deq_gbs / pk["hbm_gbs"], 4)},
-            "weighted_rmse": {"ms": round(phase[2] / K, 4), "gb_s": round(rmse_gbs, 1),
-                              "hbm_frac": round(rmse_gbs / pk["hbm_gbs"], 4),
-                              "wrmse": math.sqrt(acc[0] / acc[1]) if acc[1] else None},
-            "q8_k128": {"ms": round(phase[3] / K, 4), "gb_s": round(q8_gbs, 1),
+            "dequant_rmse_q4_0": {"ms": round(phase[1] / K, 4), "gb_s": round(drm_gbs, 1),
+                                  "hbm_frac": round(drm_gbs / pk["hbm_gbs"], 4),
+                                  "kernel": "weighted_rmse_kernel<4> writing y",
+                                  "bytes_per_value": DEQ_RMSE_BYTES_PER_VALUE,
+                                  "wrmse": math.sqrt(acc[0] / acc[1]) if acc[1] else None,
+                                  "rmse": math.sqrt(acc[2] / w.q4_elems), "maxerr": acc[3]},
+            "q8_k128": {"ms": round(phase[2] / K, 4), "gb_s": round(q8_gbs, 1),
                         "hbm_frac": round(q8_gbs / pk["hbm_gbs"], 4),
-                        "gelem_s": round(w.q8_elems / (phase[3] / K / 1e3) / 1e9, 3)},
+                        "gelem_s": round(w.q8_elems / (phase[2] / K / 1e3) / 1e9, 3)},
         },
         "gpu_launches": launches,
         "clocks": clk,

@@ -141,6 +141,29 @@ iqq_status iqq_quantize_qx_0_w_ws(int bits, const float* x, const float* qw, voi
                                   size_t workspace_bytes, uint32_t* d_flags, void* stream);
 
 /*
+ * iqq_quantize_qx_0_w_ex -- the general form of the weighted quantizers: any 32-value
+ * format, an optional workspace, an optional dequantized output and an optional
+ * round-trip error accumulator (quantization, dequantization and the weighted RMSE of a
+ * tensor in one pass over it).
+ *  workspace, workspace_bytes  as for iqq_quantize_qx_0_w_ws, but optional: with NULL the
+ *                   per-CTA row reduction is used for every width.
+ *  y_out            optional device float32 [nrows, n_per_row] (16-byte aligned): the
+ *                   kernel that writes the blocks also writes their dequantized values,
+ *                   bit for bit those of iqq_dequant_qx_0.
+ *  d_acc            optional device double[4] (8-byte aligned), caller-owned and zeroed by
+ *                   the caller.  When given, the kernel that writes the blocks also adds
+ *                   the round trip of every block written, exactly as iqq_weighted_rmse
+ *                   does over them (e = x - fp16(d) * l in binary32; {sum qw e^2, sum qw,
+ *                   sum e^2} in binary64, max |e|), so the tensor is read once for both
+ *                   ([SVD] §3.2 rmse / maxerr, weighted by the imatrix).
+ * Other arguments and errors as for iqq_quantize_qx_0_w.
+ */
+iqq_status iqq_quantize_qx_0_w_ex(int bits, const float* x, const float* qw, void* out, int64_t nrows,
+                                  int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
+                                  size_t workspace_bytes, float* y_out, double* d_acc, uint32_t* d_flags,
+                                  void* stream);
+
+/*
  * iqq_quantize_qx_0_w_static -- iqq_quantize_qx_0_w_ws without a caller workspace: the
  * per-row sigma2 of wide rows goes to a library-owned device array of IQQ_STATIC_WS_ROWS
  * floats (a file-scope __device__ variable, one per device; nothing is allocated), and
@@ -219,6 +242,16 @@ iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, int64_t nrow
  */
 iqq_status iqq_weighted_rmse_qx(int bits, const float* x, const void* blocks, const float* qw, int64_t nrows,
                                 int64_t n_per_row, int64_t rows_per_qw, double* d_acc, void* stream);
+
+/*
+ * iqq_dequant_rmse_qx -- iqq_dequant_qx_0 and iqq_weighted_rmse_qx in one pass: reads the
+ * blocks and x once, writes y = fp16(d) * l (bit for bit iqq_dequant_qx_0's output) and
+ * adds the round trip to d_acc exactly as iqq_weighted_rmse_qx does.  y is float32
+ * [nrows, n_per_row], 16-byte aligned, required (NULL: IQQ_ERR_NULL); other arguments and
+ * errors as for iqq_weighted_rmse_qx.
+ */
+iqq_status iqq_dequant_rmse_qx(int bits, const float* x, const void* blocks, const float* qw, int64_t nrows,
+                               int64_t n_per_row, int64_t rows_per_qw, float* y, double* d_acc, void* stream);
 
 /*
  * iqq_gemv_q4_0_q8_k128 -- y[t][r] = dot(dequant(W row r), dequant(A row t)): Q4_0 weight

@@ -69,6 +69,10 @@ def lib():
         L.oracle_quantize_q8_1.argtypes = [_f32p, _u8p, _i64, _i64]
         L.oracle_quantize_q8_k128.restype = ctypes.c_int
         L.oracle_quantize_q8_k128.argtypes = [_f32p, _u8p, _i64, _i64, _u32p]
+        L.oracle_q4_0_block_bytes.argtypes = []
+        L.oracle_q8_k128_block_bytes.argtypes = []
+        L.oracle_weighted_rmse_qx.restype = ctypes.c_int
+        L.oracle_weighted_rmse_qx.argtypes = [ctypes.c_int, _f32p, _u8p, _f32p, _i64, _i64, _i64, _f64p]
         L.oracle_dot_q4_0_q8_k128.restype = ctypes.c_int
         L.oracle_dot_q4_0_q8_k128.argtypes = [_u8p, _u8p, _f64p, _f64p, _i64, _i64, _i64]
         _LIB = L

@@ -51,9 +51,12 @@ def _load():
         "iqq_gemv_q4_0_q8_k128": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
         "iqq_gemv_q4_0_q8_k128_batch": [_vp, _i64, _vp, _vp],
         "iqq_weighted_rmse_qx": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+        "iqq_dequant_rmse_qx": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "iqq_quantize_qx_0_w_ws": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
                                    ctypes.c_size_t, _vp, _vp],
         "iqq_quantize_qx_0_w_static": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
+        "iqq_quantize_qx_0_w_ex": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
+                                   ctypes.c_size_t, _vp, _vp, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -332,6 +335,25 @@ def iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
     return acc
 
 
+def iqq_dequant_rmse_qx(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, stream=None):
+    """Dequantizes blocks into y and adds the round trip against x to acc, in one pass."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("blocks", blocks, torch.uint8)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("y", y, torch.float32)
+    _need_cuda("acc", acc, torch.float64)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits] or acc.numel() < 4 or y.numel() < x.numel():
+        raise ValueError("blocks, y or acc is too small")
+    _check("iqq_dequant_rmse_qx",
+           _lib.iqq_dequant_rmse_qx(bits, _ptr(x), _ptr(blocks), _ptr(qw), nrows, n, rows_per_qw, _ptr(y),
+                                    _ptr(acc), _stream(stream)))
+    return y
+
+
 def iqq_weighted_rmse_qx(bits, x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
     """iqq_weighted_rmse for Q4_0/Q5_0/Q6_0/Q8_0 blocks (bits 4/5/6/8)."""
     import torch
@@ -377,6 +399,36 @@ def quantize_qx_0_w(bits, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0
     nrows, n = _shape2(x)
     out = torch.empty((nrows, (n // 32) * QX_0_BLOCK_BYTES[bits]), dtype=torch.uint8, device=x.device)
     return iqq_quantize_qx_0_w(bits, x, qw, out, rows_per_qw, weight_mode, flags, stream)
+
+
+def iqq_quantize_qx_0_w_ex(bits, x, qw, out, workspace=None, acc=None, rows_per_qw: int = 0,
+                           weight_mode: int = 0, flags=None, stream=None, y=None):
+    """The general quantizer: optional workspace (uint8), optional dequantized output y
+    (float32 like x) and optional round-trip error accumulator acc (float64[4], zeroed by
+    the caller)."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("workspace", workspace, torch.uint8)
+    _need_cuda("acc", acc, torch.float64)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
+        raise ValueError("out is too small")
+    if acc is not None and acc.numel() < 4:
+        raise ValueError("acc needs 4 elements")
+    _need_cuda("y", y, torch.float32)
+    if y is not None and y.numel() < x.numel():
+        raise ValueError("y is too small")
+    nbytes = 0 if workspace is None else workspace.numel()
+    _check("iqq_quantize_qx_0_w_ex",
+           _lib.iqq_quantize_qx_0_w_ex(bits, _ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw, weight_mode,
+                                       _ptr(workspace), nbytes, _ptr(y), _ptr(acc), _ptr(flags),
+                                       _stream(stream)))
+    return out
 
 
 def iqq_quantize_qx_0_w_static(bits, x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,

@@ -174,12 +174,19 @@ __device__ __forceinline__ QuadC load_codes(const uint8_t* blk, int qd)
 template <int BITS>
 __host__ __device__ constexpr int block_bytes() { return BITS == 4 ? 18 : (BITS == 5 ? 22 : (BITS == 6 ? 26 : 34)); }
 
-__device__ __forceinline__ void rmse_quad(const float4 xv, const QuadC q, double (&col)[4], float& emax)
+// Adds the quad's round trip to the column sums; y (optional) receives its dequantized
+// values y = fp16(d) * l.
+__device__ __forceinline__ void rmse_quad(const float4 xv, const QuadC q, double (&col)[4], float& emax,
+                                          float4* y)
 {
+    float yk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) yk[k] = __fmul_rn(q.d, static_cast<float>(q.c[k]));
+    if (y != nullptr) __stcs(y, make_float4(yk[0], yk[1], yk[2], yk[3]));
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float xk = k == 0 ? xv.x : k == 1 ? xv.y : k == 2 ? xv.z : xv.w;
-        const float e = __fsub_rn(xk, __fmul_rn(q.d, static_cast<float>(q.c[k])));
+        const float e = __fsub_rn(xk, yk[k]);
         emax = fmaxf(emax, fabsf(e));
         const double ed = static_cast<double>(e);
         col[k] = fma(ed, ed, col[k]);
@@ -193,7 +200,7 @@ template <int BITS>
 __global__ void __launch_bounds__(kThreads)
 weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ blocks,
                      const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
-                     int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc)
+                     int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc, float* __restrict__ y)
 {
     const int64_t nq = n_per_row / 4;
     const int64_t nb = n_per_row / IQQ_Q4_0_BLOCK_VALUES;
@@ -221,11 +228,14 @@ weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ bl
                     q[u] = load_codes<BITS>(blocks + ((r + u) * nb + b) * block_bytes<BITS>(), qd);
                 }
 #pragma unroll
-                for (int u = 0; u < kRowUnroll; ++u) rmse_quad(xv[u], q[u], col, emax);
+                for (int u = 0; u < kRowUnroll; ++u)
+                    rmse_quad(xv[u], q[u], col, emax,
+                              y != nullptr ? reinterpret_cast<float4*>(y + (r + u) * n_per_row) + cq : nullptr);
             }
             for (; r < s1; ++r) {
                 const float4 xv = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + r * n_per_row) + cq);
-                rmse_quad(xv, load_codes<BITS>(blocks + (r * nb + b) * block_bytes<BITS>(), qd), col, emax);
+                rmse_quad(xv, load_codes<BITS>(blocks + (r * nb + b) * block_bytes<BITS>(), qd), col, emax,
+                          y != nullptr ? reinterpret_cast<float4*>(y + r * n_per_row) + cq : nullptr);
             }
             float4 w = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
             if (qw != nullptr) w = __ldg(reinterpret_cast<const float4*>(qw + qrow * n_per_row) + cq);
@@ -320,14 +330,14 @@ namespace {
 
 template <int BITS>
 iqq_status rmse_launch(const float* x, const void* blocks, const float* qw, int64_t nrows, int64_t n_per_row,
-                       int64_t rows_per_qw, double* d_acc, void* stream)
+                       int64_t rows_per_qw, double* d_acc, void* stream, float* y = nullptr)
 {
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
     if (n_per_row % IQQ_Q4_0_BLOCK_VALUES != 0) return IQQ_ERR_SHAPE;
     if (nrows == 0 || n_per_row == 0) return IQQ_OK;
     if (x == nullptr || blocks == nullptr || d_acc == nullptr) return IQQ_ERR_NULL;
     if (!iqq::aligned(x, 16) || !iqq::aligned(blocks, 2) || (qw && !iqq::aligned(qw, 16)) ||
-        !iqq::aligned(d_acc, 8))
+        !iqq::aligned(d_acc, 8) || !iqq::aligned(y, 16))
         return IQQ_ERR_ALIGN;
     const int64_t nq = n_per_row / 4;
     const int64_t gx = (nq + kThreads - 1) / kThreads;
@@ -342,7 +352,7 @@ iqq_status rmse_launch(const float* x, const void* blocks, const float* qw, int6
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
     weighted_rmse_kernel<BITS><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         x, static_cast<const uint8_t*>(blocks), qw, nrows, n_per_row, rows_per_qw,
-        static_cast<int>(rpc), d_acc);
+        static_cast<int>(rpc), d_acc, y);
     return iqq::launch_status();
 }
 
@@ -353,6 +363,20 @@ extern "C" iqq_status iqq_weighted_rmse(const float* x, const void* blocks, cons
                                         double* d_acc, void* stream)
 {
     return rmse_launch<4>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+}
+
+extern "C" iqq_status iqq_dequant_rmse_qx(int bits, const float* x, const void* blocks, const float* qw,
+                                          int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, float* y,
+                                          double* d_acc, void* stream)
+{
+    if (y == nullptr && nrows > 0 && n_per_row > 0) return IQQ_ERR_NULL;
+    switch (bits) {
+    case 4: return rmse_launch<4>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    case 5: return rmse_launch<5>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    case 6: return rmse_launch<6>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    case 8: return rmse_launch<8>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    default: return IQQ_ERR_ARG;
+    }
 }
 
 extern "C" iqq_status iqq_weighted_rmse_qx(int bits, const float* x, const void* blocks, const float* qw,

@@ -250,11 +250,17 @@ __device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, fl
     }
 }
 
-template <int BITS>
+// EPI: the epilogue of the blocks just written may also (y_out) store their dequantized
+// values y = fp16(d) * l (exact in binary32, the dequantization's bits) and (acc_out)
+// accumulate their round trip exactly as the weighted-RMSE reduction does: with e = x - y
+// in binary32, {sum qw e^2, sum qw, sum e^2} in binary64 and max |e|, one set of atomics
+// per warp (no CTA barrier).
+template <int BITS, bool EPI>
 __global__ void __launch_bounds__(kThreads, IQQ_Q4_MIN_CTAS)
 qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
-              int chunks_per_row, const float* __restrict__ row_sigma2, uint32_t* __restrict__ flags)
+              int chunks_per_row, const float* __restrict__ row_sigma2, float* __restrict__ y_out,
+              double* __restrict__ acc_out, uint32_t* __restrict__ flags)
 {
     extern __shared__ float smem[];
     __shared__ double s_red[kWarps];
@@ -534,6 +540,57 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 }
             }
         }
+        if (EPI) {
+            const bool want_acc = acc_out != nullptr;  // uniform
+            double ew = 0.0, eq = 0.0, ee = 0.0;
+            float em = 0.0f;
+            if (valid) {
+                const float dq = __half2float(__ushort_as_half(d16));
+                float4* yb = y_out != nullptr ? reinterpret_cast<float4*>(y_out + row * n_per_row + b * QK) : nullptr;
+                // the imatrix row again (recomputed rather than kept live across the sweep)
+                const float* qre = qw != nullptr ? qw + (rows_per_qw > 0 ? row / rows_per_qw : 0) * n_per_row
+                                                 : nullptr;
+                const float4* q4p = qre != nullptr ? reinterpret_cast<const float4*>(qre + b * QK) : nullptr;
+#pragma unroll 2
+                for (int i = 0; i < QK / 4; ++i) {
+                    float yk[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) yk[k] = __fmul_rn(dq, my_l[4 * i + k]);
+                    if (yb != nullptr) __stcs(yb + i, make_float4(yk[0], yk[1], yk[2], yk[3]));
+                    if (want_acc) {
+                        const float4 qv = q4p != nullptr ? __ldg(q4p + i) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+                        const float qk[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float e = __fsub_rn(my_x[4 * i + k], yk[k]);
+                            const double ed = static_cast<double>(e);
+                            const double e2 = ed * ed;  // exact
+                            ew = fma(static_cast<double>(qk[k]), e2, ew);
+                            eq += static_cast<double>(qk[k]);
+                            ee += e2;
+                            em = fmaxf(em, fabsf(e));
+                        }
+                    }
+                }
+            }
+            if (want_acc) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    ew += __shfl_xor_sync(kFull, ew, o);
+                    eq += __shfl_xor_sync(kFull, eq, o);
+                    ee += __shfl_xor_sync(kFull, ee, o);
+                    em = fmaxf(em, __shfl_xor_sync(kFull, em, o));
+                }
+                if (lane == 0) {
+                    atomicAdd(acc_out + 0, ew);
+                    atomicAdd(acc_out + 1, eq);
+                    atomicAdd(acc_out + 2, ee);
+                    // non-negative binary64 values order like their bit patterns
+                    atomicMax(reinterpret_cast<unsigned long long*>(acc_out + 3),
+                              static_cast<unsigned long long>(__double_as_longlong(static_cast<double>(em))));
+                }
+            }
+        }
         iqq::raise_flags(flags, bad);
         __syncwarp();  // the warp's shared memory is rewritten by the next row
     }
@@ -601,10 +658,10 @@ int64_t workspace_bytes_for(int64_t nrows, int64_t n_per_row)
     return (nrows * 4 + 255) / 256 * 256;
 }
 
-template <int BITS>
+template <int BITS, bool EPI>
 iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
-                     int64_t rows_per_qw, int weight_mode, const float* row_sigma2, uint32_t* d_flags,
-                     void* stream)
+                     int64_t rows_per_qw, int weight_mode, const float* row_sigma2, float* y_out, double* acc,
+                     uint32_t* d_flags, void* stream)
 {
     const int64_t nb = n_per_row / QK;
     const int64_t chunks = (nb + kThreads - 1) / kThreads;
@@ -615,22 +672,35 @@ iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return iqq::launch_status();
     if (configured_device != dev) {
-        if (cudaFuncSetAttribute(qx_0_w_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(qx_0_w_kernel<BITS, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kDynSmem)) != cudaSuccess)
             return iqq::launch_status();
         configured_device = dev;
     }
-    qx_0_w_kernel<BITS><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
+    qx_0_w_kernel<BITS, EPI><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
         x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode,
-        static_cast<int>(chunks), row_sigma2, d_flags);
+        static_cast<int>(chunks), row_sigma2, y_out, acc, d_flags);
     return iqq::launch_status();
 }
 
+template <int BITS>
+iqq_status launch_bits(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
+                       int64_t rows_per_qw, int weight_mode, const float* rs, float* y_out, double* acc,
+                       uint32_t* d_flags, void* stream)
+{
+    if (acc != nullptr || y_out != nullptr)
+        return launch_qx<BITS, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc,
+                                     d_flags, stream);
+    return launch_qx<BITS, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, nullptr, nullptr,
+                                  d_flags, stream);
+}
+
 // workspace == nullptr: the fused reduction.  Otherwise it holds at least
-// workspace_bytes_for(nrows, n_per_row) bytes (checked by the caller).
+// workspace_bytes_for(nrows, n_per_row) bytes (checked by the caller).  acc: optional
+// round-trip error accumulator (8-byte aligned, checked by the caller).
 iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int64_t nrows,
                        int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
-                       uint32_t* d_flags, void* stream)
+                       uint32_t* d_flags, void* stream, double* acc = nullptr, float* y_out = nullptr)
 {
     if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
@@ -652,10 +722,10 @@ iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int
         rs = ws;
     }
     switch (bits) {
-    case 4: return launch_qx<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
-    case 5: return launch_qx<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
-    case 6: return launch_qx<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
-    default: return launch_qx<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, d_flags, stream);
+    case 4: return launch_bits<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
+    case 5: return launch_bits<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
+    case 6: return launch_bits<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
+    default: return launch_bits<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
     }
 }
 
@@ -720,6 +790,25 @@ extern "C" iqq_status iqq_quantize_qx_0_w_static(int bits, const float* x, const
         if (st != IQQ_OK) return st;
     }
     return IQQ_OK;
+}
+
+extern "C" iqq_status iqq_quantize_qx_0_w_ex(int bits, const float* x, const float* qw, void* out,
+                                             int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                             int weight_mode, void* workspace, size_t workspace_bytes,
+                                             float* y_out, double* d_acc, uint32_t* d_flags, void* stream)
+{
+    if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
+    if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0 || n_per_row % QK != 0) return IQQ_ERR_SHAPE;
+    const int64_t need = workspace_bytes_for(nrows, n_per_row);
+    void* ws = nullptr;
+    if (need > 0 && workspace != nullptr) {
+        if (workspace_bytes < static_cast<size_t>(need)) return IQQ_ERR_SHAPE;
+        if (!iqq::aligned(workspace, 16)) return IQQ_ERR_ALIGN;
+        ws = workspace;
+    }
+    if (!iqq::aligned(d_acc, 8) || !iqq::aligned(y_out, 16)) return IQQ_ERR_ALIGN;
+    return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, ws, d_flags, stream, d_acc,
+                       y_out);
 }
 
 extern "C" size_t iqq_quantize_qx_0_w_workspace_bytes(int64_t nrows, int64_t n_per_row)

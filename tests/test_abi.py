@@ -28,7 +28,8 @@ def test_header_declares_the_boundary():
               "iqq_weighted_rmse", "iqq_quantize_q8_1", "iqq_status_string",
               "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128",
               "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
-              "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch"):
+              "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch",
+              "iqq_quantize_qx_0_w_ex", "iqq_dequant_rmse_qx"):
         assert n in names
 
 
@@ -126,6 +127,17 @@ def test_host_validation_without_gpu(lib):
     assert B(ctypes.cast(empty, V), 2, None, None) == 0
     unaligned = (m.GemvProblem * 1)(m.GemvProblem(8, 16, 16, 4, 128, 1))
     assert B(ctypes.cast(unaligned, V), 1, None, None) == 3
+    X = lib.iqq_quantize_qx_0_w_ex
+    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, None, 0, None, V(12), None, None) == 3   # d_acc alignment
+    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, None, 0, V(8), None, None, None) == 3    # y alignment
+    assert X(4, V(16), None, V(16), 2, 53248, 0, 0, V(16), 8, None, None, None, None) == 2  # workspace too small
+    assert X(9, V(16), None, V(16), 2, 4096, 0, 0, None, 0, None, None, None, None) == 5
+    assert X(4, None, None, None, 0, 4096, 0, 0, None, 0, None, None, None, None) == 0
+    DR = lib.iqq_dequant_rmse_qx
+    assert DR(4, V(16), V(16), None, 1, 32, 0, None, V(16), None) == 1
+    assert DR(4, V(16), V(16), None, 1, 32, 0, V(8), V(16), None) == 3
+    assert DR(7, V(16), V(16), None, 1, 32, 0, V(16), V(16), None) == 5
+    assert DR(4, V(16), V(16), None, 1, 48, 0, V(16), V(16), None) == 2
     # Q4_0 x Q8_K_128 matrix-vector product
     G = lib.iqq_gemv_q4_0_q8_k128
     assert G(V(16), V(16), V(16), 4, 96, 1, None, None) == 2          # k not a multiple of 128

@@ -224,6 +224,14 @@ def test_qx_0_weighted_and_dequant(iqq, synth, bits, rows, n):
     ref = oracle.weighted_rmse_qx(bits, x, g.cpu().numpy(), qw)
     a = acc.cpu().numpy()
     assert np.allclose(a[:3], ref[:3], rtol=1e-9, atol=0) and a[3] == ref[3]
+    # the one-pass dequantization + round trip: same y bits, same sums
+    y2 = torch.empty_like(xd)
+    acc2 = torch.zeros(4, dtype=torch.float64, device="cuda")
+    iqq.iqq_dequant_rmse_qx(bits, xd, g, qd, y2, acc2)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, y)
+    a2 = acc2.cpu().numpy()
+    assert np.allclose(a2[:3], ref[:3], rtol=1e-9, atol=0) and a2[3] == ref[3]
     # any differing block: weighted error within 1e-5 of the oracle's
     if not same.all():
         yo = oracle.dequant_qx_0(bits, o, rows, n).reshape(-1, 32).astype(np.float64)
@@ -272,6 +280,36 @@ def test_qx_0_workspace_wide_rows(iqq, synth, bits, rows, n):
     _compare_qx(bits, x, qw, g_ws.cpu().numpy(), o, rows, n)
     assert np.mean(np.all(g_ws.cpu().numpy().reshape(-1, oracle.qx_block_bytes(bits)) ==
                           g_fused.cpu().numpy().reshape(-1, oracle.qx_block_bytes(bits)), axis=1)) >= 0.9999
+
+
+@pytest.mark.parametrize("bits,rows,n,rpq", [(4, 64, 4096, 0), (4, 9, 11008, 3), (5, 5, 53248, 0),
+                                              (8, 3, 12320, 1), (6, 37, 4192, 0)])
+def test_quantize_with_fused_round_trip_error(iqq, synth, bits, rows, n, rpq):
+    """One pass: the quantizer's dequantized output equals the dequantization kernel's bit for
+    bit, its accumulation of the round trip equals the oracle's weighted-RMSE reduction of
+    the same blocks (sums within 1e-9, max |e| exact), and its blocks equal the plain entry
+    point's."""
+    x = synth.weight_matrix(rows, n, seed=60 + rows).numpy()
+    nq = 1 if rpq == 0 else (rows + rpq - 1) // rpq
+    qw = np.stack([synth.imatrix(n, seed=70 + i).numpy() for i in range(nq)])
+    xd, qd = torch.from_numpy(x).cuda(), torch.from_numpy(qw if rpq else qw[0]).cuda()
+    acc = torch.zeros(4, dtype=torch.float64, device="cuda")
+    out = torch.empty(rows * (n // 32) * iqq.QX_0_BLOCK_BYTES[bits], dtype=torch.uint8, device="cuda")
+    nws = iqq.qx_0_w_workspace_bytes(rows, n)
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda") if nws else None
+    y = torch.empty_like(xd)
+    iqq.iqq_quantize_qx_0_w_ex(bits, xd, qd, out, ws, acc, rpq, y=y)
+    plain = iqq.quantize_qx_0_w(bits, xd, qd, rpq)
+    y_ref = iqq.dequant_qx_0(bits, out, rows, n)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref)
+    g = out.cpu().numpy()
+    same = np.mean(np.all(g.reshape(-1, oracle.qx_block_bytes(bits)) ==
+                          plain.cpu().numpy().reshape(-1, oracle.qx_block_bytes(bits)), axis=1))
+    assert same >= 0.9999
+    ref = oracle.weighted_rmse_qx(bits, x, g, qw if rpq else qw[0], rpq)
+    a = acc.cpu().numpy()
+    assert np.allclose(a[:3], ref[:3], rtol=1e-9, atol=0) and a[3] == ref[3]
 
 
 def test_qx_0_workspace_flags_nonfinite(iqq, synth):

@@ -183,3 +183,21 @@ def test_weighted_rmse_closed_form(orc):
         if bits == 4:
             ref = orc.weighted_rmse(x.reshape(1, 96), blk.reshape(1, -1), np.tile(qw, 3))
             assert np.array_equal(acc, ref)
+
+
+def test_weighted_rmse_stacked_imatrix(orc):
+    """One imatrix row per rows_per_qw rows: with constant rows 1, 2, 3 the weight sum is
+    the closed form n * sum_r qw[r // rows_per_qw], for every format."""
+    rng = np.random.default_rng(61)
+    rows, n = 6, 64
+    x = rng.standard_normal((rows, n)).astype(np.float32)
+    for bits in (4, 5, 6, 8):
+        for rpq, nq in ((1, 6), (2, 3), (4, 2), (0, 1)):
+            qw = np.stack([np.full(n, float(i + 1), np.float32) for i in range(nq)])
+            out, _ = orc.quantize_qx_0_w(bits, x, qw if rpq else qw[0], rpq)
+            acc = orc.weighted_rmse_qx(bits, x, out, qw if rpq else qw[0], rpq)
+            expect = n * sum((r // rpq if rpq else 0) + 1 for r in range(rows))
+            assert acc[1] == expect, (bits, rpq, acc[1], expect)
+            e = (x - orc.dequant_qx_0(bits, out, rows, n)).astype(np.float64)
+            qfull = np.array([[(r // rpq if rpq else 0) + 1.0] * n for r in range(rows)])
+            assert abs(acc[0] - float(np.sum(qfull * e * e))) <= 1e-12 * acc[0]
