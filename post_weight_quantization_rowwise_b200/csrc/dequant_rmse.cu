@@ -56,10 +56,10 @@ __device__ __forceinline__ float code_value(uint32_t nib4, int k)
 #define IQQ_DQ_CTAS 16   // CTAs per SM in the grid (dequant)
 #endif
 #ifndef IQQ_RMSE_UNROLL
-#define IQQ_RMSE_UNROLL 2  // independent rows in flight per thread (weighted RMSE)
+#define IQQ_RMSE_UNROLL 4  // independent rows in flight per thread (weighted RMSE)
 #endif
 #ifndef IQQ_RMSE_CTAS
-#define IQQ_RMSE_CTAS 16   // CTAs per SM in the grid (weighted RMSE)
+#define IQQ_RMSE_CTAS 4    // CTAs per SM in the grid (weighted RMSE; measured best of 4-32 with 1-8 rows in flight)
 #endif
 #ifndef IQQ_RMSE_MIN_ROWS
 #define IQQ_RMSE_MIN_ROWS 8  // rows per CTA at least (weighted RMSE)

@@ -19,8 +19,14 @@
 
 namespace {
 
+#ifndef IQQ_Q8_UNROLL
+#define IQQ_Q8_UNROLL 4  // 128-value blocks in flight per warp
+#endif
+#ifndef IQQ_Q8_CTAS
+#define IQQ_Q8_CTAS 8    // resident CTAs of 256 threads per SM in the grid
+#endif
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = IQQ_Q8_UNROLL;
 
 // rint with the cvt.rni saturating conversion: +-Inf -> INT_MAX / INT_MIN,
 // NaN -> 0; then the symmetric int8 clamp.
@@ -99,7 +105,7 @@ extern "C" iqq_status iqq_quantize_q8_k128(const float* x, void* out, int64_t nr
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t warps_needed = (nblocks + kUnroll - 1) / kUnroll;
     const int64_t ctas_needed = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
-    const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 resident CTAs of 256 threads per SM
+    const int64_t cap = static_cast<int64_t>(sms) * IQQ_Q8_CTAS;
     const int grid = static_cast<int>(ctas_needed < cap ? ctas_needed : cap);
     q8_k128_kernel<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const float4*>(x), static_cast<uint8_t*>(out), nblocks, d_flags);
