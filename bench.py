@@ -49,9 +49,9 @@ RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
-# kernel (4096x4096 launch: 67.196 MB read + 1.494 MB written for 16,777,216 values); set
+# kernel (4096x4096 launch: see the qx_0_w_kernel profile summary, 4.111 B per value); set
 # to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = 4.0942
+Q4_0_DRAM_BYTES_PER_VALUE = 4.1110
 
 
 def peaks():

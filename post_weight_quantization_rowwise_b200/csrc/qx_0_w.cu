@@ -78,6 +78,9 @@ constexpr int kUb = kAwx + 32 * kRow4;
 constexpr int kWarpFloats = kUb + 32 * kRow4;
 static_assert(kScratch + 2 * 32 * kRow1 <= kWarpFloats, "staging fits in the sweep area");
 
+#ifndef IQQ_PASS1_SPEC
+#define IQQ_PASS1_SPEC 2  // greedy pass 1: trials evaluated together against one state (measured: 2 best of 1-8)
+#endif
 #ifndef IQQ_Q4_MIN_CTAS
 #define IQQ_Q4_MIN_CTAS 4  // resident CTAs per SM the register budget is sized for
 #endif
@@ -443,36 +446,59 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
                 suml2 = __fmaf_rn(wj, __fmul_rn(l, l), suml2);
             }
         }
-        // greedy pass 1: this thread's block, sequential over j, exactly as defined
+        // greedy pass 1: this thread's block, sequential over j, exactly as defined.  The
+        // state (sumlx, suml2, score, d) changes only when a move is accepted, so the trials
+        // of IQQ_PASS1_SPEC consecutive elements are evaluated together against the current
+        // state; the first one that passes the cheap rejection test is then decided exactly
+        // as the sequential pass decides it, and the scan resumes after it.  The sequence of
+        // accepted moves and every rounding are those of the element-by-element pass.
         bool changed = false;
         if (mode == 2) {
             float d = __fdiv_rn(sumlx, suml2);
-#pragma unroll 2
-            for (int j = 0; j < QK; ++j) {
-                const float xj = my_x[j], wj = my_w[j], lj = my_l[j];
-                const float g = __fmul_rn(d, __fmul_rn(wj, __fsub_rn(xj, __fmul_rn(d, lj))));
-                const float sg = g > 0.0f ? 1.0f : -1.0f;
-                const float ln = __fadd_rn(lj, sg);
-                const float nlx = __fadd_rn(sumlx, __fmul_rn(sg, __fmul_rn(wj, xj)));
-                const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), suml2);
-                const float a2 = __fmul_rn(nlx, nlx);
-                // rejected for certain when fl(nlx^2) <= thr = fl(fl(score*nl2)*(1 - 2^-22)):
-                // with no underflow or overflow (thr in [1e-30, 1e30]) thr < score*nl2, so
-                // then nlx^2/nl2 < score exactly and its rounded quotient cannot exceed score
-                const float thr = __fmul_rn(__fmul_rn(score, nl2), 0.99999976158142089844f);
-                const bool maybe = !(a2 <= thr && thr >= 1e-30f && thr <= 1e30f);
-                if (maybe && (g > 0.0f || g < 0.0f) && ln >= static_cast<float>(-NMAX) &&
-                    ln <= static_cast<float>(NMAX - 1) && nl2 > 0.0f) {
-                    const float ns = __fdiv_rn(a2, nl2);
-                    if (ns > score) {
-                        my_l[j] = ln;
-                        sumlx = nlx;
-                        suml2 = nl2;
-                        score = ns;
-                        d = __fdiv_rn(sumlx, suml2);
-                        changed = true;
-                    }
+            constexpr int U = IQQ_PASS1_SPEC;
+            int j = 0;
+#pragma unroll 1
+            while (j < QK) {
+                float t_ln[U], t_nlx[U], t_nl2[U], t_a2[U];
+                int first = U;
+#pragma unroll
+                for (int u = U - 1; u >= 0; --u) {
+                    const int jj = j + u < QK ? j + u : QK - 1;  // past the end: recomputes the last, unused
+                    const float xj = my_x[jj], wj = my_w[jj], lj = my_l[jj];
+                    const float g = __fmul_rn(d, __fmul_rn(wj, __fsub_rn(xj, __fmul_rn(d, lj))));
+                    const float sg = g > 0.0f ? 1.0f : -1.0f;
+                    t_ln[u] = __fadd_rn(lj, sg);
+                    t_nlx[u] = __fadd_rn(sumlx, __fmul_rn(sg, __fmul_rn(wj, xj)));
+                    t_nl2[u] = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), suml2);
+                    t_a2[u] = __fmul_rn(t_nlx[u], t_nlx[u]);
+                    // rejected for certain when fl(nlx^2) <= thr = fl(fl(score*nl2)*(1 - 2^-22)):
+                    // with no underflow or overflow (thr in [1e-30, 1e30]) thr < score*nl2, so
+                    // then nlx^2/nl2 < score exactly and its rounded quotient cannot exceed score
+                    const float thr = __fmul_rn(__fmul_rn(score, t_nl2[u]), 0.99999976158142089844f);
+                    const bool maybe = !(t_a2[u] <= thr && thr >= 1e-30f && thr <= 1e30f);
+                    const bool cand = maybe && (g > 0.0f || g < 0.0f) && t_ln[u] >= static_cast<float>(-NMAX) &&
+                                      t_ln[u] <= static_cast<float>(NMAX - 1) && t_nl2[u] > 0.0f && j + u < QK;
+                    if (cand) first = u;  // descending u: the lowest candidate wins
                 }
+                if (first == U) {
+                    j += U;
+                    continue;
+                }
+                // element j + first: the sequential pass's decision, from the same state
+                float ln = t_ln[0], nlx = t_nlx[0], nl2 = t_nl2[0], a2 = t_a2[0];
+#pragma unroll
+                for (int u = 1; u < U; ++u)
+                    if (first == u) { ln = t_ln[u]; nlx = t_nlx[u]; nl2 = t_nl2[u]; a2 = t_a2[u]; }
+                const float ns = __fdiv_rn(a2, nl2);
+                if (ns > score) {
+                    my_l[j + first] = ln;
+                    sumlx = nlx;
+                    suml2 = nl2;
+                    score = ns;
+                    d = __fdiv_rn(sumlx, suml2);
+                    changed = true;
+                }
+                j += first + 1;
             }
         }
         // passes 2..5, warp-cooperatively, for the blocks whose first pass moved a code
