@@ -108,9 +108,12 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        return self.summarize(getattr(self, "t0", 0.0), t1)
+
+    def summarize(self, t0: float, t1: float):
+        """Median SM clock, the maximum, and the throttle reasons active in [t0, t1 + 0.1]."""
         mhz, mx, reasons = [], None, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        t0 = getattr(self, "t0", 0.0)
         for ts, ln in self.lines:
             if ts < t0 or ts > t1 + 0.1:
                 continue

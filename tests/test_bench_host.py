@@ -1,0 +1,53 @@
+"""Host-side logic of bench.py (no GPU): the peak denominators, the clock summary, the
+warm-up guard and the reference arm's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def test_peaks_read_the_measured_file():
+    import bench
+    p = bench.peaks()
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        m = json.load(f)
+    assert p["source"] == "measured"
+    assert p["hbm_gbs"] == float(m["hbm_gbs"]) and p["sm_max_mhz"] == float(m["sm_max_mhz"])
+
+
+def test_clock_summary_keeps_the_window_and_the_reasons():
+    import bench
+    c = bench.ClockSampler(0)
+    row = "0, {mhz}, 1965, 900.0, 0x0, Not Active, Not Active, {sw}, {cap}"
+    c.lines = [(0.5, row.format(mhz=500, sw="Not Active", cap="Not Active")),      # before the window
+               (1.0, row.format(mhz=1965, sw="Not Active", cap="Active")),
+               (1.1, row.format(mhz=1800, sw="Not Active", cap="Not Active")),
+               (1.2, row.format(mhz=1900, sw="Active", cap="Not Active")),
+               (1.3, "garbage"),
+               (9.0, row.format(mhz=100, sw="Not Active", cap="Not Active"))]     # after it
+    out = c.summarize(0.9, 1.25)
+    assert out["samples"] == 3 and out["sm_mhz"] == 1900 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+
+
+def test_warmup_below_three_is_refused():
+    r = subprocess.run([sys.executable, "bench.py", "--warmup", "2"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 2 and "warmup" in r.stderr
+
+
+def test_reference_arm_prints_one_json_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
+                        "--cpu-seconds", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "vs_baseline", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
