@@ -51,7 +51,7 @@ FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
 # kernel (4096x4096 launch: see the qx_0_w_kernel profile summary, 4.111 B per value); set
 # to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = 4.1110
+Q4_0_DRAM_BYTES_PER_VALUE = None
 
 
 def peaks():
@@ -358,6 +358,12 @@ def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
         wm[str(mode)] = {"gelem_s": round(n / qms / 1e6, 3), "wrmse": math.sqrt(a[0] / a[1])}
     out["weight_modes"] = {"tensor": t.name, "modes": "0 qw*sqrt(s2+x2), 1 qw, 2 qw*x2, 3 qw*|x|, "
                            "4 qw*(s2+x2), 5 qw*(sqrt(s2)+|x|)", **wm}
+    fz = {}
+    for f in (0.0, 0.25, 0.5, 1.0, 2.0, 4.0):
+        iqq.iqq_quantize_qx_0_w_ex(4, x, qw, blocks, weight_mode=0, fudge=f)
+        a = iqq.weighted_rmse(x, blocks, qw).cpu().tolist()
+        fz[str(f)] = {"wrmse": math.sqrt(a[0] / a[1])}
+    out["fudge"] = {"tensor": t.name, "mode": "qw*sqrt(fudge*s2 + x2)", **fz}
     del x, qw, blocks
     ab = {}
     for tt in sweep:

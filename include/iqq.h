@@ -145,6 +145,10 @@ iqq_status iqq_quantize_qx_0_w_ws(int bits, const float* x, const float* qw, voi
  * format, an optional workspace, an optional dequantized output and an optional
  * round-trip error accumulator (quantization, dequantization and the weighted RMSE of a
  * tensor in one pass over it).
+ *  fudge            the importance's correction factor ([W] §四 names a fudge factor that
+ *                   corrects the approximate Hessian, without its values): it scales the
+ *                   sigma2 term of weight modes 0, 4 and 5, sigma2 -> fl(fudge * sigma2);
+ *                   1 changes nothing.  Finite and >= 0, else IQQ_ERR_ARG.
  *  workspace, workspace_bytes  as for iqq_quantize_qx_0_w_ws, but optional: with NULL the
  *                   per-CTA row reduction is used for every width.
  *  y_out            optional device float32 [nrows, n_per_row] (16-byte aligned): the
@@ -159,9 +163,9 @@ iqq_status iqq_quantize_qx_0_w_ws(int bits, const float* x, const float* qw, voi
  * Other arguments and errors as for iqq_quantize_qx_0_w.
  */
 iqq_status iqq_quantize_qx_0_w_ex(int bits, const float* x, const float* qw, void* out, int64_t nrows,
-                                  int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
-                                  size_t workspace_bytes, float* y_out, double* d_acc, uint32_t* d_flags,
-                                  void* stream);
+                                  int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
+                                  void* workspace, size_t workspace_bytes, float* y_out, double* d_acc,
+                                  uint32_t* d_flags, void* stream);
 
 /*
  * iqq_quantize_qx_0_w_static -- iqq_quantize_qx_0_w_ws without a caller workspace: the

@@ -61,6 +61,9 @@ def lib():
         L.oracle_quantize_qx_0_w.restype = ctypes.c_int
         L.oracle_quantize_qx_0_w.argtypes = [ctypes.c_int, _f32p, _f32p, _u8p, _i64, _i64, _i64,
                                              ctypes.c_int, _u32p]
+        L.oracle_quantize_qx_0_w_f.restype = ctypes.c_int
+        L.oracle_quantize_qx_0_w_f.argtypes = [ctypes.c_int, _f32p, _f32p, _u8p, _i64, _i64, _i64,
+                                               ctypes.c_int, ctypes.c_float, _u32p]
         L.oracle_dequant_qx_0.restype = ctypes.c_int
         L.oracle_dequant_qx_0.argtypes = [ctypes.c_int, _u8p, _f32p, _i64, _i64]
         L.oracle_qx_block_bytes.restype = ctypes.c_int
@@ -161,8 +164,9 @@ def qx_block_search(xb, w, nmax: int):
     return np.float32(d), L, Ls, info
 
 
-def quantize_qx_0_w(bits: int, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0):
-    """Weighted quantization to the 32-value format with `bits` (4, 5, 6, 8); (blocks, flags)."""
+def quantize_qx_0_w(bits: int, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0, fudge: float = 1.0):
+    """Weighted quantization to the 32-value format with `bits` (4, 5, 6, 8); (blocks, flags).
+    fudge scales the sigma2 term of the importance (weight modes 0, 4, 5)."""
     x = _f32(x)
     nrows, n = x.shape
     qw = None if qw is None else _f32(qw)
@@ -171,8 +175,8 @@ def quantize_qx_0_w(bits: int, x, qw=None, rows_per_qw: int = 0, weight_mode: in
         raise ValueError("bits must be 4, 5, 6 or 8")
     out = np.zeros((nrows, (n // 32) * bb), np.uint8)
     flags = np.zeros(1, np.uint32)
-    rc = lib().oracle_quantize_qx_0_w(bits, _ptr(x, _f32p), _ptr(qw, _f32p), _ptr(out, _u8p), nrows, n,
-                                      rows_per_qw, weight_mode, _ptr(flags, _u32p))
+    rc = lib().oracle_quantize_qx_0_w_f(bits, _ptr(x, _f32p), _ptr(qw, _f32p), _ptr(out, _u8p), nrows, n,
+                                        rows_per_qw, weight_mode, ctypes.c_float(fudge), _ptr(flags, _u32p))
     if rc != 0:
         raise ValueError("oracle_quantize_qx_0_w: bad arguments")
     return out, int(flags[0])

@@ -423,9 +423,14 @@ static int unpack_code(int bits, const uint8_t *blk, int j)
 }
 
 /* Weighted quantization of a tensor to any of the 32-value formats. */
-int oracle_quantize_qx_0_w(int bits, const float *x, const float *qw, uint8_t *out, int64_t nrows,
-                           int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
-                           uint32_t *flags)
+/* fudge: the importance's correction factor of [W] §四 (the fudge factor the code
+ * takes from ggml_get_quantize_fudge_factor; its values are not printed).  Reading: §四
+ * introduces it as a correction of the approximate (diagonal) Hessian, i.e. of the
+ * importance, so it scales the sigma2 term of the forms that have one:
+ * sigma2_used = fl(fudge * sigma2) for modes 0, 4 and 5; fudge = 1 changes nothing. */
+int oracle_quantize_qx_0_w_f(int bits, const float *x, const float *qw, uint8_t *out, int64_t nrows,
+                             int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
+                             uint32_t *flags)
 {
     const int bb = oracle_qx_block_bytes(bits);
     if (bb < 0 || n_per_row % 32 != 0 || nrows < 0 || n_per_row < 0) return -1;
@@ -444,7 +449,7 @@ int oracle_quantize_qx_0_w(int bits, const float *x, const float *qw, uint8_t *o
                 if (qr && qr[j] < 0.0f) *flags |= FLAG_NEG_QW;
             }
         }
-        float sigma2 = oracle_row_sigma2(xr, n_per_row);
+        float sigma2 = fudge * oracle_row_sigma2(xr, n_per_row);
         for (int64_t b = 0; b < nb; ++b) {
             const float *xb = xr + b * 32;
             oracle_block_weights(xb, qr ? qr + b * 32 : NULL, 32, sigma2, weight_mode, w);
@@ -453,6 +458,14 @@ int oracle_quantize_qx_0_w(int bits, const float *x, const float *qw, uint8_t *o
         }
     }
     return 0;
+}
+
+int oracle_quantize_qx_0_w(int bits, const float *x, const float *qw, uint8_t *out, int64_t nrows,
+                           int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                           uint32_t *flags)
+{
+    return oracle_quantize_qx_0_w_f(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, 1.0f,
+                                    flags);
 }
 
 /* y = fp16_to_float(d) * l for any of the 32-value formats (exact in binary32). */

@@ -55,8 +55,8 @@ def _load():
         "iqq_quantize_qx_0_w_ws": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
                                    ctypes.c_size_t, _vp, _vp],
         "iqq_quantize_qx_0_w_static": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
-        "iqq_quantize_qx_0_w_ex": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
-                                   ctypes.c_size_t, _vp, _vp, _vp, _vp],
+        "iqq_quantize_qx_0_w_ex": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
+                                   _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
@@ -402,7 +402,7 @@ def quantize_qx_0_w(bits, x, qw=None, rows_per_qw: int = 0, weight_mode: int = 0
 
 
 def iqq_quantize_qx_0_w_ex(bits, x, qw, out, workspace=None, acc=None, rows_per_qw: int = 0,
-                           weight_mode: int = 0, flags=None, stream=None, y=None):
+                           weight_mode: int = 0, flags=None, stream=None, y=None, fudge: float = 1.0):
     """The general quantizer: optional workspace (uint8), optional dequantized output y
     (float32 like x) and optional round-trip error accumulator acc (float64[4], zeroed by
     the caller)."""
@@ -426,7 +426,7 @@ def iqq_quantize_qx_0_w_ex(bits, x, qw, out, workspace=None, acc=None, rows_per_
     nbytes = 0 if workspace is None else workspace.numel()
     _check("iqq_quantize_qx_0_w_ex",
            _lib.iqq_quantize_qx_0_w_ex(bits, _ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw, weight_mode,
-                                       _ptr(workspace), nbytes, _ptr(y), _ptr(acc), _ptr(flags),
+                                       fudge, _ptr(workspace), nbytes, _ptr(y), _ptr(acc), _ptr(flags),
                                        _stream(stream)))
     return out
 

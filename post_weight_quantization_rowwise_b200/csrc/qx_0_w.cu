@@ -261,7 +261,7 @@ __device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, fl
 template <int BITS, bool EPI>
 __global__ void __launch_bounds__(kThreads, IQQ_Q4_MIN_CTAS)
 qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
-              int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+              int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
               int chunks_per_row, const float* __restrict__ row_sigma2, float* __restrict__ y_out,
               double* __restrict__ acc_out, uint32_t* __restrict__ flags)
 {
@@ -341,6 +341,8 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
             const double sum = block_reduce_sum(acc, s_red);
             sigma2 = static_cast<float>(sum / static_cast<double>(n_per_row));
         }
+        // the importance's correction factor on the sigma2 term (1: none)
+        sigma2 = __fmul_rn(fudge, sigma2);
 
         if (valid && qr != nullptr && (rows_per_qw > 0 ? row % rows_per_qw == 0 : row == 0)) {
             float qmin = q4[0].x, qnf = 0.0f;
@@ -686,8 +688,8 @@ int64_t workspace_bytes_for(int64_t nrows, int64_t n_per_row)
 
 template <int BITS, bool EPI>
 iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
-                     int64_t rows_per_qw, int weight_mode, const float* row_sigma2, float* y_out, double* acc,
-                     uint32_t* d_flags, void* stream)
+                     int64_t rows_per_qw, int weight_mode, float fudge, const float* row_sigma2, float* y_out,
+                     double* acc, uint32_t* d_flags, void* stream)
 {
     const int64_t nb = n_per_row / QK;
     const int64_t chunks = (nb + kThreads - 1) / kThreads;
@@ -704,21 +706,21 @@ iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, 
         configured_device = dev;
     }
     qx_0_w_kernel<BITS, EPI><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
-        x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode,
+        x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode, fudge,
         static_cast<int>(chunks), row_sigma2, y_out, acc, d_flags);
     return iqq::launch_status();
 }
 
 template <int BITS>
 iqq_status launch_bits(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
-                       int64_t rows_per_qw, int weight_mode, const float* rs, float* y_out, double* acc,
-                       uint32_t* d_flags, void* stream)
+                       int64_t rows_per_qw, int weight_mode, float fudge, const float* rs, float* y_out,
+                       double* acc, uint32_t* d_flags, void* stream)
 {
     if (acc != nullptr || y_out != nullptr)
-        return launch_qx<BITS, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc,
-                                     d_flags, stream);
-    return launch_qx<BITS, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, nullptr, nullptr,
-                                  d_flags, stream);
+        return launch_qx<BITS, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out,
+                                     acc, d_flags, stream);
+    return launch_qx<BITS, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, nullptr,
+                                  nullptr, d_flags, stream);
 }
 
 // workspace == nullptr: the fused reduction.  Otherwise it holds at least
@@ -726,7 +728,8 @@ iqq_status launch_bits(const float* x, const float* qw, void* out, int64_t nrows
 // round-trip error accumulator (8-byte aligned, checked by the caller).
 iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int64_t nrows,
                        int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
-                       uint32_t* d_flags, void* stream, double* acc = nullptr, float* y_out = nullptr)
+                       uint32_t* d_flags, void* stream, double* acc = nullptr, float* y_out = nullptr,
+                       float fudge = 1.0f)
 {
     if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
@@ -748,10 +751,10 @@ iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int
         rs = ws;
     }
     switch (bits) {
-    case 4: return launch_bits<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
-    case 5: return launch_bits<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
-    case 6: return launch_bits<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
-    default: return launch_bits<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, rs, y_out, acc, d_flags, stream);
+    case 4: return launch_bits<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    case 5: return launch_bits<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    case 6: return launch_bits<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    default: return launch_bits<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
     }
 }
 
@@ -820,8 +823,9 @@ extern "C" iqq_status iqq_quantize_qx_0_w_static(int bits, const float* x, const
 
 extern "C" iqq_status iqq_quantize_qx_0_w_ex(int bits, const float* x, const float* qw, void* out,
                                              int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
-                                             int weight_mode, void* workspace, size_t workspace_bytes,
-                                             float* y_out, double* d_acc, uint32_t* d_flags, void* stream)
+                                             int weight_mode, float fudge, void* workspace,
+                                             size_t workspace_bytes, float* y_out, double* d_acc,
+                                             uint32_t* d_flags, void* stream)
 {
     if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0 || n_per_row % QK != 0) return IQQ_ERR_SHAPE;
@@ -833,8 +837,9 @@ extern "C" iqq_status iqq_quantize_qx_0_w_ex(int bits, const float* x, const flo
         ws = workspace;
     }
     if (!iqq::aligned(d_acc, 8) || !iqq::aligned(y_out, 16)) return IQQ_ERR_ALIGN;
+    if (!(fudge >= 0.0f) || !isfinite(fudge)) return IQQ_ERR_ARG;
     return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, ws, d_flags, stream, d_acc,
-                       y_out);
+                       y_out, fudge);
 }
 
 extern "C" size_t iqq_quantize_qx_0_w_workspace_bytes(int64_t nrows, int64_t n_per_row)

@@ -128,11 +128,13 @@ def test_host_validation_without_gpu(lib):
     unaligned = (m.GemvProblem * 1)(m.GemvProblem(8, 16, 16, 4, 128, 1))
     assert B(ctypes.cast(unaligned, V), 1, None, None) == 3
     X = lib.iqq_quantize_qx_0_w_ex
-    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, None, 0, None, V(12), None, None) == 3   # d_acc alignment
-    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, None, 0, V(8), None, None, None) == 3    # y alignment
-    assert X(4, V(16), None, V(16), 2, 53248, 0, 0, V(16), 8, None, None, None, None) == 2  # workspace too small
-    assert X(9, V(16), None, V(16), 2, 4096, 0, 0, None, 0, None, None, None, None) == 5
-    assert X(4, None, None, None, 0, 4096, 0, 0, None, 0, None, None, None, None) == 0
+    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, None, V(12), None, None) == 3   # d_acc alignment
+    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, V(8), None, None, None) == 3    # y alignment
+    assert X(4, V(16), None, V(16), 2, 53248, 0, 0, 1.0, V(16), 8, None, None, None, None) == 2  # workspace too small
+    assert X(9, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, None, None, None, None) == 5
+    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, -1.0, None, 0, None, None, None, None) == 5   # fudge < 0
+    assert X(4, V(16), None, V(16), 2, 4096, 0, 0, float("nan"), None, 0, None, None, None, None) == 5
+    assert X(4, None, None, None, 0, 4096, 0, 0, 1.0, None, 0, None, None, None, None) == 0
     DR = lib.iqq_dequant_rmse_qx
     assert DR(4, V(16), V(16), None, 1, 32, 0, None, V(16), None) == 1
     assert DR(4, V(16), V(16), None, 1, 32, 0, V(8), V(16), None) == 3

@@ -245,7 +245,7 @@ def test_qx_0_weighted_and_dequant(iqq, synth, bits, rows, n):
             assert abs(eg - eo) <= 1e-5 * eo
 
 
-def _compare_qx(bits, x, qw, g, o, rows, n, min_exact=0.9999):
+def _compare_qx(bits, x, qw, g, o, rows, n, min_exact=0.9999, mode=0, fudge=1.0):
     bb = oracle.qx_block_bytes(bits)
     gb = g.reshape(-1, bb)
     ob = o.reshape(-1, bb)
@@ -257,8 +257,8 @@ def _compare_qx(bits, x, qw, g, o, rows, n, min_exact=0.9999):
         xb = x.reshape(-1, 32).astype(np.float64)
         for i in np.nonzero(~same)[0]:
             r, c = divmod(int(i), n // 32)
-            w = oracle.block_weights(x[r, 32 * c:32 * c + 32], qw[32 * c:32 * c + 32],
-                                     oracle.row_sigma2(x[r]), 0).astype(np.float64)
+            s2 = float(np.float32(fudge) * np.float32(oracle.row_sigma2(x[r])))
+            w = oracle.block_weights(x[r, 32 * c:32 * c + 32], qw[32 * c:32 * c + 32], s2, mode).astype(np.float64)
             eg, eo = np.sum(w * (xb[i] - yg[i]) ** 2), np.sum(w * (xb[i] - yo[i]) ** 2)
             assert abs(eg - eo) <= 1e-5 * eo
 
@@ -310,6 +310,21 @@ def test_quantize_with_fused_round_trip_error(iqq, synth, bits, rows, n, rpq):
     ref = oracle.weighted_rmse_qx(bits, x, g, qw if rpq else qw[0], rpq)
     a = acc.cpu().numpy()
     assert np.allclose(a[:3], ref[:3], rtol=1e-9, atol=0) and a[3] == ref[3]
+
+
+@pytest.mark.parametrize("bits,mode,fudge", [(4, 0, 0.5), (4, 0, 4.0), (4, 0, 0.0), (4, 4, 2.0),
+                                              (5, 5, 0.25), (8, 0, 3.0)])
+def test_quantize_fudge_factor(iqq, synth, bits, mode, fudge):
+    """The importance's correction factor on sigma2 against the oracle's reading of it."""
+    rows, n = 48, 4096
+    x = synth.weight_matrix(rows, n, seed=90 + bits + mode).numpy()
+    qw = synth.imatrix(n, seed=91).numpy()
+    xd, qd = torch.from_numpy(x).cuda(), torch.from_numpy(qw).cuda()
+    out = torch.empty(rows * (n // 32) * iqq.QX_0_BLOCK_BYTES[bits], dtype=torch.uint8, device="cuda")
+    iqq.iqq_quantize_qx_0_w_ex(bits, xd, qd, out, weight_mode=mode, fudge=fudge)
+    torch.cuda.synchronize()
+    o, _ = oracle.quantize_qx_0_w(bits, x, qw, 0, mode, fudge=fudge)
+    _compare_qx(bits, x, qw, out.cpu().numpy(), o, rows, n, mode=mode, fudge=fudge)
 
 
 def test_qx_0_workspace_flags_nonfinite(iqq, synth):
@@ -378,6 +393,26 @@ def test_dequant_bit_exact(iqq, synth):
     yg = iqq.dequant_q4_0(torch.from_numpy(raw.reshape(64, -1)).cuda(), 64, 2048)
     yo = oracle.dequant_q4_0(raw.reshape(64, -1), 64, 2048)
     assert np.array_equal(yg.cpu().numpy().view(np.uint32), yo.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", [(4096, 4096), (11008, 4096), (4096, 11008)])
+def test_dequant_rmse_one_pass_full_size(iqq, synth, shape):
+    """The bench's one-pass dequantization + round trip at the layer set's full sizes, in its
+    launch configuration: every dequantized value bit-exact against the oracle's decoder, and
+    the sums of the whole tensor within 1e-9 of the oracle's reduction."""
+    r, n = shape
+    xg = synth.weight_matrix(r, n, seed=700 + r + n, bf16=True, device="cuda")
+    qg = synth.imatrix(n, seed=n + 7, device="cuda")
+    blocks = iqq.quantize_q4_0_w(xg, qg)
+    y = torch.empty_like(xg)
+    acc = torch.zeros(4, dtype=torch.float64, device="cuda")
+    iqq.iqq_dequant_rmse_qx(4, xg, blocks, qg, y, acc)
+    torch.cuda.synchronize()
+    x, qw, b = xg.cpu().numpy(), qg.cpu().numpy(), blocks.cpu().numpy()
+    assert np.array_equal(y.cpu().numpy(), oracle.dequant_q4_0(b, r, n))
+    ref = oracle.weighted_rmse(x, b, qw)
+    a = acc.cpu().numpy()
+    assert np.allclose(a[:3], ref[:3], rtol=1e-9, atol=0) and a[3] == ref[3]
 
 
 @pytest.mark.parametrize("rows_per_qw", [0, 256])

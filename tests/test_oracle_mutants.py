@@ -42,6 +42,8 @@ MUTANTS = {
                          "const int nib = i < 16 ? (wb[2 + i] >> 4) : (wb[2 + i - 16] & 0xf);"),
     "dot_activation_scale_dropped": ("const double av = (double)d8 * (double)(int8_t)ab[4 + j % ORACLE_QK8];",
                                      "const double av = (double)(int8_t)ab[4 + j % ORACLE_QK8];"),
+    "fudge_dropped": ("float sigma2 = fudge * oracle_row_sigma2(xr, n_per_row);",
+                      "float sigma2 = oracle_row_sigma2(xr, n_per_row);"),
     "fp16_ties_down": ("if (rem > half || (rem == half && (q & 1u))) q += 1u;",
                        "if (rem > half) q += 1u;"),
 }

@@ -201,3 +201,34 @@ def test_weighted_rmse_stacked_imatrix(orc):
             e = (x - orc.dequant_qx_0(bits, out, rows, n)).astype(np.float64)
             qfull = np.array([[(r // rpq if rpq else 0) + 1.0] * n for r in range(rows)])
             assert abs(acc[0] - float(np.sum(qfull * e * e))) <= 1e-12 * acc[0]
+
+
+@pytest.mark.parametrize("bits", (4, 5, 8))
+def test_fudge_factor_special_cases(orc, bits):
+    """[W] §四's fudge factor, read as scaling the sigma2 term of the importance: fudge = 1
+    is the plain quantizer; fudge = 0 removes sigma2, so qw*sqrt(sigma2 + x^2) becomes
+    qw*|x| (sqrt of the rounded x^2 rounds back to |x| for normal x), qw*(sigma2 + x^2)
+    becomes qw*x^2 and qw*(sqrt(sigma2) + |x|) becomes qw*|x| -- bit for bit; and a
+    power-of-two fudge scales sigma2 exactly, so it equals quantizing with that sigma2."""
+    rng = np.random.default_rng(70 + bits)
+    x = (rng.standard_normal((12, 256)) * 0.02).astype(np.float32)
+    qw = np.exp(rng.standard_normal(256)).astype(np.float32)
+    plain, _ = orc.quantize_qx_0_w(bits, x, qw, 0, 0)
+    assert np.array_equal(orc.quantize_qx_0_w(bits, x, qw, 0, 0, fudge=1.0)[0], plain)
+    m3, _ = orc.quantize_qx_0_w(bits, x, qw, 0, 3)
+    m2, _ = orc.quantize_qx_0_w(bits, x, qw, 0, 2)
+    assert np.array_equal(orc.quantize_qx_0_w(bits, x, qw, 0, 0, fudge=0.0)[0], m3)
+    assert np.array_equal(orc.quantize_qx_0_w(bits, x, qw, 0, 4, fudge=0.0)[0], m2)
+    assert np.array_equal(orc.quantize_qx_0_w(bits, x, qw, 0, 5, fudge=0.0)[0], m3)
+    # modes without sigma2 ignore it
+    for mode in (1, 2, 3):
+        assert np.array_equal(orc.quantize_qx_0_w(bits, x, qw, 0, mode, fudge=7.0)[0],
+                              orc.quantize_qx_0_w(bits, x, qw, 0, mode)[0])
+    # fudge 4 on a row equals the block search with sigma2 * 4, through the block functions
+    f4, _ = orc.quantize_qx_0_w(bits, x[:1], qw, 0, 0, fudge=4.0)
+    s2 = np.float32(4.0) * np.float32(orc.row_sigma2(x[0]))
+    for b in range(0, 256, 32):
+        w = orc.block_weights(x[0, b:b + 32], qw[b:b + 32], float(s2), 0)
+        d, L, _, _ = orc.qx_block_search(x[0, b:b + 32], w, orc.NMAX[bits])
+        blk = _pack(bits, np.float32(d), L.astype(np.int64).tolist(), orc)
+        assert bytes(f4[0, (b // 32) * len(blk):(b // 32 + 1) * len(blk)]) == blk
