@@ -49,9 +49,9 @@ RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
-# kernel (4096x4096 launch: see the qx_0_w_kernel profile summary, 4.111 B per value); set
+# kernel (4096x4096 launch: see the qx_0_w_kernel profile summary, 4.097 B per value); set
 # to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = None
+Q4_0_DRAM_BYTES_PER_VALUE = 4.0975
 
 
 def peaks():
