@@ -11,13 +11,17 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 
-def test_peaks_read_the_measured_file():
+def test_peaks_read_the_measured_file_or_fall_back():
     import bench
     p = bench.peaks()
-    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-        m = json.load(f)
-    assert p["source"] == "measured"
-    assert p["hbm_gbs"] == float(m["hbm_gbs"]) and p["sm_max_mhz"] == float(m["sm_max_mhz"])
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        assert p["source"] == "measured"
+        assert p["hbm_gbs"] == float(m["hbm_gbs"]) and p["sm_max_mhz"] == float(m["sm_max_mhz"])
+    else:
+        assert p == {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
 def test_clock_summary_keeps_the_window_and_the_reasons():
