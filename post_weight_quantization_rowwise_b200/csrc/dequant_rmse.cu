@@ -1,20 +1,21 @@
-// dequant_rmse.cu -- Q4_0 dequantization and the round-trip weighted RMSE on sm_100a.
+// dequant_rmse.cu -- dequantization and the round-trip weighted RMSE of the 32-value
+// block formats on sm_100a.
 //
-// Block format (written by q4_0_w.cu): bytes 0-1 binary16 d (LE), byte 2+i holds
-// code i + 8 in its low nibble and code i+16 + 8 in its high nibble.  A value
-// decodes to fp16(d) * (nibble - 8), exact in binary32.
+// Q4_0 blocks (written by qx_0_w.cu): bytes 0-1 binary16 d (LE), byte 2+i holds code
+// i + 8 in its low nibble and code i+16 + 8 in its high nibble.  A value decodes to
+// fp16(d) * (nibble - 8), exact in binary32.  Q5_0 / Q6_0 / Q8_0 layouts are in iqq.h.
 //
 // The weighted RMSE follows the quantize-stats statistics named on page
 // "量化方法论实证：为什么 LQER/L²QER 难以改进 ik_llama.cpp 的 k-quants 与
 // i-quants" (www.0539edu.com/news/4792009) §3.2 (rmse and maxerr), weighted by
 // the imatrix entries qw: with e = x - y rounded to binary32 it adds
-// {sum qw e^2, sum qw, sum e^2} in binary64 and takes max|e|.  The decoded y
-// never goes to memory.
+// {sum qw e^2, sum qw, sum e^2} in binary64 and takes max|e|.  The decoded y goes
+// to memory only when asked for (the one-pass dequantization + round trip).
 //
-// Both kernels are HBM bound.  Thread mapping: one thread per 4 consecutive
-// values (a "quad"); 8 quads make a block, so the 8 threads of a block share
-// its 18 bytes through L1 and every warp reads/writes 512 contiguous bytes of
-// float data per access.
+// All kernels are HBM bound.  Dequantization: one thread per 4 consecutive values (a
+// "quad"); 8 quads make a block, so the 8 threads of a block share its bytes through L1
+// and every warp writes 512 contiguous bytes per store.  Round trip: one thread per
+// column quad over a run of rows (4 in flight), per-column binary64 sums.
 #include <cuda_fp16.h>
 
 #include "common.cuh"

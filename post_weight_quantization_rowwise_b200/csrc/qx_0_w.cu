@@ -34,10 +34,12 @@
 //  - rint of 0 <= v < 2^22 is either cvt.rni (one conversion-pipe op) or
 //    (v + 1.5*2^23) - 1.5*2^23 (two FMA-pipe adds); the sweep mixes the two
 //    to balance the pipes, and the clamp is one min against B_j;
-//  - greedy pass 1 runs per thread (sequential, as defined); the few blocks
-//    whose first pass moved a code finish passes 2..5 warp-cooperatively;
+//  - greedy pass 1 runs per thread (sequential, as defined, two trials evaluated per
+//    state); the few blocks whose first pass moved a code finish passes 2..5
+//    warp-cooperatively;
 //  - sigma2 is a binary64 CTA reduction over the row (exact squares), the one
-//    place where the summation order differs from the sequential definition.
+//    place where the summation order differs from the sequential definition; rows
+//    spanning 4 or more CTAs may take it from a per-row pass into a workspace.
 //
 // CTA = 128 threads = 128 consecutive blocks of one row ("chunk"); each CTA
 // reduces sigma2 over its whole row (the row is read from HBM once and from L2
@@ -176,11 +178,9 @@ __device__ __forceinline__ void sweep_group(int k0, const float (&xv)[QK], const
                 t[c] = __fmaf_rn(wv[q], __fmul_rn(m, m), t[c]);
             }
         }
-#ifndef IQQ_SWEEP_NO_FENCE
         // compiler-only fence: keeps each group's shared-memory loads beside its
         // arithmetic instead of hoisting all of them (which costs registers)
         asm volatile("" ::: "memory");
-#endif
     }
 #pragma unroll
     for (int c = 0; c < N; ++c) keep_best(s[c], t[c], k0 + c, best, kbest);
