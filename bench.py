@@ -402,13 +402,15 @@ def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
     return out
 
 
-def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
+def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     """The same step through the public API from pinned host buffers, every byte of input
     crossing PCIe each step: per tensor H2D of x and qw, its two kernels, D2H of the
     blocks; H2D of the activations, Q8_K_128, D2H of its blocks and of the accumulator.
     The copies run on their own streams (host to device, device to host) with two device
     staging slots, so tensor i + 1 uploads and tensor i - 1 downloads while tensor i
-    computes; events order every reuse of a slot or buffer."""
+    computes; events order every reuse of a slot or buffer.  ``barrier`` (several ranks)
+    runs after the warm-up pass so that every rank's timed copies share the host at once.
+    Returns (line, seconds per step, values per step)."""
     import torch
     n = 7 * layers
 
@@ -470,6 +472,8 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
 
     one()
     torch.cuda.synchronize()
+    if barrier is not None:
+        barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     end_up, end_dn = torch.cuda.Event(), torch.cuda.Event()
     e0.record(cs)
@@ -485,9 +489,10 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int):
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3 / steps
     elems = sum(t.numel for t in w.tensors[:n]) + w.act.numel()
-    return {"value": elems / sec / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "layers": layers,
-            "h2d_gb_s": round(h2d / sec / 1e9, 1), "overlap": "copies on two streams beside the kernels"}
+    return ({"value": elems / sec / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+             "d2h_bytes_per_step": int(d2h), "layers": layers,
+             "h2d_gb_s": round(h2d / sec / 1e9, 1), "overlap": "copies on two streams beside the kernels"},
+            sec, elems)
 
 
 def main_ours(args):
@@ -550,8 +555,19 @@ def main_ours(args):
                             B200_SMS * FP32_LANES_PER_SM * pk0["sm_max_mhz"] * 1e6 / 1e12, pk0["hbm_gbs"])
 
     e2e = None
-    if rank == 0 and world == 1 and not args.no_e2e:
-        e2e = run_e2e(iqq, w, dev, max(1, min(args.steps, 3)), args.e2e_layers)
+    if not args.no_e2e:
+        # every rank streams its own share of the layers (the pinned host memory of the
+        # whole job stays that of one rank at --e2e-layers); the slowest rank's time counts
+        e2e_layers = max(1, args.e2e_layers // world)
+        e2e, e2e_sec, e2e_elems = run_e2e(iqq, w, dev, max(1, min(args.steps, 3)), e2e_layers,
+                                          barrier=dist.barrier if world > 1 else None)
+        if world > 1:
+            e2e_sec = replicas.max_over_ranks([e2e_sec], device=dev)[0]
+            e2e.update(value=e2e_elems * world / e2e_sec / 1e9,
+                       h2d_bytes_per_step=e2e["h2d_bytes_per_step"] * world,
+                       d2h_bytes_per_step=e2e["d2h_bytes_per_step"] * world,
+                       h2d_gb_s=round(e2e["h2d_bytes_per_step"] * world / e2e_sec / 1e9, 1),
+                       layers_per_rank=e2e_layers, ranks=world)
 
     if world > 1:
         dist.destroy_process_group()
