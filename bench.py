@@ -676,13 +676,15 @@ def main_reference(args):
 
 
 def profile_case(name: str):
-    """Small fixed cases for ncu captures (one GPU, a few launches, tens of MB)."""
+    """Fixed cases for ncu captures (one GPU, a few launches): gemv_11008x4096 (25 MB of
+    blocks) and gemv_16384x53248 (490 MB, the large matrix of the GEMV phase)."""
     import torch
     import post_weight_quantization_rowwise_b200 as iqq
-    if name != "gemv_11008x4096":
+    shapes = {"gemv_11008x4096": (11008, 4096), "gemv_16384x53248": (16384, 53248)}
+    if name not in shapes:
         raise SystemExit(f"unknown profile case {name}")
     torch.manual_seed(0)
-    n_out, k = 11008, 4096
+    n_out, k = shapes[name]
     w = torch.randint(0, 256, (n_out * (k // 32) * 18,), dtype=torch.uint8, device="cuda")
     w.view(-1, 18)[:, 1] &= 0x3B  # finite binary16 scales
     a1 = iqq.quantize_q8_k128(torch.randn(1, k, device="cuda"))

@@ -19,16 +19,18 @@
 // the exact dot product before the final rounding.
 //
 // Mapping (HBM-bound on the weight stream at small token counts): a launch serves up to 64
-// problems (matrices); its CTAs are apportioned to them by weight bytes and each CTA owns a
-// contiguous range of one problem's rows.  Every warp of the CTA takes rows r_begin + warp,
-// + 16, ... and streams each row through its own shared-memory stages in units of up to 64
-// pairs of blocks (2304 bytes), copied with cp.async.bulk and completing on the warp's own
-// mbarriers; lane 0 keeps D units in flight.  A lane takes up to two pairs of blocks per
-// unit (36 bytes each, read as nine 32-bit words: conflict-free because 9 is odd).  Partial
-// sums stay in registers across the units of a row; one butterfly per row.  The CTA
-// synchronizes once, after staging its problem's activations for its token tile (int8 codes
-// with a 16-byte-chunk swizzle that keeps the per-lane 128-bit loads conflict-free, the
-// binary32 scales and the int16 block sums).
+// problems (matrices) with one wave of CTAs.  The problems' weights, laid end to end, are
+// split into equal byte ranges, one per CTA; a CTA takes the rows that start in its range,
+// of one problem or of several in turn (so the wave is balanced to a row whatever the
+// problems' sizes).  Every warp of the CTA takes rows r_begin + warp, + 16, ... and streams
+// each row through its own shared-memory stages in units of up to 64 pairs of blocks (2304
+// bytes), copied with cp.async.bulk and completing on the warp's own mbarriers; lane 0
+// keeps D units in flight.  A lane takes up to two pairs of blocks per unit (36 bytes each,
+// read as nine 32-bit words: conflict-free because 9 is odd).  Partial sums stay in
+// registers across the units of a row; one butterfly per row.  Per problem the CTA
+// synchronizes after staging the problem's activations for its token tile (int8 codes with
+// a 16-byte-chunk swizzle that keeps the per-lane 128-bit loads conflict-free, the binary32
+// scales and the int16 block sums), and once more before staging the next problem's.
 //
 // Every wait on an mbarrier is bounded by a clock limit; on expiry the warp raises
 // IQQ_FLAG_WAIT_TIMEOUT, drains its copies in flight (again bounded) and returns.
@@ -44,7 +46,8 @@ constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kUnitPairs = 64;                    // pairs of blocks per streamed unit
 constexpr int kUnitBytes = kUnitPairs * 36 + 16;  // + room for the 8-byte start offset
-constexpr int kSmemMax = 227 * 1024;
+constexpr int kStaticSmem = kWarps * 4 * 8;        // the kernel's per-warp range slots
+constexpr int kSmemMax = 227 * 1024 - kStaticSmem;  // dynamic shared memory per CTA, at most
 constexpr int kSmemPerSm = 228 * 1024;
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the maximum SM clock
 constexpr uint32_t kSuspendHintNs = 100000;
@@ -122,7 +125,9 @@ constexpr int kMaxBatch = 64;  // problems per launch (kernel parameters stay un
 
 struct Params {
     Problem prob[kMaxBatch];
-    int cta_begin[kMaxBatch + 1];  // CTAs [cta_begin[p], cta_begin[p + 1]) serve problem p
+    int64_t cum_bytes[kMaxBatch + 1];  // weight bytes of the problems before p
+    int64_t share_q, share_r;          // B / C and B % C for B weight bytes over C byte shares
+    int ctas, tiles;                   // C, and the token tiles per share (CTAs = C * tiles)
     int count;
     int stages;                    // D, units in flight per warp
     int off_stage, off_bar;        // shared-memory layout; activations below off_stage
@@ -184,7 +189,7 @@ __device__ __forceinline__ double half_bits_to_double(unsigned short h)
 // i of a block's codes has value i in its low nibble and value i + 16 in its high nibble.
 struct PairW {
     uint32_t qs[8];
-    double d4a, d4b;
+    uint32_t dh;  // the binary16 scales: block a's in the low half, block b's in the high half
 };
 
 __device__ __forceinline__ void load_pair(const uint32_t* w9, PairW& q)
@@ -197,13 +202,15 @@ __device__ __forceinline__ void load_pair(const uint32_t* w9, PairW& q)
         q.qs[m] = __funnelshift_r(w[m], w[m + 1], 16);
         q.qs[4 + m] = w[5 + m];
     }
-    q.d4a = half_bits_to_double(static_cast<unsigned short>(w[0] & 0xffffu));
-    q.d4b = half_bits_to_double(static_cast<unsigned short>(w[4] >> 16));
+    q.dh = __byte_perm(w[0], w[4], 0x7610);
 }
 
-// acc += the two block terms of pair p for one token.
-__device__ __forceinline__ void pair_token(const PairW& q, const uint8_t* q8t, const int16_t* bst,
-                                           const float* d8t, int p, int sw, double& acc)
+__device__ __forceinline__ double scale_a(const PairW& q) { return half_bits_to_double(static_cast<unsigned short>(q.dh & 0xffffu)); }
+__device__ __forceinline__ double scale_b(const PairW& q) { return half_bits_to_double(static_cast<unsigned short>(q.dh >> 16)); }
+
+// acc += the two block terms of pair p for one token (d4a, d4b: the pair's scales).
+__device__ __forceinline__ void pair_token(const PairW& q, double d4a, double d4b, const uint8_t* q8t,
+                                           const int16_t* bst, const float* d8t, int p, int sw, double& acc)
 {
     const uint8_t* qrow = q8t + (p << 6);
     uint4 v[4];
@@ -224,8 +231,28 @@ __device__ __forceinline__ void pair_token(const PairW& q, const uint8_t* q8t, c
     const int ia = la + (ha >> 4) - 8 * static_cast<int>(static_cast<int16_t>(bsw & 0xffffu));
     const int ib = lb + (hb >> 4) - 8 * static_cast<int>(static_cast<int16_t>(bsw >> 16));
     const double d8 = static_cast<double>(d8t[p >> 1]);
-    acc = fma(d8, q.d4a * static_cast<double>(ia), acc);
-    acc = fma(d8, q.d4b * static_cast<double>(ib), acc);
+    acc = fma(d8, d4a * static_cast<double>(ia), acc);
+    acc = fma(d8, d4b * static_cast<double>(ib), acc);
+}
+
+// First row of a problem whose weights start at or after byte `off` of the problem (rows of
+// `rowbytes` bytes; 0 before the problem, n_out past its end).  32-bit division when the
+// offset allows it (the 64-bit one is a long call).
+__device__ __forceinline__ int64_t row_at(int64_t off, int rowbytes, int64_t n_out)
+{
+    if (off <= 0) return 0;
+    const int64_t r = off < (1LL << 31) ? static_cast<int64_t>((static_cast<uint32_t>(off) + (rowbytes - 1)) /
+                                                               static_cast<uint32_t>(rowbytes))
+                                        : (off + rowbytes - 1) / rowbytes;
+    return r < n_out ? r : n_out;
+}
+
+// Start of share c of the launch's B weight bytes: floor(c * B / C) =
+// c * (B / C) + floor(c * (B % C) / C), where c * (B % C) < C^2 < 2^32.
+__device__ __forceinline__ int64_t share_start(const Params& P, uint32_t c)
+{
+    return static_cast<int64_t>(c) * P.share_q +
+           static_cast<int64_t>(c * static_cast<uint32_t>(P.share_r) / static_cast<uint32_t>(P.ctas));
 }
 
 template <int TT>
@@ -234,149 +261,220 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    // this CTA's problem and its contiguous share of the problem's rows
-    int pi = 0;
-    while (pi + 1 < P.count && P.cta_begin[pi + 1] <= static_cast<int>(blockIdx.x)) ++pi;
-    const Problem& pr = P.prob[pi];
-    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * TT;
-    if (tok0 >= pr.n_tok) return;  // a token tile another problem needs
-    const int lc = static_cast<int>(blockIdx.x) - P.cta_begin[pi];
-    const int nc = P.cta_begin[pi + 1] - P.cta_begin[pi];
-    const int64_t r_begin = pr.n_out * lc / nc, r_end = pr.n_out * (lc + 1) / nc;
-    const int nt = static_cast<int>(pr.n_tok - tok0 < TT ? pr.n_tok - tok0 : TT);
-    const int k = pr.k, nb8 = k >> 7, nb4 = k >> 5, npairs = k >> 6;
-    View V;
-    V.w = pr.w;
-    V.k = k;
-    V.rowbytes = (k >> 5) * 18;
-    V.wbytes = pr.n_out * V.rowbytes;
-    V.nseg = (npairs + kUnitPairs - 1) / kUnitPairs;
-    const int act_q8_bytes = (k + 15) & ~15;
-    uint8_t* q8s = smem;                                                                  // [TT][k]
-    float* d8s = reinterpret_cast<float*>(smem + TT * act_q8_bytes);                      // [TT][k/128]
-    int16_t* bss = reinterpret_cast<int16_t*>(smem + ((TT * act_q8_bytes + TT * nb8 * 4 + 15) & ~15));
+    // CTA id = share * tiles + token tile: the token tiles of one share are neighbours in
+    // launch order, so they run side by side and the share's weights come from DRAM about
+    // once (the others read them from L2)
+    const uint32_t share = blockIdx.x / static_cast<uint32_t>(P.tiles);
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.x - share * static_cast<uint32_t>(P.tiles)) * TT;
     uint8_t* stages = smem + P.off_stage + warp * P.stages * kUnitBytes;               // this warp's
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.off_bar) + warp * P.stages;  // this warp's
-    const int D = P.stages, nseg = V.nseg;
+    const int D = P.stages;
 
     // Programmatic dependent launch: let the next kernel of the stream be scheduled as this
-    // grid's CTAs retire, and wait for the previous kernel (completion and memory flush)
-    // before the first access to global memory.  Both are no-ops without the launch
-    // attribute.
+    // grid's CTAs retire.  (A no-op without the launch attribute.)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // issue pointer: the next unit (irow, iseg) to copy
-    int64_t irow = r_begin + warp;
-    int iseg = 0;
     if (lane == 0) {
-        for (int s = 0; s < D; ++s) mbar_init(&bars[s], 1u);
+        for (int i = 0; i < D; ++i) mbar_init(&bars[i], 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int s = 0; s < D && irow < r_end; ++s) {
-        if (lane == 0) issue_unit(V, stages + s * kUnitBytes, &bars[s], irow, iseg);
-        if (++iseg == nseg) {
-            iseg = 0;
-            irow += kWarps;
-        }
-    }
 
-    // Stage the token tile's activations while the first units are in flight: one warp per
-    // 140-byte block, lane i copying code word i.
-    for (int b = warp; b < nt * nb8; b += kWarps) {
-        const int t = b / nb8, g = b - t * nb8;
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(pr.a + ((tok0 + t) * nb8 + g) * 140);
-        const uint32_t v = __ldg(src + 1 + lane);
-        *reinterpret_cast<uint32_t*>(q8s + t * act_q8_bytes + q8_swizzle(128 * g + 4 * lane)) = v;
-        if (lane < 3) {
-            const uint32_t e = __ldg(src + (lane == 0 ? 0 : 32 + lane));
-            if (lane == 0) d8s[t * nb8 + g] = __uint_as_float(e);
-            else *reinterpret_cast<uint32_t*>(bss + t * nb4 + 4 * g + 2 * (lane - 1)) = e;
-        }
-    }
-    __syncthreads();  // the only CTA-wide barrier
-
+    // the stage ring, shared by the issue and consume pointers (equal between problems)
+    int s = 0;
+    uint32_t ph = 0;
+    bool aborted = false, staged = false;
     // units start on 64-pair boundaries, so a lane's pairs p0 + lane and p0 + lane + 32 share
     // the swizzle phase (p >> 1) & 3 = (lane >> 1) & 3
     const int sw = (lane >> 1) & 3;
-    double acc[TT];
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] = 0.0;
-    // consume pointer: unit (row, seg) in stage s, phase parity ph
-    int64_t row = r_begin + warp;
-    int seg = 0, s = 0;
-    uint32_t ph = 0;
-    bool aborted = false;
-    while (row < r_end) {
-        const bool timed_out = !mbar_wait(&bars[s], ph);
-        if (__any_sync(0xffffffffu, timed_out)) {
-            aborted = true;
-            break;
-        }
-        const int p0 = seg * kUnitPairs;
-        const int np = npairs - p0 < kUnitPairs ? npairs - p0 : kUnitPairs;
-        const int64_t start = row * V.rowbytes + 36LL * p0;
-        const uint32_t* w9 = reinterpret_cast<const uint32_t*>(stages + s * kUnitBytes + (start & 15));
 
-        PairW q0, q1;
-        const bool has0 = lane < np, has1 = lane + 32 < np;
-        if (has0) load_pair(w9 + 9 * lane, q0);
-        if (has1) load_pair(w9 + 9 * (lane + 32), q1);
+    // This CTA's equal share [t0, t1) of the launch's weight bytes (the problems' weights
+    // laid end to end): it takes the rows that start inside it, of one problem or several.
+    // The first and last problems it touches and its first / end row in them are found once,
+    // here, and parked in shared memory (the 64-bit divisions are calls that would otherwise
+    // force the row loops' registers to the stack).
+    __shared__ int64_t s_rng[kWarps][4];
+    static_assert(sizeof(s_rng) == kStaticSmem, "static shared memory of the launch plan");
+    {
+        const int64_t t0 = share_start(P, share), t1 = share_start(P, share + 1);
+        int pf = 0;
+        while (pf + 1 < P.count && P.cum_bytes[pf + 1] <= t0) ++pf;
+        int pl = pf;
+        while (pl + 1 < P.count && P.cum_bytes[pl + 1] < t1) ++pl;
+        if (lane == 0) {
+            s_rng[warp][0] = pf;
+            s_rng[warp][1] = row_at(t0 - P.cum_bytes[pf], (P.prob[pf].k >> 5) * 18, P.prob[pf].n_out);
+            s_rng[warp][2] = pl;
+            s_rng[warp][3] = row_at(t1 - P.cum_bytes[pl], (P.prob[pl].k >> 5) * 18, P.prob[pl].n_out);
+        }
         __syncwarp();
-        // every lane holds its words: refill the stage with the next unit to copy
-        if (irow < r_end) {
-            if (lane == 0) issue_unit(V, stages + s * kUnitBytes, &bars[s], irow, iseg);
-            if (++iseg == nseg) {
-                iseg = 0;
-                irow += kWarps;
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < TT; ++t) {
-            if (t < nt) {
-                const uint8_t* q8t = q8s + t * act_q8_bytes;
-                const int16_t* bst = bss + t * nb4;
-                const float* d8t = d8s + t * nb8;
-                if (has0) pair_token(q0, q8t, bst, d8t, p0 + lane, sw, acc[t]);
-                if (has1) pair_token(q1, q8t, bst, d8t, p0 + lane + 32, sw, acc[t]);
-            }
-        }
-        if (++seg == nseg) {  // the row is complete
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-            }
-            if (lane == 0) {
-#pragma unroll
-                for (int t = 0; t < TT; ++t)
-                    if (t < nt) pr.y[(tok0 + t) * pr.n_out + row] = static_cast<float>(acc[t]);
-            }
-#pragma unroll
-            for (int t = 0; t < TT; ++t) acc[t] = 0.0;
-            seg = 0;
-            row += kWarps;
-        }
-        if (++s == D) {
-            s = 0;
-            ph ^= 1u;
-        }
     }
 
-    if (aborted && lane == 0) {
-        // a wait ran out: report, then wait (bounded) for this warp's copies in flight, which
-        // are the units from (row, seg) up to the issue pointer
-        iqq::raise_flags(P.flags, IQQ_FLAG_WAIT_TIMEOUT);
-        for (int j = 0; j < D && (row < irow || (row == irow && seg < iseg)); ++j) {
-            (void)mbar_wait(&bars[s], ph);
-            if (++seg == nseg) {
+    // Everything above reads only the parameters and shared memory.  Wait for the previous
+    // kernel of the stream (completion and memory flush) before the first access to global
+    // memory.  (A no-op without the launch attribute.)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    for (int pi = static_cast<int>(s_rng[warp][0]); pi <= static_cast<int>(s_rng[warp][2]); ++pi) {
+        const Problem& pr = P.prob[pi];
+        const int k = pr.k, nb8 = k >> 7, nb4 = k >> 5, npairs = k >> 6;
+        View V;
+        V.w = pr.w;
+        V.k = k;
+        V.rowbytes = nb4 * 18;
+        V.wbytes = pr.n_out * V.rowbytes;
+        V.nseg = (npairs + kUnitPairs - 1) / kUnitPairs;
+        const int64_t r_begin = pi == static_cast<int>(s_rng[warp][0]) ? s_rng[warp][1] : 0;
+        const int64_t r_end = pi == static_cast<int>(s_rng[warp][2]) ? s_rng[warp][3] : pr.n_out;
+        // rows of this CTA, counted from r_begin (a share of one wave: far below 2^31)
+        const int nrows = static_cast<int>(r_end - r_begin);
+        if (nrows <= 0 || tok0 >= pr.n_tok) continue;  // the same for the whole CTA
+        const int nt = static_cast<int>(pr.n_tok - tok0 < TT ? pr.n_tok - tok0 : TT);
+        const int act_q8_bytes = (k + 15) & ~15;
+        uint8_t* q8s = smem;                                                                  // [TT][k]
+        float* d8s = reinterpret_cast<float*>(smem + TT * act_q8_bytes);                      // [TT][k/128]
+        int16_t* bss = reinterpret_cast<int16_t*>(smem + ((TT * act_q8_bytes + TT * nb8 * 4 + 15) & ~15));
+        const int nseg = V.nseg;
+
+        // issue pointer: the next unit (irow, iseg) to copy; the first D go out now
+        int irow = warp;
+        int iseg = 0;
+        int is = s;
+        if (!aborted) {
+            for (int u = 0; u < D && irow < nrows; ++u) {
+                if (lane == 0) issue_unit(V, stages + is * kUnitBytes, &bars[is], r_begin + irow, iseg);
+                if (++iseg == nseg) {
+                    iseg = 0;
+                    irow += kWarps;
+                }
+                if (++is == D) is = 0;
+            }
+        }
+
+        // Stage the token tile's activations while the first units are in flight: one warp
+        // per 140-byte block, lane i copying code word i, several blocks of a warp in
+        // flight at once (the tile's blocks are contiguous in global memory: its tokens'
+        // rows follow one another).  The barrier before it keeps the previous problem's
+        // activations until every warp has finished with them.
+        if (staged) __syncthreads();
+        staged = true;
+        {
+            // (4 with one token: 8 would push the row loop's registers to the stack)
+            constexpr int kStageBlocks = TT == 1 ? 4 : 8;
+            const int nblk = nt * nb8;
+            const uint8_t* abase = pr.a + tok0 * nb8 * 140;
+            for (int b0 = warp; b0 < nblk; b0 += kStageBlocks * kWarps) {
+                uint32_t v[kStageBlocks], e[kStageBlocks];
+#pragma unroll
+                for (int u = 0; u < kStageBlocks; ++u) {
+                    const int b = b0 + u * kWarps;
+                    v[u] = 0u;
+                    e[u] = 0u;
+                    if (b < nblk) {
+                        const uint32_t* src = reinterpret_cast<const uint32_t*>(abase + static_cast<int64_t>(b) * 140);
+                        v[u] = __ldg(src + 1 + lane);
+                        if (lane < 3) e[u] = __ldg(src + (lane == 0 ? 0 : 32 + lane));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kStageBlocks; ++u) {
+                    const int b = b0 + u * kWarps;
+                    if (b < nblk) {
+                        const int t = b / nb8, g = b - t * nb8;
+                        *reinterpret_cast<uint32_t*>(q8s + t * act_q8_bytes + q8_swizzle(128 * g + 4 * lane)) = v[u];
+                        if (lane == 0) d8s[t * nb8 + g] = __uint_as_float(e[u]);
+                        else if (lane < 3)
+                            *reinterpret_cast<uint32_t*>(bss + t * nb4 + 4 * g + 2 * (lane - 1)) = e[u];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (aborted) continue;  // a warp that gave up still meets every barrier
+
+        double acc[TT];
+#pragma unroll
+        for (int t = 0; t < TT; ++t) acc[t] = 0.0;
+        // consume pointer: unit (row, seg) in stage s, phase parity ph
+        int row = warp;
+        int seg = 0;
+        while (row < nrows) {
+            const bool timed_out = !mbar_wait(&bars[s], ph);
+            if (__any_sync(0xffffffffu, timed_out)) {
+                aborted = true;
+                break;
+            }
+            const int p0 = seg * kUnitPairs;
+            const int np = npairs - p0 < kUnitPairs ? npairs - p0 : kUnitPairs;
+            const int64_t start = (r_begin + row) * V.rowbytes + 36LL * p0;
+            const uint32_t* w9 = reinterpret_cast<const uint32_t*>(stages + s * kUnitBytes + (start & 15));
+
+            PairW q0, q1;
+            const bool has0 = lane < np, has1 = lane + 32 < np;
+            if (has0) load_pair(w9 + 9 * lane, q0);
+            if (has1) load_pair(w9 + 9 * (lane + 32), q1);
+            __syncwarp();
+            // every lane holds its words: refill the stage with the next unit to copy
+            if (irow < nrows) {
+                if (lane == 0) issue_unit(V, stages + s * kUnitBytes, &bars[s], r_begin + irow, iseg);
+                if (++iseg == nseg) {
+                    iseg = 0;
+                    irow += kWarps;
+                }
+            }
+            if (TT == 1) {
+                // one token: each scale is used once, converted where it is used (fewer
+                // registers live across the unit)
+                if (has0) pair_token(q0, scale_a(q0), scale_b(q0), q8s, bss, d8s, p0 + lane, sw, acc[0]);
+                if (has1) pair_token(q1, scale_a(q1), scale_b(q1), q8s, bss, d8s, p0 + lane + 32, sw, acc[0]);
+            } else {
+                const double a0 = scale_a(q0), b0s = scale_b(q0), a1 = scale_a(q1), b1s = scale_b(q1);
+#pragma unroll
+                for (int t = 0; t < TT; ++t) {
+                    if (t < nt) {
+                        const uint8_t* q8t = q8s + t * act_q8_bytes;
+                        const int16_t* bst = bss + t * nb4;
+                        const float* d8t = d8s + t * nb8;
+                        if (has0) pair_token(q0, a0, b0s, q8t, bst, d8t, p0 + lane, sw, acc[t]);
+                        if (has1) pair_token(q1, a1, b1s, q8t, bst, d8t, p0 + lane + 32, sw, acc[t]);
+                    }
+                }
+            }
+            if (++seg == nseg) {  // the row is complete
+#pragma unroll
+                for (int t = 0; t < TT; ++t) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int t = 0; t < TT; ++t)
+                        if (t < nt) pr.y[(tok0 + t) * pr.n_out + r_begin + row] = static_cast<float>(acc[t]);
+                }
+#pragma unroll
+                for (int t = 0; t < TT; ++t) acc[t] = 0.0;
                 seg = 0;
                 row += kWarps;
             }
             if (++s == D) {
                 s = 0;
                 ph ^= 1u;
+            }
+        }
+
+        if (aborted && lane == 0) {
+            // a wait ran out: report, then wait (bounded) for this warp's copies in flight,
+            // which are the units from (row, seg) up to the issue pointer
+            iqq::raise_flags(P.flags, IQQ_FLAG_WAIT_TIMEOUT);
+            for (int j = 0; j < D && (row < irow || (row == irow && seg < iseg)); ++j) {
+                (void)mbar_wait(&bars[s], ph);
+                if (++seg == nseg) {
+                    seg = 0;
+                    row += kWarps;
+                }
+                if (++s == D) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
         }
     }
@@ -431,7 +529,7 @@ int smem_bytes(const Params& P) { return P.off_bar + kWarps * P.stages * 8; }
 // (allocated per warp in units of 256).
 int ctas_per_sm(int smem, int regs)
 {
-    int occ = kSmemPerSm / (smem + 1024);
+    int occ = kSmemPerSm / (smem + kStaticSmem + 1024);
     const int regs_cta = ((regs * 32 + 255) / 256) * 256 * kWarps;
     if (65536 / regs_cta < occ) occ = 65536 / regs_cta;
     return occ;
@@ -479,8 +577,9 @@ bool plan_tt(Params& P, int kmax, int dev, int& ctas)
     return true;
 }
 
-// Launches P.count (<= kMaxBatch) problems: CTAs apportioned to the problems by their
-// weight bytes (at least one each, at most one per 16 rows), the token tiles on grid y.
+// Launches P.count (<= kMaxBatch) problems: c0 byte shares, one wave of CTAs (fewer when the
+// problems have fewer than 16 rows per CTA) splitting the problems' weight bytes evenly, each
+// share times the token tiles, on a one-dimensional grid.
 template <int TT>
 iqq_status launch_tt(Params& P, int kmax, int64_t max_tok, cudaStream_t st, bool& fits)
 {
@@ -496,24 +595,24 @@ iqq_status launch_tt(Params& P, int kmax, int64_t max_tok, cudaStream_t st, bool
             return iqq::launch_status();
         opted.store(kSmemMax, std::memory_order_relaxed);
     }
-    const int64_t target = static_cast<int64_t>(sm_count_gemv(dev)) * ctas;
-    double total = 0.0;
-    for (int i = 0; i < P.count; ++i) total += static_cast<double>(P.prob[i].n_out) * (P.prob[i].k / 32) * 18;
-    int c0 = 0;
+    int64_t rows = 0;
+    P.cum_bytes[0] = 0;
     for (int i = 0; i < P.count; ++i) {
-        const double bytes = static_cast<double>(P.prob[i].n_out) * (P.prob[i].k / 32) * 18;
-        int64_t n = static_cast<int64_t>(static_cast<double>(target) * bytes / total + 0.5);
-        const int64_t most = (P.prob[i].n_out + kWarps - 1) / kWarps;
-        if (n > most) n = most;
-        if (n < 1) n = 1;
-        P.cta_begin[i] = c0;
-        c0 += static_cast<int>(n);
+        P.cum_bytes[i + 1] = P.cum_bytes[i] + P.prob[i].n_out * ((P.prob[i].k / 32) * 18);
+        rows += P.prob[i].n_out;
     }
-    P.cta_begin[P.count] = c0;
+    int64_t c0 = static_cast<int64_t>(sm_count_gemv(dev)) * ctas;
+    if (c0 > (rows + kWarps - 1) / kWarps) c0 = (rows + kWarps - 1) / kWarps;
+    if (c0 < 1) c0 = 1;
+    if (c0 > 65535) c0 = 65535;  // keeps c * (B % C) below 2^32
+    P.share_q = P.cum_bytes[P.count] / c0;
+    P.share_r = P.cum_bytes[P.count] % c0;
     const int64_t gy = (max_tok + TT - 1) / TT;
-    if (gy > 65535) return IQQ_ERR_SHAPE;
+    if (gy > 65535 || c0 * gy > 0x7fffffffLL) return IQQ_ERR_SHAPE;
+    P.ctas = static_cast<int>(c0);
+    P.tiles = static_cast<int>(gy);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(c0), static_cast<unsigned>(gy));
+    cfg.gridDim = dim3(static_cast<unsigned>(c0 * gy));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = st;
