@@ -276,8 +276,10 @@ iqq_status iqq_dequant_rmse_qx(int bits, const float* x, const void* blocks, con
  *  k         values per row: a multiple of 128, at most IQQ_GEMV_MAX_K.  k == 0 writes
  *            zeros (the empty dot product).
  *  d_flags   optional; receives IQQ_FLAG_WAIT_TIMEOUT.
- * Blocks whose binary16 scale is not finite give unspecified values in the rows that use
- * them (iqq_quantize_q4_0_w flags such scales).
+ * Tokens are processed in tiles of up to 8 (fewer when a wide row's activations would not
+ * fit in shared memory); a token count needing more than 65535 tiles returns
+ * IQQ_ERR_SHAPE.  Blocks whose binary16 scale is not finite give unspecified values in the
+ * rows that use them (iqq_quantize_q4_0_w flags such scales).
  */
 #define IQQ_GEMV_MAX_K 65536
 iqq_status iqq_gemv_q4_0_q8_k128(const void* w_blocks, const void* a_blocks, float* y, int64_t n_out,
@@ -286,9 +288,10 @@ iqq_status iqq_gemv_q4_0_q8_k128(const void* w_blocks, const void* a_blocks, flo
 /*
  * iqq_gemv_q4_0_q8_k128_batch -- iqq_gemv_q4_0_q8_k128 for a list of independent problems
  * (for example every weight matrix of a model for one decode step) in as few launches as
- * possible: up to 64 problems per launch, the launch's CTAs apportioned to its problems by
- * their weight bytes.  Each problem's result is exactly that of iqq_gemv_q4_0_q8_k128
- * (the per-row summation order does not depend on the launch).
+ * possible: up to 64 problems per launch, one wave of CTAs each taking an equal share of
+ * the launch's weight bytes (rows of one problem or of several).  Each problem's result is
+ * exactly that of iqq_gemv_q4_0_q8_k128 (the per-row summation order does not depend on
+ * the launch).
  *  problems  HOST array of count descriptors, read during the call and not kept; every
  *            field as for iqq_gemv_q4_0_q8_k128.  The outputs y must not overlap any
  *            problem's inputs or other outputs.
