@@ -152,3 +152,28 @@ def test_gemv_batch_matches_single_calls(iqq, synth):
             continue
         yo, s = oracle.dot_q4_0_q8_k128(w.cpu().numpy(), a.cpu().numpy(), n_out, k, n_tok)
         _check(y.cpu().numpy(), yo, s, k)
+
+
+def test_gemv_batch_ctas_spanning_problems(iqq, synth):
+    """64 small problems (1-5 rows, k up to 768, 1-9 tokens): the launch has a dozen CTAs,
+    each taking rows of several problems in turn, and the second token tile skips the
+    problems with at most 8 tokens inside a CTA.  Every output equals its single call bit
+    for bit and lies within the bound of the oracle's value."""
+    rng = np.random.default_rng(41)
+    items, singles, refs = [], [], []
+    for i in range(64):
+        n_out, k, n_tok = 1 + (i * 7) % 5, 128 * (1 + (i * 3) % 6), 1 + (i * 5) % 9
+        w = torch.from_numpy(_random_q4_0(rng, n_out, k)).cuda()
+        a = torch.from_numpy(_activations(synth, n_tok, k, seed=100 + i)).cuda()
+        y = torch.full((n_tok, n_out), float("nan"), device="cuda")
+        items.append((w, a, y, k))
+        singles.append(iqq.gemv_q4_0_q8_k128(w, a, n_out, k, n_tok))
+        refs.append((n_out, k, n_tok))
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    iqq.iqq_gemv_q4_0_q8_k128_batch(iqq.gemv_problems(items), flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    for (w, a, y, k), single, (n_out, _, n_tok) in zip(items, singles, refs):
+        assert torch.equal(y, single)
+        yo, s = oracle.dot_q4_0_q8_k128(w.cpu().numpy(), a.cpu().numpy(), n_out, k, n_tok)
+        _check(y.cpu().numpy(), yo, s, k)
