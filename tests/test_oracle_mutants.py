@@ -44,6 +44,12 @@ MUTANTS = {
                                      "const double av = (double)(int8_t)ab[4 + j % ORACLE_QK8];"),
     "fudge_dropped": ("float sigma2 = fudge * oracle_row_sigma2(xr, n_per_row);",
                       "float sigma2 = oracle_row_sigma2(xr, n_per_row);"),
+    "rmse_qw_row_index": ("const float *qr = qw ? qw + (rows_per_qw > 0 ? r / rows_per_qw : 0) * n_per_row : NULL;\n        for (int64_t b = 0; b < nb; ++b) {\n            const uint8_t *blk",
+                           "const float *qr = qw ? qw + (rows_per_qw > 0 ? r / (rows_per_qw + 1) : 0) * n_per_row : NULL;\n        for (int64_t b = 0; b < nb; ++b) {\n            const uint8_t *blk"),
+    "qx_qw_row_index": ("int8_t L[32];\n    for (int64_t r = 0; r < nrows; ++r) {\n        const float *xr = x + r * n_per_row;\n        const float *qr = qw ? qw + (rows_per_qw > 0 ? r / rows_per_qw : 0)",
+                         "int8_t L[32];\n    for (int64_t r = 0; r < nrows; ++r) {\n        const float *xr = x + r * n_per_row;\n        const float *qr = qw ? qw + (rows_per_qw > 0 ? r / (rows_per_qw + 1) : 0)"),
+    "mode5_sigma2_for_sigma": ("case 5: m = sigma + fabsf(x); break;", "case 5: m = sigma2 + fabsf(x); break;"),
+    "mode4_sqrt": ("case 4: m = sigma2 + t; break;", "case 4: m = sqrtf(sigma2 + t); break;"),
     "fp16_ties_down": ("if (rem > half || (rem == half && (q & 1u))) q += 1u;",
                        "if (rem > half) q += 1u;"),
 }

@@ -203,6 +203,22 @@ def test_weighted_rmse_stacked_imatrix(orc):
             assert abs(acc[0] - float(np.sum(qfull * e * e))) <= 1e-12 * acc[0]
 
 
+@pytest.mark.parametrize("bits", (4, 5, 6, 8))
+def test_stacked_imatrix_selects_row(orc, bits):
+    """One imatrix row per rows_per_qw rows (the experts' stacked imatrix): the stacked call
+    equals quantizing each group of rows with its own imatrix row, for every format, and
+    the rows do matter (one row for all gives other blocks)."""
+    rng = np.random.default_rng(70 + bits)
+    x = (rng.standard_normal((12, 128)) * 0.02).astype(np.float32)
+    qw = np.exp(2.0 * rng.standard_normal((4, 128))).astype(np.float32)
+    stacked, _ = orc.quantize_qx_0_w(bits, x, qw, rows_per_qw=3)
+    for g in range(4):
+        part, _ = orc.quantize_qx_0_w(bits, x[3 * g:3 * g + 3], qw[g])
+        assert np.array_equal(stacked[3 * g:3 * g + 3], part), g
+    one, _ = orc.quantize_qx_0_w(bits, x, qw[0])
+    assert not np.array_equal(one[3:], stacked[3:])
+
+
 @pytest.mark.parametrize("bits", (4, 5, 8))
 def test_fudge_factor_special_cases(orc, bits):
     """[W] §四's fudge factor, read as scaling the sigma2 term of the importance: fudge = 1
