@@ -50,6 +50,12 @@ MUTANTS = {
                          "int8_t L[32];\n    for (int64_t r = 0; r < nrows; ++r) {\n        const float *xr = x + r * n_per_row;\n        const float *qr = qw ? qw + (rows_per_qw > 0 ? r / (rows_per_qw + 1) : 0)"),
     "mode5_sigma2_for_sigma": ("case 5: m = sigma + fabsf(x); break;", "case 5: m = sigma2 + fabsf(x); break;"),
     "mode4_sqrt": ("case 4: m = sigma2 + t; break;", "case 4: m = sqrtf(sigma2 + t); break;"),
+    "greedy_four_passes": ("for (int pass = 0; pass < 5; ++pass) {", "for (int pass = 0; pass < 4; ++pass) {"),
+    "greedy_six_passes": ("for (int pass = 0; pass < 5; ++pass) {", "for (int pass = 0; pass < 6; ++pass) {"),
+    "q8_bsum_stride": ("for (int j = 0; j < 32; ++j) s += q[32 * i + j];",
+                       "for (int j = 0; j < 32; ++j) s += q[4 * j + i];"),
+    "q8_0_offset_codes": ("for (int j = 0; j < 32; ++j) blk[2 + j] = (uint8_t)L[j];",
+                          "for (int j = 0; j < 32; ++j) blk[2 + j] = (uint8_t)(L[j] + 128);"),
     "fp16_ties_down": ("if (rem > half || (rem == half && (q & 1u))) q += 1u;",
                        "if (rem > half) q += 1u;"),
 }

@@ -243,6 +243,20 @@ def test_sweep_picks_lowest_error_candidate_lowest_k_on_ties(orc):
         assert first == k + 9
 
 
+def test_greedy_pass_limit_is_reached_and_kept(orc):
+    """The greedy refinement runs at most 5 passes (a pass with no accepted move ends it
+    and is counted).  On a seeded 256x4096 tensor the counts fall off geometrically and
+    the bound is reached by a few blocks, never exceeded."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((256, 4096)) * 0.02).astype(np.float32)
+    qw = np.exp(rng.standard_normal(4096)).astype(np.float32)
+    _, _, passes = orc.quantize_q4_0_w(x, qw, want_passes=True)
+    counts = np.bincount(passes.ravel(), minlength=7)
+    assert counts[0] == 0 and counts[6:].sum() == 0, counts
+    assert counts[5] >= 3, counts
+    assert all(counts[p] > counts[p + 1] for p in range(1, 5)), counts
+
+
 def test_greedy_never_worse_and_locally_optimal(orc):
     """The greedy stage never ends above the sweep's error, and when it stops early no
     single +-1 code move lowers the fp64 error by more than the binary32 resolution of
