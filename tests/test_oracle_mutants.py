@@ -52,6 +52,10 @@ MUTANTS = {
     "mode4_sqrt": ("case 4: m = sigma2 + t; break;", "case 4: m = sqrtf(sigma2 + t); break;"),
     "greedy_four_passes": ("for (int pass = 0; pass < 5; ++pass) {", "for (int pass = 0; pass < 4; ++pass) {"),
     "greedy_six_passes": ("for (int pass = 0; pass < 5; ++pass) {", "for (int pass = 0; pass < 6; ++pass) {"),
+    "sweep_drops_last_candidate": ("for (int k = -9; k <= 9; ++k) {", "for (int k = -9; k <= 8; ++k) {"),
+    "fallback_scale_sign": ("return 1.0f / iscale0;", "return -1.0f / iscale0;"),
+    "sigma2_sample_mean": ("return (float)(s / (double)n);", "return (float)(s / (double)(n - 1));"),
+    "mode3_signed": ("case 3: m = fabsf(x); break;", "case 3: m = x; break;"),
     "q8_bsum_stride": ("for (int j = 0; j < 32; ++j) s += q[32 * i + j];",
                        "for (int j = 0; j < 32; ++j) s += q[4 * j + i];"),
     "q8_0_offset_codes": ("for (int j = 0; j < 32; ++j) blk[2 + j] = (uint8_t)L[j];",
