@@ -563,11 +563,10 @@ def main_ours(args):
                                           barrier=dist.barrier if world > 1 else None)
         if world > 1:
             e2e_sec = replicas.max_over_ranks([e2e_sec], device=dev)[0]
-            e2e.update(value=e2e_elems * world / e2e_sec / 1e9,
-                       h2d_bytes_per_step=e2e["h2d_bytes_per_step"] * world,
-                       d2h_bytes_per_step=e2e["d2h_bytes_per_step"] * world,
-                       h2d_gb_s=round(e2e["h2d_bytes_per_step"] * world / e2e_sec / 1e9, 1),
-                       layers_per_rank=e2e_layers, ranks=world)
+            elems, h2d, d2h = replicas.sum_over_ranks(
+                [e2e_elems, e2e["h2d_bytes_per_step"], e2e["d2h_bytes_per_step"]], device=dev)
+            e2e.update(value=elems / e2e_sec / 1e9, h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
+                       h2d_gb_s=round(h2d / e2e_sec / 1e9, 1), layers_per_rank=e2e_layers, ranks=world)
 
     if world > 1:
         dist.destroy_process_group()

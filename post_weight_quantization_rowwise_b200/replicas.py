@@ -8,6 +8,8 @@ does cross ranks is bookkeeping:
   the tensors of a model) over the ranks;
 * ``rank_seed_offset``: distinct synthetic inputs per rank for weak scaling;
 * ``max_over_ranks``: the job time of a timed region (the slowest rank);
+* ``sum_over_ranks``: the job's totals (values processed, bytes copied), so that
+  a rate is all ranks' work over the slowest rank's time;
 * ``reduce_rmse``: the weighted-RMSE accumulators of all ranks combined
   (sums added, ``max|e|`` maxed), so that one tensor set split over ranks gives
   the same statistics as on one rank (up to binary64 rounding order).
@@ -51,6 +53,17 @@ def max_over_ranks(values, device=None) -> list[float]:
     d = _dist()
     if d is not None:
         d.all_reduce(t, op=d.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def sum_over_ranks(values, device=None) -> list[float]:
+    """Element-wise sum of a list of floats over all ranks (binary64: counts below 2^53
+    stay exact)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    d = _dist()
+    if d is not None:
+        d.all_reduce(t, op=d.ReduceOp.SUM)
     return [float(v) for v in t.cpu()]
 
 

@@ -1,8 +1,9 @@
 """The multi-process host logic on CPU: world size 2 over gloo.
 
 The quantizer shards into independent problems, so the only cross-rank steps are
-bookkeeping: the max-over-ranks time of the timed region and the combination of
-the weighted-RMSE accumulators.  The accumulator test splits one set of tensors
+bookkeeping: the max-over-ranks time of the timed region, the job's totals (values
+and bytes, for the end-to-end rate) and the combination of the weighted-RMSE
+accumulators.  The accumulator test splits one set of tensors
 over two ranks (each rank runs the CPU oracle on its share) and checks that the
 combined statistics equal the single-process ones.
 """
@@ -31,6 +32,8 @@ def _worker(rank, world, port, out):
         import oracle
         # job time: the slowest rank
         mx = replicas.max_over_ranks([1.0 + rank, 5.0 - rank])
+        # job totals: values and bytes of all ranks (exact for counts below 2^53)
+        tot = replicas.sum_over_ranks([1.0 + rank, 2.0 ** 40 + rank])
         # the tensor set split over ranks; each rank quantizes and scores its share
         tensors = [synth.Tensor2D(f"t{i}", 24 + 8 * i, 64, 100 + i) for i in range(5)]
         acc = torch.zeros(4, dtype=torch.float64)
@@ -42,7 +45,7 @@ def _worker(rank, world, port, out):
             acc[:3] += torch.from_numpy(part[:3])
             acc[3] = max(float(acc[3]), float(part[3]))
         total = replicas.reduce_rmse(acc)
-        out[rank] = (mx, total.tolist())
+        out[rank] = (mx, total.tolist(), tot)
     finally:
         dist.destroy_process_group()
 
@@ -77,8 +80,9 @@ def test_two_gloo_ranks_combine_like_one_process():
         blocks, _ = oracle.quantize_q4_0_w(x, qw)
         oracle.weighted_rmse(x, blocks, qw, acc=ref)
     for rank in range(world):
-        mx, total = out[rank]
+        mx, total, tot = out[rank]
         assert mx == [2.0, 5.0]
+        assert tot == [3.0, 2.0 ** 41 + 1]
         assert np.allclose(total[:3], ref[:3], rtol=1e-12, atol=0)
         assert total[3] == ref[3]
     assert abs(replicas.wrmse(out[0][1]) - np.sqrt(ref[0] / ref[1])) < 1e-12
