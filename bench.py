@@ -34,18 +34,15 @@ METRIC = "Gelem/s quantized (imatrix Q4_0, Q8_K_128) on 1 B200; % of HBM/FP32 ro
 UNIT = "Gelem/s"
 WORKLOAD = "llama2-7b layer set x32 (q4_0 imatrix + dequant + wrmse) + q8_k128 4096x7168"
 
-# Algorithmic work per value ("Roofline"):
-#   Q4_0 weighted: 145 + 8*p binary32 lane operations per value, p = mean greedy passes;
-#   Q8_K_128: 4 + 140/128 bytes per value; dequant: 18/32 + 4; wrmse: 4 + 18/32 (+ qw from L2).
+# Algorithmic work per value:
+#   Q4_0 weighted: 145 + 8*p binary32 lane operations per value, p = mean greedy passes:
+#   1 for sigma2, 5 for the weight and w*x, 19 x 7 for the candidate sweep, about 2 for the
+#   per-block constants, 4 for the final sums and packing, 8 per greedy pass;
+#   Q8_K_128: 4 + 140/128 bytes per value; dequant + round trip: 4 + 18/32 + 4 (y written).
 Q4_0_OPS_BASE = 145.0
 Q4_0_OPS_PER_PASS = 8.0
-# the round trip accumulated by the same kernel: y = d*l, e = x - y, e^2, qw*e^2 + sum,
-# sum qw, sum e^2, max |e|
-Q4_0_RMSE_OPS = 7.0
 Q8_BYTES_PER_VALUE = 4.0 + 140.0 / 128.0
-DEQ_BYTES_PER_VALUE = 18.0 / 32.0 + 4.0
 DEQ_RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0 + 4.0  # read x and the blocks, write y
-RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
