@@ -403,6 +403,9 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     """The same step through the public API from pinned host buffers, every byte of input
     crossing PCIe each step: per tensor H2D of x and qw, its two kernels, D2H of the
     blocks; H2D of the activations, Q8_K_128, D2H of its blocks and of the accumulator.
+    The layer set's weights are bf16 values (a bf16 checkpoint's), so x travels as bf16 and
+    goes through the bf16 entry points, which widen it exactly in the kernels: the blocks,
+    y and sums are those of the binary32 step.
     The copies run on their own streams (host to device, device to host) with two device
     staging slots, so tensor i + 1 uploads and tensor i - 1 downloads while tensor i
     computes; events order every reuse of a slot or buffer.  ``barrier`` (several ranks)
@@ -411,19 +414,19 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     import torch
     n = 7 * layers
 
-    def pinned_copy(t):
-        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    def pinned_copy(t, dtype=None):
+        h = torch.empty(t.shape, dtype=dtype or t.dtype, pin_memory=True)
         h.copy_(t)
         return h
 
-    host_x = [pinned_copy(w.x[i]) for i in range(n)]
+    host_x = [pinned_copy(w.x[i], torch.bfloat16) for i in range(n)]  # exact: bf16 values
     host_qw = [pinned_copy(w.qw[i]) for i in range(n)]
     host_b = [torch.empty(w.blocks[i].numel(), dtype=torch.uint8, pin_memory=True) for i in range(n)]
     host_act = pinned_copy(w.act)
     host_q8 = torch.empty(w.q8.numel(), dtype=torch.uint8, pin_memory=True)
     host_acc = torch.empty(4, dtype=torch.float64, pin_memory=True)
     big = max(t.numel for t in w.tensors[:n])
-    xd = [torch.empty(big, dtype=torch.float32, device=dev) for _ in range(2)]
+    xd = [torch.empty(big, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     qd = [torch.empty(max(t.cols for t in w.tensors[:n]), dtype=torch.float32, device=dev) for _ in range(2)]
     cs = torch.cuda.current_stream()
     up, dn = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -431,7 +434,7 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     computed = [torch.cuda.Event() for _ in range(2)]
     act_up, q8_done, acc_read = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
     downloaded = [torch.cuda.Event() for _ in range(n)]
-    h2d = sum(h.numel() * 4 for h in host_x) + sum(h.numel() * 4 for h in host_qw) + host_act.numel() * 4
+    h2d = sum(h.numel() * 2 for h in host_x) + sum(h.numel() * 4 for h in host_qw) + host_act.numel() * 4
     d2h = sum(h.numel() for h in host_b) + host_q8.numel() + 32
 
     def one():
@@ -447,8 +450,9 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
                 uploaded[k].record(up)
             cs.wait_event(uploaded[k])
             cs.wait_event(downloaded[i])  # the previous step's copy of these blocks is done
-            iqq.iqq_quantize_q4_0_w(xv, qv, w.blocks[i], stream=cs)
-            iqq.iqq_dequant_rmse_qx(4, xv, w.blocks[i], qv, w.y[:t.numel].view(t.rows, t.cols), w.acc, stream=cs)
+            iqq.iqq_quantize_qx_0_w_bf16(4, xv, qv, w.blocks[i], stream=cs)
+            iqq.iqq_dequant_rmse_qx_bf16(4, xv, w.blocks[i], qv, w.y[:t.numel].view(t.rows, t.cols), w.acc,
+                                         stream=cs)
             computed[k].record(cs)
             with torch.cuda.stream(dn):
                 dn.wait_event(computed[k])
@@ -488,7 +492,8 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     elems = sum(t.numel for t in w.tensors[:n]) + w.act.numel()
     return ({"value": elems / sec / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
              "d2h_bytes_per_step": int(d2h), "layers": layers,
-             "h2d_gb_s": round(h2d / sec / 1e9, 1), "overlap": "copies on two streams beside the kernels"},
+             "h2d_gb_s": round(h2d / sec / 1e9, 1), "x_dtype": "bf16 (exact: bf16-valued weights)",
+            "overlap": "copies on two streams beside the kernels"},
             sec, elems)
 
 

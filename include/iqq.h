@@ -168,6 +168,20 @@ iqq_status iqq_quantize_qx_0_w_ex(int bits, const float* x, const float* qw, voi
                                   uint32_t* d_flags, void* stream);
 
 /*
+ * iqq_quantize_qx_0_w_bf16 -- iqq_quantize_qx_0_w for weights stored as bf16 (the form a
+ * checkpoint usually holds).  The quantization routine of [W] §一 takes binary32 values;
+ * each bf16 is widened to binary32 exactly in the kernel (its bits are the binary32's high
+ * half), so the blocks and flags are bit for bit those of iqq_quantize_qx_0_w (and _ws) on
+ * the widened tensor, from half the bytes of x.
+ *  x          [nrows, n_per_row] bf16, 16-byte aligned.
+ *  workspace, workspace_bytes  optional, as for iqq_quantize_qx_0_w_ex.
+ * Other arguments and errors as for iqq_quantize_qx_0_w.
+ */
+iqq_status iqq_quantize_qx_0_w_bf16(int bits, const void* x, const float* qw, void* out, int64_t nrows,
+                                    int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
+                                    size_t workspace_bytes, uint32_t* d_flags, void* stream);
+
+/*
  * iqq_quantize_qx_0_w_static -- iqq_quantize_qx_0_w_ws without a caller workspace: the
  * per-row sigma2 of wide rows goes to a library-owned device array of IQQ_STATIC_WS_ROWS
  * floats (a file-scope __device__ variable, one per device; nothing is allocated), and
@@ -256,6 +270,16 @@ iqq_status iqq_weighted_rmse_qx(int bits, const float* x, const void* blocks, co
  */
 iqq_status iqq_dequant_rmse_qx(int bits, const float* x, const void* blocks, const float* qw, int64_t nrows,
                                int64_t n_per_row, int64_t rows_per_qw, float* y, double* d_acc, void* stream);
+
+/*
+ * iqq_dequant_rmse_qx_bf16 -- iqq_dequant_rmse_qx against x stored as bf16 [nrows,
+ * n_per_row] (16-byte aligned), widened exactly to binary32: y and the accumulator are bit
+ * for bit those of iqq_dequant_rmse_qx on the widened tensor.  Other arguments and errors
+ * as for iqq_dequant_rmse_qx.
+ */
+iqq_status iqq_dequant_rmse_qx_bf16(int bits, const void* x, const void* blocks, const float* qw, int64_t nrows,
+                                    int64_t n_per_row, int64_t rows_per_qw, float* y, double* d_acc,
+                                    void* stream);
 
 /*
  * iqq_gemv_q4_0_q8_k128 -- y[t][r] = dot(dequant(W row r), dequant(A row t)): Q4_0 weight

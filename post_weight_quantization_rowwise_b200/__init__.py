@@ -58,6 +58,9 @@ def _load():
         "iqq_quantize_qx_0_w_ex": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
                                    _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp],
         "iqq_weighted_rmse": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+        "iqq_quantize_qx_0_w_bf16": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
+                                     ctypes.c_size_t, _vp, _vp],
+        "iqq_dequant_rmse_qx_bf16": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -226,6 +229,28 @@ def iqq_quantize_qx_0_w_ws(bits, x, qw, out, workspace, rows_per_qw: int = 0, we
     return out
 
 
+def iqq_quantize_qx_0_w_bf16(bits, x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, workspace=None,
+                             flags=None, stream=None):
+    """iqq_quantize_qx_0_w for bf16 x [nrows, n_per_row] (widened exactly in the kernel: the
+    blocks equal those of the binary32 tensor); optional workspace as for _ws."""
+    import torch
+    _need_cuda("x", x, torch.bfloat16)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("workspace", workspace, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
+        raise ValueError("out is too small")
+    nbytes = 0 if workspace is None else workspace.numel()
+    _check("iqq_quantize_qx_0_w_bf16",
+           _lib.iqq_quantize_qx_0_w_bf16(bits, _ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw, weight_mode,
+                                         _ptr(workspace), nbytes, _ptr(flags), _stream(stream)))
+    return out
+
+
 def iqq_quantize_q8_k128(x, out, flags=None, stream=None):
     """Q8_K_128 blocks of x [nrows, n_per_row] float32 into out (uint8, q8_k128_nbytes)."""
     import torch
@@ -351,6 +376,26 @@ def iqq_dequant_rmse_qx(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, strea
     _check("iqq_dequant_rmse_qx",
            _lib.iqq_dequant_rmse_qx(bits, _ptr(x), _ptr(blocks), _ptr(qw), nrows, n, rows_per_qw, _ptr(y),
                                     _ptr(acc), _stream(stream)))
+    return y
+
+
+def iqq_dequant_rmse_qx_bf16(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, stream=None):
+    """iqq_dequant_rmse_qx against bf16 x (widened exactly: y and acc equal those of the
+    binary32 tensor)."""
+    import torch
+    _need_cuda("x", x, torch.bfloat16)
+    _need_cuda("blocks", blocks, torch.uint8)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("y", y, torch.float32)
+    _need_cuda("acc", acc, torch.float64)
+    nrows, n = _shape2(x)
+    if bits not in QX_0_BLOCK_BYTES:
+        raise ValueError("bits must be 4, 5, 6 or 8")
+    if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits] or acc.numel() < 4 or y.numel() < x.numel():
+        raise ValueError("blocks, y or acc is too small")
+    _check("iqq_dequant_rmse_qx_bf16",
+           _lib.iqq_dequant_rmse_qx_bf16(bits, _ptr(x), _ptr(blocks), _ptr(qw), nrows, n, rows_per_qw, _ptr(y),
+                                         _ptr(acc), _stream(stream)))
     return y
 
 

@@ -1,6 +1,7 @@
 // common.cuh -- helpers shared by the library's CUDA translation units.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -40,6 +41,31 @@ __device__ __forceinline__ float4 ld_stream_f4(const float4* p)
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                  : "l"(p));
     return v;
+}
+
+// Four bf16 values (little endian in two words) widened to binary32: a bf16 is the high
+// half of the binary32 with the same value, so the widening is exact.
+__device__ __forceinline__ float4 widen_bf16x4(uint2 v)
+{
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                       __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+}
+
+// Values p[0..3] as binary32, from binary32 storage (p 16-byte aligned) or bf16 storage
+// (p 8-byte aligned); read-only path.
+__device__ __forceinline__ float4 ld4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16* p)
+{
+    return widen_bf16x4(__ldg(reinterpret_cast<const uint2*>(p)));
+}
+
+// The same, streaming (no L1 allocation: data read once).
+__device__ __forceinline__ float4 ld4_stream(const float* p) { return ld_stream_f4(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 ld4_stream(const __nv_bfloat16* p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return widen_bf16x4(v);
 }
 
 // Flags word update: only lanes with a nonzero bit set touch memory.

@@ -197,9 +197,9 @@ __device__ __forceinline__ void rmse_quad(const float4 xv, const QuadC q, double
 // Rows [blockIdx.y*rows_per_cta, ...) x column quad blockIdx.x*kThreads + threadIdx.x.
 // Per column the thread keeps sum_r e^2 (binary64) and multiplies by qw once per
 // imatrix row, so qw is read and converted once per row segment, not per value.
-template <int BITS>
+template <int BITS, typename XT>
 __global__ void __launch_bounds__(kThreads)
-weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ blocks,
+weighted_rmse_kernel(const XT* __restrict__ x, const uint8_t* __restrict__ blocks,
                      const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
                      int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc, float* __restrict__ y)
 {
@@ -225,7 +225,7 @@ weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ bl
                 QuadC q[kRowUnroll];
 #pragma unroll
                 for (int u = 0; u < kRowUnroll; ++u) {
-                    xv[u] = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + (r + u) * n_per_row) + cq);
+                    xv[u] = iqq::ld4_stream(x + (r + u) * n_per_row + 4 * cq);
                     q[u] = load_codes<BITS>(blocks + ((r + u) * nb + b) * block_bytes<BITS>(), qd);
                 }
 #pragma unroll
@@ -234,7 +234,7 @@ weighted_rmse_kernel(const float* __restrict__ x, const uint8_t* __restrict__ bl
                               y != nullptr ? reinterpret_cast<float4*>(y + (r + u) * n_per_row) + cq : nullptr);
             }
             for (; r < s1; ++r) {
-                const float4 xv = iqq::ld_stream_f4(reinterpret_cast<const float4*>(x + r * n_per_row) + cq);
+                const float4 xv = iqq::ld4_stream(x + r * n_per_row + 4 * cq);
                 rmse_quad(xv, load_codes<BITS>(blocks + (r * nb + b) * block_bytes<BITS>(), qd), col, emax,
                           y != nullptr ? reinterpret_cast<float4*>(y + r * n_per_row) + cq : nullptr);
             }
@@ -329,8 +329,8 @@ extern "C" iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, i
 
 namespace {
 
-template <int BITS>
-iqq_status rmse_launch(const float* x, const void* blocks, const float* qw, int64_t nrows, int64_t n_per_row,
+template <int BITS, typename XT = float>
+iqq_status rmse_launch(const XT* x, const void* blocks, const float* qw, int64_t nrows, int64_t n_per_row,
                        int64_t rows_per_qw, double* d_acc, void* stream, float* y = nullptr)
 {
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
@@ -351,7 +351,7 @@ iqq_status rmse_launch(const float* x, const void* blocks, const float* qw, int6
     gy = (nrows + rpc - 1) / rpc;
     if (gx > 0x7fffffff || gy > 65535) return IQQ_ERR_SHAPE;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-    weighted_rmse_kernel<BITS><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+    weighted_rmse_kernel<BITS, XT><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         x, static_cast<const uint8_t*>(blocks), qw, nrows, n_per_row, rows_per_qw,
         static_cast<int>(rpc), d_acc, y);
     return iqq::launch_status();
@@ -389,6 +389,21 @@ extern "C" iqq_status iqq_weighted_rmse_qx(int bits, const float* x, const void*
     case 5: return rmse_launch<5>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
     case 6: return rmse_launch<6>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
     case 8: return rmse_launch<8>(x, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream);
+    default: return IQQ_ERR_ARG;
+    }
+}
+
+extern "C" iqq_status iqq_dequant_rmse_qx_bf16(int bits, const void* x, const void* blocks, const float* qw,
+                                               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, float* y,
+                                               double* d_acc, void* stream)
+{
+    if (y == nullptr && nrows > 0 && n_per_row > 0) return IQQ_ERR_NULL;
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    switch (bits) {
+    case 4: return rmse_launch<4>(xb, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    case 5: return rmse_launch<5>(xb, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    case 6: return rmse_launch<6>(xb, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
+    case 8: return rmse_launch<8>(xb, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
     default: return IQQ_ERR_ARG;
     }
 }

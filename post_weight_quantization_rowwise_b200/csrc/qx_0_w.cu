@@ -258,9 +258,9 @@ __device__ __forceinline__ void greedy_warp(const float* sX, const float* sW, fl
 // accumulate their round trip exactly as the weighted-RMSE reduction does: with e = x - y
 // in binary32, {sum qw e^2, sum qw, sum e^2} in binary64 and max |e|, one set of atomics
 // per warp (no CTA barrier).
-template <int BITS, bool EPI>
+template <int BITS, bool EPI, typename XT>
 __global__ void __launch_bounds__(kThreads, IQQ_Q4_MIN_CTAS)
-qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
+qx_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
               int chunks_per_row, const float* __restrict__ row_sigma2, float* __restrict__ y_out,
               double* __restrict__ acc_out, uint32_t* __restrict__ flags)
@@ -284,7 +284,7 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
     for (int64_t cta = blockIdx.x; cta < nwork; cta += gridDim.x) {
         const int64_t row = cta / chunks_per_row;
         const int chunk = static_cast<int>(cta - row * chunks_per_row);
-        const float* xr = x + row * n_per_row;
+        const XT* xr = x + row * n_per_row;
         const int64_t qrow = rows_per_qw > 0 ? row / rows_per_qw : 0;
         const float* qr = qw != nullptr ? qw + qrow * n_per_row : nullptr;
         uint32_t bad = 0u;
@@ -296,10 +296,10 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
         float xv[QK];
         float4 q4[QK / 4];
         if (valid) {
-            const float4* xb4 = reinterpret_cast<const float4*>(xr + b * QK);
+            const XT* xb = xr + b * QK;
 #pragma unroll
             for (int i = 0; i < QK / 4; ++i) {
-                const float4 v = __ldg(xb4 + i);
+                const float4 v = iqq::ld4(xb + 4 * i);
                 xv[4 * i] = v.x; xv[4 * i + 1] = v.y; xv[4 * i + 2] = v.z; xv[4 * i + 3] = v.w;
             }
             if (qr != nullptr) {
@@ -325,9 +325,8 @@ qx_0_w_kernel(const float* __restrict__ x, const float* __restrict__ qw, uint8_t
         } else {
             double acc = 0.0;
             float nf = 0.0f;
-            const float4* xr4 = reinterpret_cast<const float4*>(xr);
             for (int64_t i = threadIdx.x; i < n_per_row / 4; i += kThreads) {
-                const float4 v = __ldg(xr4 + i);
+                const float4 v = iqq::ld4(xr + 4 * i);
                 acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
                 acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
                 acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
@@ -637,17 +636,18 @@ constexpr int kPrepassThreads = 256;
 
 // sigma2 of each row (the same binary64 sum of exact squares and rounding as the fused
 // reduction), one CTA per row, and the non-finite check of x.
+template <typename XT>
 __global__ void __launch_bounds__(kPrepassThreads)
-row_sigma2_kernel(const float* __restrict__ x, int64_t nrows, int64_t n_per_row, float* __restrict__ out,
+row_sigma2_kernel(const XT* __restrict__ x, int64_t nrows, int64_t n_per_row, float* __restrict__ out,
                   uint32_t* __restrict__ flags)
 {
     __shared__ double s_red[kPrepassThreads / 32];
     for (int64_t row = blockIdx.x; row < nrows; row += gridDim.x) {
-        const float4* xr4 = reinterpret_cast<const float4*>(x + row * n_per_row);
+        const XT* xr = x + row * n_per_row;
         double acc = 0.0;
         float nf = 0.0f;
         for (int64_t i = threadIdx.x; i < n_per_row / 4; i += kPrepassThreads) {
-            const float4 v = iqq::ld_stream_f4(xr4 + i);
+            const float4 v = iqq::ld4_stream(xr + 4 * i);
             acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
             acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
             acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
@@ -686,8 +686,8 @@ int64_t workspace_bytes_for(int64_t nrows, int64_t n_per_row)
     return (nrows * 4 + 255) / 256 * 256;
 }
 
-template <int BITS, bool EPI>
-iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
+template <int BITS, bool EPI, typename XT>
+iqq_status launch_qx(const XT* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
                      int64_t rows_per_qw, int weight_mode, float fudge, const float* row_sigma2, float* y_out,
                      double* acc, uint32_t* d_flags, void* stream)
 {
@@ -700,33 +700,34 @@ iqq_status launch_qx(const float* x, const float* qw, void* out, int64_t nrows, 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return iqq::launch_status();
     if (configured_device != dev) {
-        if (cudaFuncSetAttribute(qx_0_w_kernel<BITS, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(qx_0_w_kernel<BITS, EPI, XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kDynSmem)) != cudaSuccess)
             return iqq::launch_status();
         configured_device = dev;
     }
-    qx_0_w_kernel<BITS, EPI><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
+    qx_0_w_kernel<BITS, EPI, XT><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
         x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode, fudge,
         static_cast<int>(chunks), row_sigma2, y_out, acc, d_flags);
     return iqq::launch_status();
 }
 
-template <int BITS>
-iqq_status launch_bits(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
+template <int BITS, typename XT>
+iqq_status launch_bits(const XT* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
                        int64_t rows_per_qw, int weight_mode, float fudge, const float* rs, float* y_out,
                        double* acc, uint32_t* d_flags, void* stream)
 {
     if (acc != nullptr || y_out != nullptr)
-        return launch_qx<BITS, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out,
+        return launch_qx<BITS, true, XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out,
                                      acc, d_flags, stream);
-    return launch_qx<BITS, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, nullptr,
+    return launch_qx<BITS, false, XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, nullptr,
                                   nullptr, d_flags, stream);
 }
 
 // workspace == nullptr: the fused reduction.  Otherwise it holds at least
 // workspace_bytes_for(nrows, n_per_row) bytes (checked by the caller).  acc: optional
 // round-trip error accumulator (8-byte aligned, checked by the caller).
-iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int64_t nrows,
+template <typename XT>
+iqq_status quantize_qx(int bits, const XT* x, const float* qw, void* out, int64_t nrows,
                        int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
                        uint32_t* d_flags, void* stream, double* acc = nullptr, float* y_out = nullptr,
                        float fudge = 1.0f)
@@ -744,17 +745,17 @@ iqq_status quantize_qx(int bits, const float* x, const float* qw, void* out, int
     if (workspace != nullptr && workspace_bytes_for(nrows, n_per_row) > 0) {
         float* ws = static_cast<float*>(workspace);
         const int64_t g = nrows < 0x7fffffff ? nrows : 0x7fffffff;
-        row_sigma2_kernel<<<static_cast<int>(g), kPrepassThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        row_sigma2_kernel<XT><<<static_cast<int>(g), kPrepassThreads, 0, static_cast<cudaStream_t>(stream)>>>(
             x, nrows, n_per_row, ws, d_flags);
         const iqq_status st = iqq::launch_status();
         if (st != IQQ_OK) return st;
         rs = ws;
     }
     switch (bits) {
-    case 4: return launch_bits<4>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
-    case 5: return launch_bits<5>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
-    case 6: return launch_bits<6>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
-    default: return launch_bits<8>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    case 4: return launch_bits<4, XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    case 5: return launch_bits<5, XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    case 6: return launch_bits<6, XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
+    default: return launch_bits<8, XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, rs, y_out, acc, d_flags, stream);
     }
 }
 
@@ -862,4 +863,22 @@ extern "C" iqq_status iqq_quantize_qx_0_w_ws(int bits, const float* x, const flo
     }
     return quantize_qx(bits, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode,
                        need > 0 ? workspace : nullptr, d_flags, stream);
+}
+
+extern "C" iqq_status iqq_quantize_qx_0_w_bf16(int bits, const void* x, const float* qw, void* out,
+                                               int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                                               int weight_mode, void* workspace, size_t workspace_bytes,
+                                               uint32_t* d_flags, void* stream)
+{
+    if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
+    if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0 || n_per_row % QK != 0) return IQQ_ERR_SHAPE;
+    const int64_t need = workspace_bytes_for(nrows, n_per_row);
+    void* ws = nullptr;
+    if (need > 0 && workspace != nullptr) {
+        if (workspace_bytes < static_cast<size_t>(need)) return IQQ_ERR_SHAPE;
+        if (!iqq::aligned(workspace, 16)) return IQQ_ERR_ALIGN;
+        ws = workspace;
+    }
+    return quantize_qx(bits, static_cast<const __nv_bfloat16*>(x), qw, out, nrows, n_per_row, rows_per_qw,
+                       weight_mode, ws, d_flags, stream);
 }

@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
               "iqq_quantize_qx_0_w", "iqq_dequant_qx_0", "iqq_gemv_q4_0_q8_k128",
               "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
               "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch",
-              "iqq_quantize_qx_0_w_ex", "iqq_dequant_rmse_qx"):
+              "iqq_quantize_qx_0_w_ex", "iqq_dequant_rmse_qx", "iqq_quantize_qx_0_w_bf16",
+              "iqq_dequant_rmse_qx_bf16"):
         assert n in names
 
 
@@ -140,6 +141,21 @@ def test_host_validation_without_gpu(lib):
     assert DR(4, V(16), V(16), None, 1, 32, 0, V(8), V(16), None) == 3
     assert DR(7, V(16), V(16), None, 1, 32, 0, V(16), V(16), None) == 5
     assert DR(4, V(16), V(16), None, 1, 48, 0, V(16), V(16), None) == 2
+    # bf16 weights: the same checks (x 16-byte aligned), the optional workspace
+    QB = lib.iqq_quantize_qx_0_w_bf16
+    assert QB(7, V(16), None, V(16), 2, 4096, 0, 0, None, 0, None, None) == 5
+    assert QB(4, V(16), None, V(16), 2, 4097, 0, 0, None, 0, None, None) == 2
+    assert QB(4, None, None, V(16), 2, 4096, 0, 0, None, 0, None, None) == 1
+    assert QB(4, V(8), None, V(16), 2, 4096, 0, 0, None, 0, None, None) == 3
+    assert QB(4, V(16), None, V(16), 2, 4096, 0, 6, None, 0, None, None) == 5
+    assert QB(4, V(16), None, V(16), 2, 53248, 0, 0, V(16), 8, None, None) == 2   # workspace too small
+    assert QB(4, V(16), None, V(16), 2, 53248, 0, 0, V(8), 256, None, None) == 3
+    assert QB(4, None, None, None, 0, 4096, 0, 0, None, 0, None, None) == 0
+    DB = lib.iqq_dequant_rmse_qx_bf16
+    assert DB(4, V(16), V(16), None, 1, 32, 0, None, V(16), None) == 1
+    assert DB(4, V(8), V(16), None, 1, 32, 0, V(16), V(16), None) == 3
+    assert DB(7, V(16), V(16), None, 1, 32, 0, V(16), V(16), None) == 5
+    assert DB(4, V(16), V(16), None, 1, 48, 0, V(16), V(16), None) == 2
     # Q4_0 x Q8_K_128 matrix-vector product
     G = lib.iqq_gemv_q4_0_q8_k128
     assert G(V(16), V(16), V(16), 4, 96, 1, None, None) == 2          # k not a multiple of 128

@@ -458,3 +458,60 @@ def test_runs_on_a_side_stream(iqq, synth):
         out = iqq.quantize_q4_0_w(x, stream=s)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("bits", [4, 5, 6, 8])
+@pytest.mark.parametrize("rows,n,rpq", [(64, 4096, 0), (9, 11008, 3), (3, 53248, 0), (7, 4192, 1)])
+def test_bf16_input_equals_the_widened_tensor(iqq, synth, bits, rows, n, rpq):
+    """bf16 weights give, bit for bit, the blocks and flags of their exact binary32 widening
+    (fused path, and with the workspace for wide rows), and the one-pass round trip against
+    the bf16 tensor gives the binary32 one's y, sums and max|e|; the blocks meet the oracle
+    bar."""
+    xb = synth.weight_matrix(rows, n, seed=rows * 7 + n + bits, bf16=True).to(torch.bfloat16).cuda()
+    x32 = xb.float()
+    nq = (rows + rpq - 1) // rpq if rpq else 1
+    qw = torch.stack([synth.imatrix(n, seed=n + i) for i in range(nq)]) if rpq else synth.imatrix(n, seed=n)
+    qd = qw.cuda()
+    f32, fbf = (torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2))
+    g32 = iqq.quantize_qx_0_w(bits, x32, qd, rows_per_qw=rpq, flags=f32)
+    gbf = torch.empty_like(g32)
+    iqq.iqq_quantize_qx_0_w_bf16(bits, xb, qd, gbf, rows_per_qw=rpq, flags=fbf)
+    torch.cuda.synchronize()
+    assert torch.equal(gbf, g32) and int(fbf.item()) == int(f32.item()) == 0
+    nws = iqq.qx_0_w_workspace_bytes(rows, n)
+    if nws > 0:
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        g32w = iqq.quantize_qx_0_w_ws(bits, x32, qd, rows_per_qw=rpq)
+        gbfw = torch.empty_like(g32)
+        iqq.iqq_quantize_qx_0_w_bf16(bits, xb, qd, gbfw, rows_per_qw=rpq, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(gbfw, g32w)
+    if rpq == 0:
+        x = x32.cpu().numpy()
+        o, _ = oracle.quantize_qx_0_w(bits, x, qw.numpy())
+        _compare_qx(bits, x, qw.numpy(), gbf.cpu().numpy(), o, rows, n)
+    y32, ybf = torch.empty_like(x32), torch.empty_like(x32)
+    a32, abf = (torch.zeros(4, dtype=torch.float64, device="cuda") for _ in range(2))
+    iqq.iqq_dequant_rmse_qx(bits, x32, g32, qd, y32, a32, rows_per_qw=rpq)
+    iqq.iqq_dequant_rmse_qx_bf16(bits, xb, g32, qd, ybf, abf, rows_per_qw=rpq)
+    torch.cuda.synchronize()
+    assert torch.equal(ybf, y32)
+    a32, abf = a32.cpu().tolist(), abf.cpu().tolist()
+    for i in range(3):  # binary64 atomics: the order of the per-CTA partial sums may vary
+        assert abs(abf[i] - a32[i]) <= 1e-12 * abs(a32[i])
+    assert abf[3] == a32[3]
+
+
+def test_bf16_input_flags_nonfinite(iqq):
+    """An infinity in bf16 x raises IQQ_FLAG_NONFINITE_INPUT on the fused path and in the
+    per-row pass of wide rows."""
+    for n in (4096, 53248):
+        x = torch.zeros(4, n, dtype=torch.bfloat16, device="cuda")
+        x[2, 100] = float("inf")
+        out = torch.empty((4, (n // 32) * 18), dtype=torch.uint8, device="cuda")
+        flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nws = iqq.qx_0_w_workspace_bytes(4, n)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda") if nws else None
+        iqq.iqq_quantize_qx_0_w_bf16(4, x, None, out, workspace=ws, flags=flags)
+        torch.cuda.synchronize()
+        assert int(flags.item()) & iqq.FLAG_NONFINITE_INPUT
