@@ -177,3 +177,27 @@ def test_gemv_batch_ctas_spanning_problems(iqq, synth):
         assert torch.equal(y, single)
         yo, s = oracle.dot_q4_0_q8_k128(w.cpu().numpy(), a.cpu().numpy(), n_out, k, n_tok)
         _check(y.cpu().numpy(), yo, s, k)
+
+
+def test_gemv_batch_rows_wider_than_a_share(iqq, synth):
+    """One 65536-wide row among 40 one-row problems of width 128: the CTAs split the bytes
+    evenly, so one CTA takes the wide row alone and another has no row to start; every
+    output equals its single call bit for bit and lies within the bound of the oracle's
+    value."""
+    rng = np.random.default_rng(42)
+    items, singles, refs = [], [], []
+    for i, (n_out, k, n_tok) in enumerate([(1, 65536, 2)] + [(1, 128, 1 + i % 3) for i in range(40)]):
+        w = torch.from_numpy(_random_q4_0(rng, n_out, k)).cuda()
+        a = torch.from_numpy(_activations(synth, n_tok, k, seed=200 + i)).cuda()
+        y = torch.full((n_tok, n_out), float("nan"), device="cuda")
+        items.append((w, a, y, k))
+        singles.append(iqq.gemv_q4_0_q8_k128(w, a, n_out, k, n_tok))
+        refs.append((n_out, k, n_tok))
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    iqq.iqq_gemv_q4_0_q8_k128_batch(iqq.gemv_problems(items), flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    for (w, a, y, k), single, (n_out, _, n_tok) in zip(items, singles, refs):
+        assert torch.equal(y, single)
+        yo, s = oracle.dot_q4_0_q8_k128(w.cpu().numpy(), a.cpu().numpy(), n_out, k, n_tok)
+        _check(y.cpu().numpy(), yo, s, k)
