@@ -595,7 +595,7 @@ def main_ours(args):
         "data": "synthetic (seeded; no model weights or calibration data)",
         "config": {"workload": WORKLOAD, "layers": args.layers, "tensors": n_q4,
                    "q4_0_values": w.q4_elems, "q8_k128_values": w.q8_elems,
-                   "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (replicas)"},
+                   "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (a layer set per rank, no data-path collective)"},
         "roofline": {"bound": "alu", "kernel": "qx_0_w_kernel<4>",
                      "achieved": round(achieved, 3),
                      "peak": round(peak_ops, 3), "unit": "Tops/s",
