@@ -26,7 +26,9 @@
  *  - Data problems found on the device (NaN/Inf input, negative importance,
  *    a scale beyond binary16) are ORed as IQQ_FLAG_* bits into the optional
  *    caller-owned device word *d_flags (may be NULL).  Nothing on the device
- *    traps, asserts or waits.
+ *    traps or asserts.  The only waits on the device are the GEMV kernel's
+ *    waits for its own bulk copies: each is bounded (about 2 s), and on expiry
+ *    the kernel sets IQQ_FLAG_WAIT_TIMEOUT, drains its copies and returns.
  *  - Empty input (nrows == 0 or n_per_row == 0) is valid and enqueues
  *    nothing; pointers may then be NULL.
  *  - Layouts are row-major: element (r, j) of an [nrows, n_per_row] float
@@ -80,7 +82,10 @@ typedef enum {
  *
  *  x          [nrows, n_per_row] float32, 16-byte aligned.
  *  qw         imatrix rows, float32, 16-byte aligned, or NULL (qw = 1).  Row r
- *             uses qw + (rows_per_qw > 0 ? r / rows_per_qw : 0) * n_per_row.
+ *             uses qw + (rows_per_qw > 0 ? r / rows_per_qw : 0) * n_per_row, so qw
+ *             must hold (rows_per_qw > 0 ? ceil(nrows / rows_per_qw) : 1) * n_per_row
+ *             values on the device of x (the library cannot check this; the Python
+ *             binding does).
  *  out        nrows * n_per_row / 32 blocks of 18 bytes, 2-byte aligned:
  *             bytes 0-1 binary16 d (little endian), byte 2+i holds
  *             (l[i]+8) | (l[i+16]+8) << 4 for i = 0..15.

@@ -4,8 +4,11 @@ Thin Python binding over the C ABI in ``include/iqq.h`` (``libiqq.so`` in this
 package).  The functions have the ABI's names; they only check and marshal
 arguments (torch CUDA tensors -> device pointers, sizes and the current CUDA
 stream).  Every step of the computation runs in the library's CUDA kernels:
-there is no CPU or PyTorch fallback, and importing this package raises if the
-library is missing or fails to load.
+there is no CPU or PyTorch fallback.
+
+The library is loaded on the first call into it (importing the package alone,
+for example for its ``synth`` input generators, maps no native code); that
+first call raises ImportError if ``libiqq.so`` is missing or fails to load.
 
 Block formats (little endian):
   Q4_0      18 bytes per 32 values: binary16 d | qs[16], qs[i] = (l[i]+8) | (l[i+16]+8) << 4
@@ -77,7 +80,23 @@ def _load():
     return lib
 
 
-_lib = _load()
+class _LazyLib:
+    """libiqq.so, loaded on first use (ImportError when missing: no fallback exists)."""
+
+    _handle = None
+
+    def __getattr__(self, name):
+        if _LazyLib._handle is None:
+            _LazyLib._handle = _load()
+        return getattr(_LazyLib._handle, name)
+
+
+_lib = _LazyLib()
+
+
+def loaded() -> bool:
+    """True once libiqq.so has been loaded into this process."""
+    return _LazyLib._handle is not None
 
 
 class IQQError(RuntimeError):
@@ -132,6 +151,36 @@ def _need_cuda(name, t, dtype=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def qw_rows_needed(nrows: int, rows_per_qw: int) -> int:
+    """imatrix rows an operation over nrows rows reads: one per rows_per_qw rows
+    (ceil), or one shared row when rows_per_qw is 0."""
+    if rows_per_qw < 0:
+        raise ValueError("rows_per_qw must be >= 0")
+    if nrows <= 0:
+        return 0
+    return -(-nrows // rows_per_qw) if rows_per_qw > 0 else 1
+
+
+def _check_qw(qw, nrows: int, n_per_row: int, rows_per_qw: int, device=None) -> None:
+    """Rejects an imatrix the kernels would read past: qw must hold
+    qw_rows_needed(nrows, rows_per_qw) * n_per_row values (None: qw = 1) and live on
+    the device of the data it weights."""
+    need = qw_rows_needed(nrows, rows_per_qw) * n_per_row
+    if qw is None:
+        return
+    if qw.numel() < need:
+        raise ValueError(f"qw holds {qw.numel()} values; {nrows} rows of {n_per_row} with "
+                         f"rows_per_qw={rows_per_qw} read {need}")
+    if device is not None and qw.device != device:
+        raise ValueError(f"qw is on {qw.device}, the data on {device}")
+
+
+def _same_device(x, **others) -> None:
+    for name, t in others.items():
+        if t is not None and t.device != x.device:
+            raise ValueError(f"{name} is on {t.device}, x on {x.device}")
+
+
 def _shape2(x):
     if x.dim() != 2:
         raise ValueError("x must be 2-D [nrows, n_per_row]")
@@ -159,6 +208,8 @@ def iqq_quantize_q4_0_w(x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, 
     _need_cuda("out", out, torch.uint8)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags)
     if out.numel() < q4_0_nbytes(nrows, n):
         raise ValueError("out is too small")
     _check("iqq_quantize_q4_0_w",
@@ -179,6 +230,8 @@ def iqq_quantize_qx_0_w(bits, x, qw, out, rows_per_qw: int = 0, weight_mode: int
     _need_cuda("out", out, torch.uint8)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
@@ -194,6 +247,7 @@ def iqq_dequant_qx_0(bits, blocks, y, stream=None):
     _need_cuda("blocks", blocks, torch.uint8)
     _need_cuda("y", y, torch.float32)
     nrows, n = _shape2(y)
+    _same_device(y, blocks=blocks)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
@@ -218,6 +272,8 @@ def iqq_quantize_qx_0_w_ws(bits, x, qw, out, workspace, rows_per_qw: int = 0, we
     _need_cuda("workspace", workspace, torch.uint8)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags, workspace=workspace)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
@@ -240,6 +296,8 @@ def iqq_quantize_qx_0_w_bf16(bits, x, qw, out, rows_per_qw: int = 0, weight_mode
     _need_cuda("workspace", workspace, torch.uint8)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags, workspace=workspace)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
@@ -258,6 +316,7 @@ def iqq_quantize_q8_k128(x, out, flags=None, stream=None):
     _need_cuda("out", out, torch.uint8)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _same_device(x, out=out, flags=flags)
     if out.numel() < q8_k128_nbytes(nrows, n):
         raise ValueError("out is too small")
     _check("iqq_quantize_q8_k128",
@@ -274,6 +333,7 @@ def iqq_quantize_q8_1(x, out, overflow=None, flags=None, stream=None):
     _need_cuda("overflow", overflow, torch.int64)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _same_device(x, out=out, overflow=overflow, flags=flags)
     if out.numel() < nrows * (n // 32) * 36:
         raise ValueError("out is too small")
     _check("iqq_quantize_q8_1",
@@ -288,6 +348,7 @@ def iqq_dequant_q4_0(blocks, y, stream=None):
     _need_cuda("blocks", blocks, torch.uint8)
     _need_cuda("y", y, torch.float32)
     nrows, n = _shape2(y)
+    _same_device(y, blocks=blocks)
     if blocks.numel() < q4_0_nbytes(nrows, n):
         raise ValueError("blocks is too small")
     _check("iqq_dequant_q4_0", _lib.iqq_dequant_q4_0(_ptr(blocks), _ptr(y), nrows, n, _stream(stream)))
@@ -303,6 +364,7 @@ def iqq_gemv_q4_0_q8_k128(w_blocks, a_blocks, y, k: int, flags=None, stream=None
     _need_cuda("y", y, torch.float32)
     _need_cuda("flags", flags, torch.int32)
     n_tok, n_out = _shape2(y)
+    _same_device(y, w_blocks=w_blocks, a_blocks=a_blocks, flags=flags)
     if w_blocks.numel() < q4_0_nbytes(n_out, k):
         raise ValueError("w_blocks is too small")
     if a_blocks.numel() < q8_k128_nbytes(n_tok, k):
@@ -352,6 +414,8 @@ def iqq_weighted_rmse(x, blocks, qw, acc, rows_per_qw: int = 0, stream=None):
     _need_cuda("qw", qw, torch.float32)
     _need_cuda("acc", acc, torch.float64)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, blocks=blocks, acc=acc)
     if blocks.numel() < q4_0_nbytes(nrows, n) or acc.numel() < 4:
         raise ValueError("blocks or acc is too small")
     _check("iqq_weighted_rmse",
@@ -369,6 +433,8 @@ def iqq_dequant_rmse_qx(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, strea
     _need_cuda("y", y, torch.float32)
     _need_cuda("acc", acc, torch.float64)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, blocks=blocks, y=y, acc=acc)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits] or acc.numel() < 4 or y.numel() < x.numel():
@@ -389,6 +455,8 @@ def iqq_dequant_rmse_qx_bf16(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, 
     _need_cuda("y", y, torch.float32)
     _need_cuda("acc", acc, torch.float64)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, blocks=blocks, y=y, acc=acc)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits] or acc.numel() < 4 or y.numel() < x.numel():
@@ -407,6 +475,8 @@ def iqq_weighted_rmse_qx(bits, x, blocks, qw, acc, rows_per_qw: int = 0, stream=
     _need_cuda("qw", qw, torch.float32)
     _need_cuda("acc", acc, torch.float64)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, blocks=blocks, acc=acc)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if blocks.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits] or acc.numel() < 4:
@@ -459,6 +529,8 @@ def iqq_quantize_qx_0_w_ex(bits, x, qw, out, workspace=None, acc=None, rows_per_
     _need_cuda("acc", acc, torch.float64)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags, workspace=workspace, y=y, acc=acc)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:
@@ -485,6 +557,8 @@ def iqq_quantize_qx_0_w_static(bits, x, qw, out, rows_per_qw: int = 0, weight_mo
     _need_cuda("out", out, torch.uint8)
     _need_cuda("flags", flags, torch.int32)
     nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags)
     if bits not in QX_0_BLOCK_BYTES:
         raise ValueError("bits must be 4, 5, 6 or 8")
     if out.numel() < nrows * (n // 32) * QX_0_BLOCK_BYTES[bits]:

@@ -791,33 +791,34 @@ extern "C" iqq_status iqq_quantize_qx_0_w_static(int bits, const float* x, const
         return IQQ_ERR_ALIGN;  // every host check before the first CUDA call
     void* ws = nullptr;
     if (cudaGetSymbolAddress(&ws, g_static_sigma2) != cudaSuccess) return iqq::launch_status();
-    // row batches that fit the static rows; each batch is a tensor of its own rows (the
-    // imatrix row of a batch row follows from its global index)
+    // row batches that fit the static rows; each batch is a tensor of its own rows.  With one
+    // imatrix row per rows_per_qw rows, a batch is a whole number of imatrix groups, so that
+    // it starts on an imatrix-row boundary and takes its imatrix rows from there; only a
+    // group larger than the array itself is split, one part of one group per batch.
     const int64_t bb = bits == 4 ? Fmt<4>::bytes : bits == 5 ? Fmt<5>::bytes : bits == 6 ? Fmt<6>::bytes : Fmt<8>::bytes;
-    for (int64_t r0 = 0; r0 < nrows; r0 += IQQ_STATIC_WS_ROWS) {
-        const int64_t nr = nrows - r0 < IQQ_STATIC_WS_ROWS ? nrows - r0 : IQQ_STATIC_WS_ROWS;
+    const bool grouped = qw != nullptr && rows_per_qw > 0;
+    const int64_t batch = grouped && rows_per_qw <= IQQ_STATIC_WS_ROWS
+                              ? (IQQ_STATIC_WS_ROWS / rows_per_qw) * rows_per_qw
+                              : IQQ_STATIC_WS_ROWS;
+    for (int64_t r0 = 0; r0 < nrows;) {
+        int64_t nr = nrows - r0 < batch ? nrows - r0 : batch;
         const float* qb = qw;
-        if (qw != nullptr && rows_per_qw > 0) {
-            // a batch starts on an imatrix-row boundary only if IQQ_STATIC_WS_ROWS is a
-            // multiple of rows_per_qw; otherwise quantize the batch row by imatrix segment
-            if (IQQ_STATIC_WS_ROWS % rows_per_qw != 0) {
-                for (int64_t s0 = r0; s0 < r0 + nr;) {
-                    const int64_t q = s0 / rows_per_qw;
-                    const int64_t s1 = (q + 1) * rows_per_qw < r0 + nr ? (q + 1) * rows_per_qw : r0 + nr;
-                    const iqq_status st = quantize_qx(bits, x + s0 * n_per_row, qw + q * n_per_row,
-                                                      static_cast<uint8_t*>(out) + s0 * (n_per_row / QK) * bb,
-                                                      s1 - s0, n_per_row, 0, weight_mode, ws, d_flags, stream);
-                    if (st != IQQ_OK) return st;
-                    s0 = s1;
-                }
-                continue;
+        int64_t rpq = rows_per_qw;
+        if (grouped) {
+            const int64_t q = r0 / rows_per_qw;
+            qb = qw + q * n_per_row;
+            if (rows_per_qw > IQQ_STATIC_WS_ROWS) {
+                // a part of one imatrix group: it ends at the group's end at the latest
+                const int64_t group_end = (q + 1) * rows_per_qw;
+                if (r0 + nr > group_end) nr = group_end - r0;
+                rpq = 0;
             }
-            qb = qw + (r0 / rows_per_qw) * n_per_row;
         }
         const iqq_status st = quantize_qx(bits, x + r0 * n_per_row, qb,
                                           static_cast<uint8_t*>(out) + r0 * (n_per_row / QK) * bb, nr, n_per_row,
-                                          rows_per_qw, weight_mode, ws, d_flags, stream);
+                                          rpq, weight_mode, ws, d_flags, stream);
         if (st != IQQ_OK) return st;
+        r0 += nr;
     }
     return IQQ_OK;
 }

@@ -181,3 +181,39 @@ def test_python_binding_requires_cuda_tensors():
     import post_weight_quantization_rowwise_b200 as m
     with pytest.raises(ValueError):
         m.quantize_q4_0_w(torch.zeros(2, 64))
+
+
+def test_binding_rejects_an_imatrix_the_kernels_would_overrun():
+    """The binding checks qw's size against the rows it covers before any CUDA call: one
+    imatrix row per rows_per_qw rows (ceil), or one shared row."""
+    import torch
+    import post_weight_quantization_rowwise_b200 as m
+    assert m.qw_rows_needed(6, 3) == 2 and m.qw_rows_needed(7, 3) == 3
+    assert m.qw_rows_needed(5, 0) == 1 and m.qw_rows_needed(0, 4) == 0
+    with pytest.raises(ValueError):
+        m.qw_rows_needed(4, -1)
+    n = 64
+    m._check_qw(None, 6, n, 3)                                  # qw = 1: nothing to read
+    m._check_qw(torch.zeros(2 * n), 6, n, 3)                    # exactly enough
+    with pytest.raises(ValueError):
+        m._check_qw(torch.zeros(n), 6, n, 3)                    # one row for two groups
+    with pytest.raises(ValueError):
+        m._check_qw(torch.zeros(2 * n), 7, n, 3)                # the third group's row is missing
+    with pytest.raises(ValueError):
+        m._check_qw(torch.zeros(n - 1), 1, n, 0)                # a short shared row
+    with pytest.raises(ValueError):
+        m._check_qw(torch.zeros(n), 1, n, 0, device=torch.device("meta"))  # another device
+
+
+def test_importing_the_package_maps_no_library():
+    """Only a call loads libiqq.so: the input generators can be imported without it."""
+    import subprocess
+    import sys
+    code = ("import post_weight_quantization_rowwise_b200 as m\n"
+            "from post_weight_quantization_rowwise_b200 import synth\n"
+            "assert not m.loaded()\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "assert 'libiqq.so' not in maps, 'mapped at import'\n"
+            "m.version()\n"
+            "assert m.loaded() and 'libiqq.so' in open('/proc/self/maps').read()\n")
+    subprocess.run([sys.executable, "-c", code], check=True, cwd=ROOT)

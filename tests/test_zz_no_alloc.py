@@ -39,17 +39,20 @@ def test_two_calls_match_the_workspace_entry(iqq, synth):
 
 
 def test_row_batches_and_imatrix_segments(iqq, synth):
-    """More rows than the static array: batches of rows, with a shared imatrix row and with
-    one imatrix row per 3 rows (batches then split at imatrix-row boundaries)."""
+    """More rows than the static array: batches of rows, with a shared imatrix row, with one
+    imatrix row per 3 rows (batches of 16383 rows, whole groups) and with one per 4 rows (4
+    divides the array's rows: the second batch takes its imatrix rows from row 4096 on)."""
     rows, n = STATIC_ROWS + 3, 12320
     x = synth.weight_matrix(rows, n, seed=21, device="cuda")
     q1 = synth.imatrix(n, seed=22, device="cuda")
     q3 = torch.stack([synth.imatrix(n, seed=100 + i, device="cuda") for i in range((rows + 2) // 3)])
-    for qw, rpq in ((q1, 0), (q3, 3)):
-        a = _static(iqq, 4, x, qw, rpq)
-        b = iqq.quantize_qx_0_w_ws(4, x, qw, rows_per_qw=rpq)
-        torch.cuda.synchronize()
-        assert torch.equal(a, b.view(-1))
+    q4 = synth.imatrix(n * ((rows + 3) // 4), seed=200_000, device="cuda").view(-1, n)
+    for bits in (4, 8):
+        for qw, rpq in ((q1, 0), (q3, 3), (q4, 4)):
+            a = _static(iqq, bits, x, qw, rpq)
+            b = iqq.quantize_qx_0_w_ws(bits, x, qw, rows_per_qw=rpq)
+            torch.cuda.synchronize()
+            assert torch.equal(a, b.view(-1)), (bits, rpq)
 
 
 def test_narrow_rows_and_flags(iqq, synth):
