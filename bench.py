@@ -132,7 +132,8 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle
 
 def _oracle_chunk(args):
-    """Worker: the oracle's whole path on one sample chunk (runs in a spawned process)."""
+    """Worker: the oracle's whole path on one chunk of the fixed sample (a spawned process).
+    The inputs are drawn first and not timed (the GPU arm's inputs are resident too)."""
     import oracle
     from post_weight_quantization_rowwise_b200 import synth
     kind, rows, cols, seed, bf16 = args
@@ -150,44 +151,53 @@ def _oracle_chunk(args):
     return x.size, time.perf_counter() - t0, int(passes.sum()), int(passes.size)
 
 
-def oracle_sample(target_seconds: float = 12.0, cores: int | None = None, pool=None):
-    """Times the unchanged single-threaded oracle on a bounded sample of the workload,
-    one process per core: rows of every tensor shape of the layer set (same recipe,
-    in the layer set's proportions of values) and Q8_K_128 activation rows (in the
-    step's proportion).  The rate is the sum over processes of each process's own rate
-    (independent rows, so the copies do not interact).
-    Returns (Gelem/s, cores, sample description, mean greedy passes)."""
-    import multiprocessing as mp
+# The oracle's sample of the workload: 2^25 Q4_0 values (quantize + dequant + weighted RMSE)
+# spread over the seven tensor shapes of the layer set in the set's proportions, plus Q8_K_128
+# activation rows in the step's proportion (4096 x 7168 per 32 layers), cut into chunks of
+# about 1 M values so that every core stays busy.  The same fixed sample serves the
+# cpu_baseline leg and every step of the reference arm.
+ORACLE_SAMPLE_Q4_VALUES = 1 << 25
+ORACLE_CHUNK_VALUES = 1 << 20
+
+
+def oracle_jobs():
     from post_weight_quantization_rowwise_b200 import synth
-    cores = cores or os.cpu_count() or 1
     layer = synth.LLAMA2_7B_TENSORS
     layer_elems = sum(r * c for _, r, c in layer)
-    budget = 3.0e6 * target_seconds * cores          # values; ~3 M values/s per process
-    chunk = max(budget / (3 * cores), 4096 * 8)
     jobs = []
     for i, (name, r, c) in enumerate(layer):
-        rows = max(1, int(budget * (r * c) / layer_elems / c))
-        per = max(1, int(chunk // c))
+        rows = max(1, round(ORACLE_SAMPLE_Q4_VALUES * (r * c) / layer_elems / c))
+        per = max(1, ORACLE_CHUNK_VALUES // c)
         for k, r0 in enumerate(range(0, rows, per)):
             jobs.append(("q4", min(per, rows - r0), c, 9000 + 100 * i + k, True))
-    q8_rows = max(1, int(budget * 4096 * 7168 / (32 * layer_elems) / 7168))
+    q8_rows = max(1, round(ORACLE_SAMPLE_Q4_VALUES * 4096 * 7168 / (32 * layer_elems) / 7168))
     jobs.append(("q8", q8_rows, 7168, 2, False))
-    t0 = time.perf_counter()
+    return jobs
+
+
+def oracle_sample(cores: int | None = None, pool=None):
+    """Times the unchanged single-threaded oracle on the fixed sample, one process per host
+    core.  Each chunk's oracle time is measured in its process; the step time is the sum of
+    those times over the cores (the processes are independent).
+    Returns (Gelem/s, cores, sample description, mean greedy passes, step seconds)."""
+    import multiprocessing as mp
+    cores = cores or os.cpu_count() or 1
+    jobs = oracle_jobs()
     if pool is None:
         with mp.get_context("spawn").Pool(cores) as own:
             res = own.map(_oracle_chunk, jobs, chunksize=1)
     else:
         res = pool.map(_oracle_chunk, jobs, chunksize=1)
-    wall = time.perf_counter() - t0
     elems = sum(r[0] for r in res)
     busy = sum(r[1] for r in res)
     pass_sum = sum(r[2] for r in res)
     pass_n = sum(r[3] for r in res)
-    value = elems / (busy / cores) / 1e9
-    sample = (f"{elems / 1e6:.1f} M values ({len(jobs) - 1} Q4_0 chunks over the 7 tensor shapes "
-              f"in layer-set proportion + {q8_rows} Q8_K_128 rows); {cores} processes, "
-              f"{busy:.1f} s CPU, {wall:.1f} s wall")
-    return value, cores, sample, pass_sum / max(pass_n, 1)
+    step_s = busy / cores
+    sample = (f"fixed sample of {elems / 1e6:.1f} M values: {ORACLE_SAMPLE_Q4_VALUES / 1e6:.1f} M Q4_0 "
+              f"(quantize + dequant + weighted RMSE) over the layer set's 7 shapes in its proportions, "
+              f"plus {jobs[-1][1]} Q8_K_128 rows of 7168; {len(jobs)} chunks on {cores} processes, "
+              f"{busy:.1f} s of oracle time per pass")
+    return elems / step_s / 1e9, cores, sample, pass_sum / max(pass_n, 1), step_s
 
 
 # ----------------------------------------------------------------------------- the GPU step
@@ -401,11 +411,9 @@ def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
 
 def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     """The same step through the public API from pinned host buffers, every byte of input
-    crossing PCIe each step: per tensor H2D of x and qw, its two kernels, D2H of the
-    blocks; H2D of the activations, Q8_K_128, D2H of its blocks and of the accumulator.
-    The layer set's weights are bf16 values (a bf16 checkpoint's), so x travels as bf16 and
-    goes through the bf16 entry points, which widen it exactly in the kernels: the blocks,
-    y and sums are those of the binary32 step.
+    crossing PCIe each step: per tensor H2D of x (binary32: the layer set's outliers are not
+    bf16 values) and qw, its two kernels, D2H of the blocks; H2D of the activations,
+    Q8_K_128, D2H of its blocks and of the accumulator.
     The copies run on their own streams (host to device, device to host) with two device
     staging slots, so tensor i + 1 uploads and tensor i - 1 downloads while tensor i
     computes; events order every reuse of a slot or buffer.  ``barrier`` (several ranks)
@@ -419,14 +427,14 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
         h.copy_(t)
         return h
 
-    host_x = [pinned_copy(w.x[i], torch.bfloat16) for i in range(n)]  # exact: bf16 values
+    host_x = [pinned_copy(w.x[i]) for i in range(n)]
     host_qw = [pinned_copy(w.qw[i]) for i in range(n)]
     host_b = [torch.empty(w.blocks[i].numel(), dtype=torch.uint8, pin_memory=True) for i in range(n)]
     host_act = pinned_copy(w.act)
     host_q8 = torch.empty(w.q8.numel(), dtype=torch.uint8, pin_memory=True)
     host_acc = torch.empty(4, dtype=torch.float64, pin_memory=True)
     big = max(t.numel for t in w.tensors[:n])
-    xd = [torch.empty(big, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    xd = [torch.empty(big, dtype=torch.float32, device=dev) for _ in range(2)]
     qd = [torch.empty(max(t.cols for t in w.tensors[:n]), dtype=torch.float32, device=dev) for _ in range(2)]
     cs = torch.cuda.current_stream()
     up, dn = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -434,7 +442,7 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     computed = [torch.cuda.Event() for _ in range(2)]
     act_up, q8_done, acc_read = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
     downloaded = [torch.cuda.Event() for _ in range(n)]
-    h2d = sum(h.numel() * 2 for h in host_x) + sum(h.numel() * 4 for h in host_qw) + host_act.numel() * 4
+    h2d = sum(h.numel() * 4 for h in host_x) + sum(h.numel() * 4 for h in host_qw) + host_act.numel() * 4
     d2h = sum(h.numel() for h in host_b) + host_q8.numel() + 32
 
     def one():
@@ -450,9 +458,9 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
                 uploaded[k].record(up)
             cs.wait_event(uploaded[k])
             cs.wait_event(downloaded[i])  # the previous step's copy of these blocks is done
-            iqq.iqq_quantize_qx_0_w_bf16(4, xv, qv, w.blocks[i], stream=cs)
-            iqq.iqq_dequant_rmse_qx_bf16(4, xv, w.blocks[i], qv, w.y[:t.numel].view(t.rows, t.cols), w.acc,
-                                         stream=cs)
+            iqq.iqq_quantize_q4_0_w(xv, qv, w.blocks[i], stream=cs)
+            iqq.iqq_dequant_rmse_qx(4, xv, w.blocks[i], qv, w.y[:t.numel].view(t.rows, t.cols), w.acc,
+                                    stream=cs)
             computed[k].record(cs)
             with torch.cuda.stream(dn):
                 dn.wait_event(computed[k])
@@ -492,7 +500,7 @@ def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
     elems = sum(t.numel for t in w.tensors[:n]) + w.act.numel()
     return ({"value": elems / sec / 1e9, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
              "d2h_bytes_per_step": int(d2h), "layers": layers,
-             "h2d_gb_s": round(h2d / sec / 1e9, 1), "x_dtype": "bf16 (exact: bf16-valued weights)",
+             "h2d_gb_s": round(h2d / sec / 1e9, 1), "x_dtype": "f32",
             "overlap": "copies on two streams beside the kernels"},
             sec, elems)
 
@@ -509,7 +517,7 @@ def main_ours(args):
     # the oracle pool is spawned before this process touches the GPU
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(args.cpu_seconds)
+        cpu = oracle_sample()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -545,7 +553,8 @@ def main_ours(args):
     if world > 1:
         dist.barrier()
     total_ms, phase = times[0], times[1:]
-    acc = w.acc.cpu().tolist()
+    # the round trip of every tensor quantized by every rank (the job's statistics)
+    rt = replicas.job_rmse(w.acc, w.q4_elems, device=dev)
 
     gemv = None
     if not args.no_gemv:
@@ -613,8 +622,9 @@ def main_ours(args):
                                   "hbm_frac": round(drm_gbs / pk["hbm_gbs"], 4),
                                   "kernel": "weighted_rmse_kernel<4> writing y",
                                   "bytes_per_value": DEQ_RMSE_BYTES_PER_VALUE,
-                                  "wrmse": math.sqrt(acc[0] / acc[1]) if acc[1] else None,
-                                  "rmse": math.sqrt(acc[2] / w.q4_elems), "maxerr": acc[3]},
+                                  "wrmse": rt["wrmse"], "rmse": rt["rmse"], "maxerr": rt["maxerr"],
+                                  "round_trip_values": rt["values"],
+                                  "round_trip_scope": "all ranks' tensors (accumulators reduced over ranks)"},
             "q8_k128": {"ms": round(phase[2] / K, 4), "gb_s": round(q8_gbs, 1),
                         "hbm_frac": round(q8_gbs / pk["hbm_gbs"], 4),
                         "gelem_s": round(w.q8_elems / (phase[2] / K / 1e3) / 1e9, 3)},
@@ -646,29 +656,31 @@ def main_ours(args):
 
 
 def main_reference(args):
-    """The oracle (plain single-threaded C, one process per core) as the reference arm."""
+    """The oracle (plain single-threaded C, one process per host core) as the reference arm:
+    every step is one pass over the fixed sample of the workload (ORACLE_SAMPLE_Q4_VALUES),
+    timed as in the cpu_baseline leg."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import multiprocessing as mp
-    vals, cores, sample, p = [], None, None, None
-    per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    vals, secs, cores, sample = [], [], None, None
     ncores = os.cpu_count() or 1
     with mp.get_context("spawn").Pool(ncores) as pool:
         for i in range(args.warmup + args.steps):
-            v, cores, sample, p = oracle_sample(per_step, ncores, pool)
+            v, cores, sample, _, step_s = oracle_sample(ncores, pool)
             if i >= args.warmup:
                 vals.append(v)
+                secs.append(step_s)
+    step = statistics.median(secs)
     value = statistics.median(vals)
-    from post_weight_quantization_rowwise_b200 import synth
-    full = sum(t.numel for t in synth.llama2_7b_layer_set(args.layers)) + 4096 * 7168
     out = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": round(full / (value * 1e9) * 1e3, 1),
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
            "data": "synthetic (seeded; no model weights or calibration data)",
-           "config": {"workload": WORKLOAD, "layers": args.layers}, "impl": "reference",
+           "config": {"workload": WORKLOAD, "layers": args.layers,
+                      "step": "one pass of the oracle over the fixed sample below", "sample": sample},
+           "impl": "reference",
            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -707,7 +719,6 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--e2e-layers", type=int, default=32)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")

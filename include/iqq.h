@@ -107,6 +107,18 @@ iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void* out, int64
                                uint32_t* d_flags, void* stream);
 
 /*
+ * iqq_quantize_q4_0_w_direct -- iqq_quantize_q4_0_w computed by the direct sweep: every
+ * block evaluates all 19 candidates' sequential sums (the definition above, step by step).
+ * iqq_quantize_q4_0_w reaches the same winner by placing each code step between candidates
+ * and computing exact sums only for the candidates an error bound cannot exclude; the two
+ * write identical bytes and flags.  Kept to cross-check that path on large inputs and as
+ * the reference point of its speed.  Arguments and errors as for iqq_quantize_q4_0_w.
+ */
+iqq_status iqq_quantize_q4_0_w_direct(const float* x, const float* qw, void* out, int64_t nrows,
+                                      int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                                      uint32_t* d_flags, void* stream);
+
+/*
  * iqq_quantize_qx_0_w -- the same weighted search for the other 32-value formats
  * of the family ([W] §一: the weighting appears in quantize_row_q5_0_impl,
  * quantize_row_q6_0_impl, ...): bits = 4 (Q4_0, exactly iqq_quantize_q4_0_w),

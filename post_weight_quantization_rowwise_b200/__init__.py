@@ -46,6 +46,7 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     sigs = {
         "iqq_quantize_q4_0_w": [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
+        "iqq_quantize_q4_0_w_direct": [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_quantize_q8_k128": [_vp, _vp, _i64, _i64, _vp, _vp],
         "iqq_dequant_q4_0": [_vp, _vp, _i64, _i64, _vp],
         "iqq_quantize_q8_1": [_vp, _vp, _i64, _i64, _vp, _vp, _vp],
@@ -215,6 +216,26 @@ def iqq_quantize_q4_0_w(x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, 
     _check("iqq_quantize_q4_0_w",
            _lib.iqq_quantize_q4_0_w(_ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw,
                                     weight_mode, _ptr(flags), _stream(stream)))
+    return out
+
+
+def iqq_quantize_q4_0_w_direct(x, qw, out, rows_per_qw: int = 0, weight_mode: int = 0, flags=None,
+                               stream=None):
+    """iqq_quantize_q4_0_w by the direct sweep (every candidate's exact sums): the same bytes
+    and flags, kept to cross-check the default path."""
+    import torch
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("qw", qw, torch.float32)
+    _need_cuda("out", out, torch.uint8)
+    _need_cuda("flags", flags, torch.int32)
+    nrows, n = _shape2(x)
+    _check_qw(qw, nrows, n, rows_per_qw, x.device)
+    _same_device(x, out=out, flags=flags)
+    if out.numel() < q4_0_nbytes(nrows, n):
+        raise ValueError("out is too small")
+    _check("iqq_quantize_q4_0_w_direct",
+           _lib.iqq_quantize_q4_0_w_direct(_ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw,
+                                           weight_mode, _ptr(flags), _stream(stream)))
     return out
 
 

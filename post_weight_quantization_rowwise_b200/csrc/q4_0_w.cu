@@ -1,0 +1,836 @@
+// q4_0_w.cu -- imatrix-weighted Q4_0 quantization (nmax = 8) on sm_100a with a
+// transition-based candidate sweep.
+//
+// Page "ik_llama.cpp 量化权重之谜：weight[j] = qw[j] * sqrtf(sigma2 +
+// xb[j]*xb[j])的由来与原理" (www.dpshk.com/news/4810665), §一: per row
+// sigma2 = sum_x2 / n_per_row, per 32-value block weight[j] = qw[j] *
+// sqrtf(sigma2 + xb[j]^2), then make_qx_quants(QK4_0, 8, ...): the weighted
+// least-squares scale search (sumlx = sum w*x*l, suml2 = sum w*l*l,
+// d = sumlx/suml2) and greedy code moves driven by g = d*w*(x - d*l).  The
+// candidate set, tie rule, stopping rule, rounding and byte layout are the
+// library's readings (iqq.h): iscale_k = -c_k/xmax, c_k = (float)(80+k)/10,
+// k = -9..9; l = clamp(rint(iscale_k*x), -8, 7); fmaf sums sequential over j;
+// the strictly best sumlx^2/suml2 wins (ties to the lowest k); <= 5
+// Gauss-Seidel greedy passes; final d = sumlx/suml2 -> binary16.
+//
+// The result is bit for bit that of the direct definition.  What changes is how
+// the winning candidate is found, since evaluating all 19 candidates' sequential
+// sums costs about 130 operations per value:
+//
+//  1. Magnitudes.  With a_k = fl(c_k/|xmax|), |l| = min(rint(a_k*|x|), 8 or 7) (the
+//     bound is 8 where x has the sign of xmax), because fl(-c_k/xmax) = -sign(xmax)*a_k
+//     and rounding is sign symmetric; every term w*x*l of sumlx has the sign of -xmax, so
+//     a candidate's sums are sums of nonnegative magnitudes.
+//  2. Transitions.  |l| as a function of k is a nondecreasing step function.  Per
+//     value the kernel evaluates it exactly at the first and last candidate (at
+//     most two steps lie between them for nmax = 8) and places each step at the
+//     first candidate whose code is larger, from a real-valued estimate of where
+//     a_k*|xs| crosses the rounding boundary.  An estimate closer than 2^-10 of a
+//     candidate to the boundary (exact ties included) is settled by evaluating
+//     the code there exactly.  Each step adds |w*xs| and w*(2m+1) to per-candidate
+//     difference sums.
+//  3. Filter.  Prefix sums of the differences give every candidate's sums with a
+//     relative error below (max(32, steps) + 18)*2^-24; the exact sequential sums
+//     are within 32*2^-24 of the same real values.  A candidate whose approximate
+//     score lies further below the best approximate score than the two bounds
+//     allow cannot be the exact winner, and a candidate with no step has the same
+//     sums as its predecessor, so it cannot win the tie either.  The surviving
+//     candidates (usually one) get their exact sequential sums, spread over the
+//     warp's lanes.  Blocks outside the range where the bounds hold (tiny, huge or
+//     non-finite values, empty weights) take the direct sweep.
+//
+// Work layout: a persistent grid splits the tensor's blocks, in row-major order,
+// into equal ranges of 32-block tiles, one range per CTA.  Eight consumer warps
+// take tiles from a shared counter (one block per lane); a ninth, producer, warp
+// computes each row's sigma2 (binary64 sum of exact squares) just ahead of them,
+// which also brings the rows into L2 before the consumers load their blocks.  A
+// tile may span rows; every lane finds its own row.  Rows of any width are
+// balanced to a tile per CTA, so short rows (64 blocks) and rows that are not a
+// multiple of 32 blocks (344) leave no lanes idle.  Every wait is bounded.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace iqq {
+
+namespace {
+
+constexpr int QK = IQQ_Q4_0_BLOCK_VALUES;
+constexpr int kNmax = 8;
+constexpr int kCand = 19;
+constexpr int kConsumers = 8;                   // consumer warps per CTA
+constexpr int kThreads = (kConsumers + 1) * 32; // plus one producer warp
+constexpr int kRowS = QK + 4;                   // staging row stride: 16-byte rows, LDS.128 conflict-free
+constexpr int kMaxRows = 256;                   // sigma2 rows per chunk of a CTA's range
+constexpr int kLeadRows = 4;                    // rows the producer may run ahead of the consumers
+constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kEta = 0.0009765625f;           // 2^-10: estimate closer than this to a candidate -> exact
+constexpr long long kWaitCycles = 4000000000LL; // about 2 s at 2 GHz
+
+// Per consumer warp: x and w of its 32 blocks (row per lane, stride 36), and an area
+// used in turn by the per-candidate difference sums (float2 [18][32]), the survivors'
+// exact scores (float [32]) and the codes (float [32][33]).
+struct WarpSmem {
+    float x[32 * kRowS];
+    float w[32 * kRowS];
+    union {
+        float2 diff[18 * 32];
+        float2 res[32];  // (score, k) of an exact check
+        float l[32 * kRowS];
+    } u;
+};
+constexpr size_t kDynSmem = sizeof(WarpSmem) * kConsumers;
+
+__device__ __forceinline__ float rcp_approx(float v)
+{
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ float clamp8(float r) { return fminf(fmaxf(r, -8.0f), 7.0f); }
+
+// Bounded wait until *p >= target; returns false on expiry.
+__device__ __forceinline__ bool wait_at_least(const volatile int* p, int target)
+{
+    if (*p >= target) return true;
+    const long long t0 = clock64();
+    unsigned ns = 32;
+    while (*p < target) {
+        if (clock64() - t0 > kWaitCycles) return false;
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+    }
+    return true;
+}
+
+// The exact sequential sums of the candidate iscale = a over a staged row, and its score.
+__device__ __forceinline__ float exact_score(const float* __restrict__ xr, const float* __restrict__ wr, float a)
+{
+    float s = 0.0f, t = 0.0f;
+#pragma unroll 2
+    for (int j4 = 0; j4 < QK; j4 += 4) {
+        const float4 xv4 = *reinterpret_cast<const float4*>(xr + j4);
+        const float4 wv4 = *reinterpret_cast<const float4*>(wr + j4);
+        const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+        const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float l = clamp8(rintf(__fmul_rn(a, xq[k])));
+            s = __fmaf_rn(__fmul_rn(wq[k], xq[k]), l, s);
+            t = __fmaf_rn(wq[k], __fmul_rn(l, l), t);
+        }
+    }
+    return t > 0.0f ? __fdiv_rn(__fmul_rn(s, s), t) : -INFINITY;
+}
+
+// The greedy passes of the warp's blocks that accepted a move in their first pass (bit set in
+// `pending`), from the element after that move on, one block at a time, lane j holding
+// element j.  All trial moves of a pass that precede the next accepted move see the same
+// (sumlx, suml2, score), so they are evaluated together; the lowest accepting lane is the move
+// the sequential pass accepts first.  The state then advances and the scan resumes after that
+// element: the accepted moves and every rounding are those of the sequential passes.
+__device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, float* sL, unsigned pending,
+                                            float sumlx, float suml2, float score, int gstart)
+{
+    const int lane = threadIdx.x & 31;
+    while (pending != 0u) {
+        const int bb = __ffs(pending) - 1;
+        pending &= pending - 1u;
+        float lx = __shfl_sync(kFull, sumlx, bb);
+        float l2 = __shfl_sync(kFull, suml2, bb);
+        float sc = __shfl_sync(kFull, score, bb);
+        int start = __shfl_sync(kFull, gstart, bb);
+        const float xj = sX[bb * kRowS + lane];
+        const float wj = sW[bb * kRowS + lane];
+        float lj = sL[bb * kRowS + lane];
+        const float wxj = __fmul_rn(wj, xj);
+        float d = __fdiv_rn(lx, l2);
+        int passes = 1;
+        bool changed = true;  // pass 1 accepted the move before `start`
+        for (int guard = 0; guard < 5 * (QK + 1); ++guard) {  // at most 5 passes of <= 32 moves
+            const float g = __fmul_rn(d, __fmul_rn(wj, __fsub_rn(xj, __fmul_rn(d, lj))));
+            const float sg = g > 0.0f ? 1.0f : -1.0f;
+            const float ln = __fadd_rn(lj, sg);
+            const float nlx = __fadd_rn(lx, __fmul_rn(sg, wxj));
+            const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), l2);
+            const float a2 = __fmul_rn(nlx, nlx);
+            // rejected for certain when fl(nlx^2) <= fl(fl(sc*nl2)*(1 - 2^-22)) with that bound in
+            // [1e-30, 1e30]: then nlx^2/nl2 < sc exactly, and so is its rounded quotient
+            const float thr = __fmul_rn(__fmul_rn(sc, nl2), 0.99999976158142089844f);
+            bool ok = lane >= start && (g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f &&
+                      !(a2 <= thr && thr >= 1e-30f && thr <= 1e30f);
+            float ns = 0.0f;
+            if (ok) {
+                ns = __fdiv_rn(a2, nl2);
+                ok = ns > sc;
+            }
+            const unsigned m = __ballot_sync(kFull, ok);
+            if (m == 0u) {                       // the rest of this pass accepts nothing
+                if (!changed || passes == 5) break;
+                ++passes;
+                changed = false;
+                start = 0;
+                continue;
+            }
+            const int j0 = __ffs(m) - 1;
+            if (lane == j0) lj = ln;
+            lx = __shfl_sync(kFull, nlx, j0);
+            l2 = __shfl_sync(kFull, nl2, j0);
+            sc = __shfl_sync(kFull, ns, j0);
+            d = __fdiv_rn(lx, l2);
+            changed = true;
+            start = j0 + 1;
+            if (start == QK) {                   // the pass ended on an accepted move
+                if (passes == 5) break;
+                ++passes;
+                changed = false;
+                start = 0;
+            }
+        }
+        sL[bb * kRowS + lane] = lj;
+    }
+}
+
+// The producer warp: sigma2 of rows rA .. rA+nr-1 in order, published through s_produced.
+template <typename XT>
+__device__ void produce_rows(const XT* __restrict__ x, int64_t n_per_row, int64_t rA, int nr, float* s_sig,
+                             volatile int* s_produced, const volatile int* s_consumed_row,
+                             uint32_t* __restrict__ flags)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t n4 = n_per_row / 4;
+    for (int rr = 0; rr < nr; ++rr) {
+        // stay a few rows ahead of the furthest row a grabbed tile needs, so that the rows read
+        // here are still in L2 when the consumers load their blocks (bounded: on expiry go on)
+        if (rr > kLeadRows) {
+            const long long t0 = clock64();
+            while (*s_consumed_row + kLeadRows < rr && clock64() - t0 < kWaitCycles / 4) __nanosleep(256);
+        }
+        const XT* xr = x + (rA + rr) * n_per_row;
+        // binary64 sum of exact squares; an Inf or NaN in x makes it non-finite (the square of
+        // any finite binary32 value is finite in binary64)
+        double acc = 0.0;
+        int64_t i = lane;
+        for (; i + 15 * 32 < n4; i += 16 * 32) {
+            float4 v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = iqq::ld4(xr + 4 * (i + 32 * u));
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                acc = fma(static_cast<double>(v[u].x), static_cast<double>(v[u].x), acc);
+                acc = fma(static_cast<double>(v[u].y), static_cast<double>(v[u].y), acc);
+                acc = fma(static_cast<double>(v[u].z), static_cast<double>(v[u].z), acc);
+                acc = fma(static_cast<double>(v[u].w), static_cast<double>(v[u].w), acc);
+            }
+        }
+        for (; i < n4; i += 32) {
+            const float4 v = iqq::ld4(xr + 4 * i);
+            acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
+            acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
+            acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
+            acc = fma(static_cast<double>(v.w), static_cast<double>(v.w), acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+        const bool bad = !isfinite(acc);
+        if (lane == 0) {
+            if (bad) iqq::raise_flags(flags, IQQ_FLAG_NONFINITE_INPUT);
+            s_sig[rr] = static_cast<float>(acc / static_cast<double>(n_per_row));
+            __threadfence_block();
+            *s_produced = rr + 1;
+        }
+        __syncwarp();
+    }
+}
+
+// Stages the block's 32 values of x into the lane's row: 16-byte asynchronous copies for
+// binary32 storage (no registers held while they are in flight), widened loads for bf16.
+__device__ __forceinline__ void stage_x(float* dst, const float* src)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+#pragma unroll
+    for (int i = 0; i < QK / 4; ++i)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + 16 * i), "l"(src + 4 * i) : "memory");
+}
+__device__ __forceinline__ void stage_x(float* dst, const __nv_bfloat16* src)
+{
+#pragma unroll
+    for (int i = 0; i < QK / 4; ++i) *reinterpret_cast<float4*>(dst + 4 * i) = iqq::ld4(src + 4 * i);
+}
+__device__ __forceinline__ void stage_qw(float* dst, const float* src)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+#pragma unroll
+    for (int i = 0; i < QK / 4; ++i)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(d + 16 * i), "l"(src + 4 * i) : "memory");
+}
+__device__ __forceinline__ void staged_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The step of code n -> n+1 of a value of magnitude X whose index estimate t (+0.5) lies within
+// 2^-10 of candidate ic = round(t - 0.5): it is at ic if the code there is already > n, else at
+// ic + 1 (the neighbouring candidates are far from the rounding boundary).
+__device__ __forceinline__ int exact_step(float t, float n, float X, float A, const float* s_c)
+{
+    const int ic = min(max(__float2int_rn(__fsub_rn(t, 0.5f)), 0), 19);
+    if (ic <= 0) return 1;
+    if (ic >= 18) return 18;
+    const float v = rintf(__fmul_rn(__fdiv_rn(s_c[ic], A), X));
+    return v >= __fadd_rn(n, 1.0f) ? ic : ic + 1;
+}
+
+// Adds a step n -> n+1 of a value (|w*x| = p, weight w) to the difference sums of candidate idx.
+__device__ __forceinline__ void add_step(float2* dcol, int idx, float p, float w, float n)
+{
+    float2* c = dcol + 32 * (min(max(idx, 1), 18) - 1);
+    float2 v = *c;
+    v.x = __fadd_rn(v.x, p);
+    v.y = __fmaf_rn(w, __fmaf_rn(2.0f, n, 1.0f), v.y);
+    *c = v;
+}
+
+// One tile: blocks g .. g+31 (those below gend) of the chunk whose rows start at rA.
+template <typename XT>
+__device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
+                             int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
+                             int64_t g, int64_t gend, int64_t rA, int64_t nb, const float* s_sig,
+                             const volatile int* s_produced, int* s_consumed_row, const float* s_c, WarpSmem& ws,
+                             volatile int* s_abort, uint32_t* __restrict__ flags)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t bad = 0u;
+
+    // this lane's block: its row (relative to rA) and position in the row; 32-bit arithmetic
+    // within the chunk (fewer than kMaxRows rows of nb < 2^22 blocks)
+    const int64_t gb = g + lane;
+    const bool valid = gb < gend;
+    const uint32_t nb32 = static_cast<uint32_t>(nb);
+    const uint32_t off = static_cast<uint32_t>((valid ? gb : g) - rA * nb);
+    const uint32_t rr = off / nb32;
+    const uint32_t b = off - rr * nb32;
+    const int64_t row = rA + rr;
+
+    // x and qw of the block into the lane's rows (asynchronous while the row's sigma2 is awaited)
+    float* const my_x = ws.x + lane * kRowS;
+    float* const my_w = ws.w + lane * kRowS;
+    const int64_t qrow = rows_per_qw > 0 ? row / rows_per_qw : 0;
+    const float* qb = qw != nullptr ? qw + qrow * n_per_row + static_cast<int64_t>(b) * QK : nullptr;
+    if (valid) {
+        stage_x(my_x, x + row * n_per_row + static_cast<int64_t>(b) * QK);
+        if (qb != nullptr) stage_qw(my_w, qb);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+
+    // the sigma2 of every row of the tile (every lane observes the producer's count)
+    {
+        const uint32_t last = static_cast<uint32_t>((gend < g + 32 ? gend : g + 32) - 1 - rA * nb) / nb32;
+        if (lane == 0 && static_cast<int>(last) > *s_consumed_row) atomicMax(s_consumed_row, static_cast<int>(last));
+        const bool ok = __all_sync(kFull, wait_at_least(s_produced, static_cast<int>(last) + 1));
+        if (!ok) {
+            staged_wait();
+            if (lane == 0) {
+                iqq::raise_flags(flags, IQQ_FLAG_WAIT_TIMEOUT);
+                *s_abort = 1;
+            }
+            return;
+        }
+    }
+    __threadfence_block();
+    const float sigma2 = __fmul_rn(fudge, valid ? s_sig[rr] : 0.0f);
+    staged_wait();
+
+    // the imatrix checks on the first row of each imatrix group; importance weights in place of
+    // qw (binary32, one rounding per operation): mode 0 qw*sqrt(sigma2 + x*x), 1 qw,
+    // 2 qw*(x*x), 3 qw*|x|, 4 qw*(sigma2 + x*x), 5 qw*(sqrt(sigma2) + |x|); |xmax| and xmax
+    // (the first element of largest |x|)
+    float A = 0.0f, xmax = 0.0f;
+    int jmax = 0;
+    {
+        if (!valid) {
+#pragma unroll
+            for (int i = 0; i < QK; i += 4) {
+                *reinterpret_cast<float4*>(my_x + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(my_w + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else if (qb == nullptr) {
+#pragma unroll
+            for (int i = 0; i < QK; i += 4) *reinterpret_cast<float4*>(my_w + i) = make_float4(1.f, 1.f, 1.f, 1.f);
+        } else if (rows_per_qw > 0 ? row % rows_per_qw == 0 : row == 0) {
+            float qmin = 0.0f, qnf = 0.0f;
+#pragma unroll 2
+            for (int i = 0; i < QK; i += 4) {
+                const float4 q = *reinterpret_cast<const float4*>(my_w + i);
+                qmin = fminf(fminf(qmin, fminf(q.x, q.y)), fminf(q.z, q.w));
+                qnf = __fmaf_rn(q.x, 0.0f, __fmaf_rn(q.y, 0.0f, __fmaf_rn(q.z, 0.0f, __fmaf_rn(q.w, 0.0f, qnf))));
+            }
+            if (qnf != qnf) bad |= IQQ_FLAG_NONFINITE_INPUT;
+            if (qmin < 0.0f) bad |= IQQ_FLAG_NEG_QW;
+        }
+        const float sigma = weight_mode == 5 ? __fsqrt_rn(sigma2) : 0.0f;
+#pragma unroll 1
+        for (int i = 0; i < QK; i += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(my_x + i);
+            const float4 q = *reinterpret_cast<const float4*>(my_w + i);
+            const float xq[4] = {v.x, v.y, v.z, v.w};
+            float wq[4] = {q.x, q.y, q.z, q.w};
+            if (weight_mode == 0) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    wq[k] = __fmul_rn(wq[k], __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xq[k], xq[k]))));
+            } else if (weight_mode != 1) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float xj = xq[k];
+                    const float t = __fmul_rn(xj, xj);
+                    float m;
+                    switch (weight_mode) {
+                    case 2: m = t; break;
+                    case 3: m = fabsf(xj); break;
+                    case 4: m = __fadd_rn(sigma2, t); break;
+                    default: m = __fadd_rn(sigma, fabsf(xj)); break;
+                    }
+                    wq[k] = __fmul_rn(wq[k], m);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float a = fabsf(xq[k]);
+                if (a > A) { A = a; xmax = xq[k]; jmax = i + k; }
+            }
+            *reinterpret_cast<float4*>(my_w + i) = make_float4(wq[0], wq[1], wq[2], wq[3]);
+        }
+    }
+
+    // ---------------------------------------------------------------- transitions
+    // With iscale_k = -c_k/xmax the codes are l = clamp(rint(iscale_k*x), -8, 7), and
+    // |l| = min(rint(fl(c_k/|xmax|)*|x|), 8 or 7): every term w*x*l of sumlx has the sign
+    // of -xmax, so the sums of a candidate are sums of nonnegative magnitudes.
+    const bool active = A > 0.0f;
+    float2* const dcol = ws.u.diff + lane;  // diff[i-1][lane] for candidate i = 1..18
+#pragma unroll
+    for (int i = 0; i < 18; ++i) dcol[32 * i] = make_float2(0.0f, 0.0f);
+    const float a0 = active ? __fdiv_rn(-s_c[0], xmax) : 0.0f;
+    const float a18 = active ? __fdiv_rn(-s_c[kCand - 1], xmax) : 0.0f;
+    const float kR = __fmul_rn(10.0f, A);  // 80*|xmax|/nmax: the step index scale
+    float S0 = 0.0f, T0 = 0.0f, nsteps = 0.0f;
+    uint32_t m_unc = 0u, m_two = 0u;
+#pragma unroll 1
+    for (int j4 = 0; j4 < QK; j4 += 4) {
+        const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
+        const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+        const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+        const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
+        const uint32_t bit = 1u << j4;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float xs = xq[k], w = wq[k];
+            const float p = fabsf(__fmul_rn(w, xs));
+            const float l0 = rintf(__fmul_rn(a0, xs));            // |l0| <= 7: no clamp needed
+            const float l18 = clamp8(rintf(__fmul_rn(a18, xs)));
+            const float m0 = fabsf(l0);
+            S0 = __fmaf_rn(p, m0, S0);
+            T0 = __fmaf_rn(w, __fmul_rn(m0, m0), T0);
+            const float dm = __fsub_rn(fabsf(l18), m0);          // 0, 1 or 2 steps
+            nsteps = __fadd_rn(nsteps, dm);
+            // t + 0.5, t = (m0 + 0.5)*R - 71: the (real) candidate index of the first step; the
+            // step goes to round(t + 0.5) unless t lies within 2^-10 of a candidate (then exact).
+            // Computed for every value (no branch); values without a step add zeros.
+            const float R = __fmul_rn(kR, rcp_approx(fabsf(xs)));
+            const float t = __fmaf_rn(m0, R, __fmaf_rn(0.5f, R, -70.5f));
+            const float y = __fadd_rn(t, kMagic);
+            const float dist = __fsub_rn(t, __fsub_rn(y, kMagic));
+            // candidate index - 1, clamped to [0, 17] (memory safety for any input)
+            const uint32_t i1 = min(__float_as_uint(y) - (__float_as_uint(kMagic) + 1u), 17u);
+            const bool step = dm > 0.5f;
+            const bool sure = step && fabsf(dist) < 0.5f - kEta;
+            float2* c = dcol + 32 * i1;
+            float2 v = *c;
+            v.x = __fadd_rn(v.x, p);
+            v.y = __fmaf_rn(w, __fmaf_rn(2.0f, m0, 1.0f), v.y);
+            if (sure) *c = v;
+            if (step && !sure) m_unc |= bit << k;
+            if (dm > 1.5f) m_two |= bit << k;
+        }
+    }
+    // The first largest element (|x| = |xmax|) always has one step, 7 -> 8, and it lies on a
+    // rounding tie: at candidate 4 (c = 7.5) when fl(fl(7.5/|xmax|)*|xmax|) >= 7.5 (rint
+    // rounds 7.5 to 8), else at candidate 5.  It is placed here, per block, rather than
+    // among the uncertain steps below.
+    if (active && ((m_unc >> jmax) & 1u)) {
+        const float v4 = __fmul_rn(__fdiv_rn(s_c[4], A), A);
+        const float w = my_w[jmax];
+        float2* c = dcol + 32 * (v4 >= 7.5f ? 3 : 4);
+        float2 v = *c;
+        v.x = __fadd_rn(v.x, fabsf(__fmul_rn(w, xmax)));
+        v.y = __fmaf_rn(w, 15.0f, v.y);
+        *c = v;
+        m_unc &= ~(1u << jmax);
+    }
+    // the other uncertain first steps, then the second steps, per lane from the staged row
+    {
+        uint32_t todo = m_unc;
+        while (todo != 0u) {
+            const int j = __ffs(todo) - 1;
+            todo &= todo - 1u;
+            const float xs = my_x[j], w = my_w[j];
+            const float X = fabsf(xs);
+            const float m0 = fabsf(rintf(__fmul_rn(a0, xs)));
+            const float R = __fmul_rn(kR, rcp_approx(X));
+            const float t = __fmaf_rn(m0, R, __fmaf_rn(0.5f, R, -70.5f));  // as in the loop above
+            add_step(dcol, exact_step(t, m0, X, A, s_c), fabsf(__fmul_rn(w, xs)), w, m0);
+        }
+        todo = m_two;
+        while (todo != 0u) {
+            const int j = __ffs(todo) - 1;
+            todo &= todo - 1u;
+            const float xs = my_x[j], w = my_w[j];
+            const float X = fabsf(xs);
+            const float m0 = fabsf(rintf(__fmul_rn(a0, xs)));
+            const float R = __fmul_rn(kR, rcp_approx(X));
+            const float t = __fadd_rn(__fmaf_rn(m0, R, __fmaf_rn(0.5f, R, -70.5f)), R);  // second step
+            const float n = __fadd_rn(m0, 1.0f);
+            const float y = __fadd_rn(t, kMagic);
+            const float dist = __fsub_rn(t, __fsub_rn(y, kMagic));
+            int idx = static_cast<int>(__float_as_uint(y) - __float_as_uint(kMagic));
+            if (!(fabsf(dist) < 0.5f - kEta && idx >= 1 && idx <= 18)) idx = exact_step(t, n, X, A, s_c);
+            add_step(dcol, idx, fabsf(__fmul_rn(w, xs)), w, n);
+        }
+    }
+
+    // ---------------------------------------------------------------- approximate scores
+    // Prefix sums of the differences; candidate i's approximate score replaces its (consumed)
+    // difference sums.  A candidate with no step has its predecessor's sums: dominated (it
+    // cannot win the tie).
+    uint32_t dom = 0u;
+    float S = S0, T = T0;
+    float mx = __fmul_rn(__fmul_rn(S, S), rcp_approx(T));
+    const float sc0 = mx;
+#pragma unroll 2
+    for (int i = 1; i < kCand; ++i) {
+        float2* c = dcol + 32 * (i - 1);
+        const float2 v = *c;
+        if (v.x == 0.0f && v.y == 0.0f) dom |= 1u << i;
+        S = __fadd_rn(S, v.x);
+        T = __fadd_rn(T, v.y);
+        const float sci = __fmul_rn(__fmul_rn(S, S), rcp_approx(T));
+        c->x = sci;
+        mx = fmaxf(mx, sci);
+    }
+    // bounds: |approx - real| <= (max(32, steps) + 18) u per sum, exact sums within 32 u,
+    // 6 u for the approximate quotient, 2 u for the exact one (u = 2^-24)
+    const bool regular = active && A >= 0x1p-100f && A <= 0x1p100f && S0 >= 0x1p-50f && T0 >= 0x1p-50f &&
+                         S <= 0x1p50f && T <= 0x1p50f && mx >= 0x1p-100f && mx <= 0x1p100f;
+    uint32_t surv = 0u;
+    {
+        const float nr = __fadd_rn(fmaxf(nsteps, 32.0f), 18.0f);
+        const float margin = __fmul_rn(__fmaf_rn(6.0f, nr, 256.0f), 0x1p-24f);  // 2*(3 nr + 6 + 98 + 24 slack) u
+        const float thr = __fmul_rn(mx, __fsub_rn(1.0f, margin));
+        if (sc0 >= thr) surv = 1u;
+#pragma unroll 3
+        for (int i = 1; i < kCand; ++i)
+            if (!((dom >> i) & 1u) && dcol[32 * (i - 1)].x >= thr) surv |= 1u << i;
+    }
+    // blocks outside the bounds: every candidate gets its exact sums (the direct sweep)
+    if (!regular) surv = active ? (1u << kCand) - 1u : 0u;
+    __syncwarp();  // the difference sums are read: the area now holds the survivors' scores
+
+    // ---------------------------------------------------------------- exact winner
+    int kbest = surv != 0u ? __ffs(surv) - 1 : 0;
+    float best = -INFINITY;
+    {
+        const int cnt = __popc(surv);
+        const int need = cnt >= 2 ? cnt : 0;
+        // exclusive prefix of need over the warp
+        int start = need;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFull, start, o);
+            if (lane >= o) start += v;
+        }
+        const int total = __shfl_sync(kFull, start, 31);
+        start -= need;
+        for (int base = 0; base < total; base += 32) {  // warp-uniform
+            const int q = base + lane;
+            // owner: the last lane whose range starts at or before q
+            int lo = 0;
+#pragma unroll
+            for (int step = 16; step > 0; step >>= 1) {
+                const int s = __shfl_sync(kFull, start, lo + step);
+                if (s <= q) lo += step;
+            }
+            const int owner = lo;
+            const int ostart = __shfl_sync(kFull, start, owner);
+            const uint32_t osurv = __shfl_sync(kFull, surv, owner);
+            const float oxmax = __shfl_sync(kFull, xmax, owner);
+            float r = -INFINITY;
+            int kk = 0;
+            if (q < total) {
+                kk = static_cast<int>(min(__fns(osurv, 0, q - ostart + 1), static_cast<unsigned>(kCand - 1)));
+                r = exact_score(ws.x + owner * kRowS, ws.w + owner * kRowS, __fdiv_rn(-s_c[kk], oxmax));
+            }
+            ws.u.res[lane] = make_float2(r, __int_as_float(kk));
+            __syncwarp();
+            if (need > 0) {
+                // this lane's items of the round, in increasing k: strictly better wins
+                const int q0 = max(start, base), q1 = min(start + need, base + 32);
+                for (int qq = q0; qq < q1; ++qq) {
+                    const float2 e = ws.u.res[qq - base];
+                    if (e.x > best) {
+                        best = e.x;
+                        kbest = __float_as_int(e.y);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+    __syncwarp();  // the area now holds the codes
+
+    // ---------------------------------------------------------------- codes and greedy state
+    // mode 0: nothing to search (all-zero block or no block), 1: no candidate with positive
+    // weighted code energy (codes of iscale = -nmax/xmax, d = 1/iscale), 2: search
+    int mode = 0;
+    float* const my_l = ws.u.l + lane * kRowS;
+    float sumlx = 0.0f, suml2 = 0.0f, score = 0.0f, dfb = 0.0f;
+    {
+        float a = 0.0f;
+        if (active) {
+            if (!regular && best == -INFINITY) {
+                a = __fdiv_rn(static_cast<float>(-kNmax), xmax);
+                dfb = __fdiv_rn(1.0f, a);
+                mode = 1;
+            } else {
+                a = __fdiv_rn(-s_c[kbest], xmax);
+                mode = 2;
+            }
+        }
+#pragma unroll 1
+        for (int j4 = 0; j4 < QK; j4 += 4) {
+            const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
+            const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+            const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+            const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
+            float lq[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                lq[k] = clamp8(rintf(__fmul_rn(a, xq[k])));
+                sumlx = __fmaf_rn(__fmul_rn(wq[k], xq[k]), lq[k], sumlx);
+                suml2 = __fmaf_rn(wq[k], __fmul_rn(lq[k], lq[k]), suml2);
+            }
+            *reinterpret_cast<float4*>(my_l + j4) = make_float4(lq[0], lq[1], lq[2], lq[3]);
+        }
+        if (mode == 2) score = __fdiv_rn(__fmul_rn(sumlx, sumlx), suml2);
+    }
+
+    // greedy pass 1, this lane's block.  Until the first accepted move the state (sumlx =
+    // S, suml2 = T, score, d) is that of the sweep, so every element's trial can be screened
+    // against it at once.  With r = x/d - l and eps = w (x/d)^2 / T (d = S/T), the trial at
+    // an element raises the score (in real arithmetic) by (w/T')(2|r| - 1 + eps) relative,
+    // and the binary32 comparison cannot accept it unless that exceeds -7u (u = 2^-24):
+    // so it is rejected for certain when w (1 - 2|r| - eps) >= 7u (T + 17 w).  Evaluated
+    // with r, eps from q = fl(x * fl(T/S)) (error below 65u in 1 - 2|r| - eps while
+    // |q| < 8.5) as fl(w * fl(fl(1 - 2^-15 - 2|r|) - eps)) >= 2^-20 T.  The elements not
+    // excluded are tried exactly, in order; at the first accepted move the block is handed
+    // to the warp-cooperative passes, which continue from the next element.
+    bool changed = false;
+    int gstart = 0;
+    if (mode == 2) {
+        const float D = __fdiv_rn(suml2, sumlx), invT = __fdiv_rn(1.0f, suml2);
+        const float thr = __fmul_rn(suml2, 0x1p-20f);
+        uint32_t maybe = 0u;
+#pragma unroll 1
+        for (int j4 = 0; j4 < QK; j4 += 4) {
+            const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
+            const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+            const float4 lv4 = *reinterpret_cast<const float4*>(my_l + j4);
+            const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+            const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
+            const float lq[4] = {lv4.x, lv4.y, lv4.z, lv4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float q = __fmul_rn(xq[k], D);
+                const float r = __fsub_rn(q, lq[k]);
+                const float eps = __fmul_rn(__fmul_rn(wq[k], __fmul_rn(q, q)), invT);
+                const float b = __fsub_rn(__fmaf_rn(-2.0f, fabsf(r), 1.0f - 0x1p-15f), eps);
+                const bool sure_reject = __fmul_rn(wq[k], b) >= thr;
+                maybe |= static_cast<uint32_t>(!sure_reject) << (j4 + k);
+            }
+        }
+        float d = __fdiv_rn(sumlx, suml2);
+        while (maybe != 0u) {
+            const int j = __ffs(maybe) - 1;
+            maybe &= maybe - 1u;
+            const float xj = my_x[j], wj = my_w[j], lj = my_l[j];
+            const float g = __fmul_rn(d, __fmul_rn(wj, __fsub_rn(xj, __fmul_rn(d, lj))));
+            const float sg = g > 0.0f ? 1.0f : -1.0f;
+            const float ln = __fadd_rn(lj, sg);
+            if (!(g > 0.0f || g < 0.0f) || ln < -8.0f || ln > 7.0f) continue;
+            const float nlx = __fadd_rn(sumlx, __fmul_rn(sg, __fmul_rn(wj, xj)));
+            const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), suml2);
+            if (!(nl2 > 0.0f)) continue;
+            const float ns = __fdiv_rn(__fmul_rn(nlx, nlx), nl2);
+            if (ns > score) {
+                my_l[j] = ln;
+                sumlx = nlx;
+                suml2 = nl2;
+                score = ns;
+                changed = true;
+                gstart = j + 1;
+                break;
+            }
+        }
+    }
+    const unsigned pending = __ballot_sync(kFull, changed);
+    if (pending != 0u) {
+        __syncwarp();
+        greedy_rest(ws.x, ws.w, ws.u.l, pending, sumlx, suml2, score, gstart);
+    }
+    __syncwarp();
+
+    // ---------------------------------------------------------------- final scale and block
+    uint16_t d16 = 0;
+    {
+        float d = dfb;
+        if (mode == 2) {
+            float sfx = 0.0f, sf2 = 0.0f;
+#pragma unroll 1
+            for (int j4 = 0; j4 < QK; j4 += 4) {
+                const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
+                const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+                const float4 lv4 = *reinterpret_cast<const float4*>(my_l + j4);
+                const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+                const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
+                const float lq[4] = {lv4.x, lv4.y, lv4.z, lv4.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    sfx = __fmaf_rn(__fmul_rn(wq[k], xq[k]), lq[k], sfx);
+                    sf2 = __fmaf_rn(wq[k], __fmul_rn(lq[k], lq[k]), sf2);
+                }
+            }
+            d = __fdiv_rn(sfx, sf2);
+        }
+        if (mode != 0) {
+            d16 = __half_as_ushort(__float2half_rn(d));
+            if ((d16 & 0x7fffu) == 0x7c00u && isfinite(d)) bad |= IQQ_FLAG_SCALE_OVERFLOW;
+        }
+    }
+    if (valid) {
+        uint16_t* o16 = reinterpret_cast<uint16_t*>(out + (row * nb + b) * IQQ_Q4_0_BLOCK_BYTES);
+        o16[0] = d16;
+        // biased code n = l + 8: the low byte of (l + 8 + 1.5*2^23)
+#pragma unroll 2
+        for (int i = 0; i < QK / 4; ++i) {
+            const uint32_t n0 = __float_as_uint(__fadd_rn(my_l[2 * i], kMagic + 8.0f)) & 15u;
+            const uint32_t n1 = __float_as_uint(__fadd_rn(my_l[2 * i + 1], kMagic + 8.0f)) & 15u;
+            const uint32_t n2 = __float_as_uint(__fadd_rn(my_l[2 * i + 16], kMagic + 8.0f)) & 15u;
+            const uint32_t n3 = __float_as_uint(__fadd_rn(my_l[2 * i + 17], kMagic + 8.0f)) & 15u;
+            o16[1 + i] = static_cast<uint16_t>(n0 | (n2 << 4) | (n1 << 8) | (n3 << 12));
+        }
+    }
+    iqq::raise_flags(flags, bad);
+    __syncwarp();  // the warp's shared memory is rewritten by the next tile
+}
+
+template <typename XT>
+__global__ void __maxnreg__(96)  // 2 CTAs of 288 threads per SM (at most 5 warps of an SMSP's 16K registers)
+q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out, int64_t nrows,
+              int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* __restrict__ flags)
+{
+    extern __shared__ float4 smem4[];
+    WarpSmem* const wsm = reinterpret_cast<WarpSmem*>(smem4);
+    __shared__ float s_sig[kMaxRows];
+    __shared__ float s_c[kCand];
+    __shared__ int s_produced, s_next, s_consumed_row, s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nb = n_per_row / QK;
+    const int64_t total = nrows * nb;
+    const int64_t tiles = (total + 31) / 32;
+    // this CTA's tiles: an equal share (+-1) of the tensor's
+    const int64_t per = tiles / gridDim.x, extra = tiles % gridDim.x;
+    const int64_t t0 = blockIdx.x * per + min(static_cast<int64_t>(blockIdx.x), extra);
+    const int64_t t1 = t0 + per + (static_cast<int64_t>(blockIdx.x) < extra ? 1 : 0);
+    if (threadIdx.x < kCand) s_c[threadIdx.x] = __fdiv_rn(static_cast<float>(kNmax * (71 + threadIdx.x)), 80.0f);
+    if (threadIdx.x == 0) s_abort = 0;
+    int64_t g = t0 * 32;
+    const int64_t gend = t1 * 32 < total ? t1 * 32 : total;
+    while (g < gend) {
+        // a chunk of whole tiles touching at most kMaxRows rows
+        const int64_t rA = g / nb;
+        int64_t gB = (rA + kMaxRows) * nb / 32 * 32;
+        if (gB > gend) gB = gend;
+        const int nr = static_cast<int>((gB - 1) / nb - rA + 1);
+        __syncthreads();  // every warp is done with the previous chunk
+        if (threadIdx.x == 0) {
+            s_produced = 0;
+            s_next = 0;
+            s_consumed_row = 0;
+        }
+        __syncthreads();
+        if (warp == kConsumers) {
+            produce_rows<XT>(x, n_per_row, rA, nr, s_sig, &s_produced, &s_consumed_row, flags);
+        } else {
+            WarpSmem& ws = wsm[warp];
+            while (true) {
+                int t = 0;
+                if (lane == 0) t = atomicAdd(&s_next, 1);
+                t = __shfl_sync(kFull, t, 0);
+                const int64_t gt = g + static_cast<int64_t>(t) * 32;
+                if (gt >= gB || *reinterpret_cast<volatile int*>(&s_abort) != 0) break;
+                consume_tile<XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, gt, gB, rA, nb,
+                                 s_sig, &s_produced, &s_consumed_row, s_c, ws, &s_abort, flags);
+            }
+        }
+        g = gB;
+    }
+}
+
+template <typename XT>
+iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                  int weight_mode, float fudge, uint32_t* d_flags, void* stream)
+{
+    static thread_local int configured_device = -1;
+    static thread_local int grid_cap = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return iqq::launch_status();
+    if (configured_device != dev) {
+        if (cudaFuncSetAttribute(q4_0_w_kernel<XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kDynSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(q4_0_w_kernel<XT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            return iqq::launch_status();
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return iqq::launch_status();
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, q4_0_w_kernel<XT>, kThreads, kDynSmem) !=
+            cudaSuccess)
+            return iqq::launch_status();
+        grid_cap = sms * (per_sm > 0 ? per_sm : 1);
+        configured_device = dev;
+    }
+    const int64_t tiles = (nrows * (n_per_row / QK) + 31) / 32;
+    const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
+    q4_0_w_kernel<XT><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
+        x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags);
+    return iqq::launch_status();
+}
+
+}  // namespace
+
+// Whether the kernel above serves a tensor of this width: rows of fewer than 2^22 blocks (the
+// chunk arithmetic is 32-bit).
+bool q4_0_w_fits(int64_t n_per_row) { return n_per_row / QK < (int64_t(1) << 22); }
+
+iqq_status launch_q4_0_w(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
+                         int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream)
+{
+    return launch<float>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
+}
+
+iqq_status launch_q4_0_w(const __nv_bfloat16* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
+                         int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream)
+{
+    return launch<__nv_bfloat16>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
+}
+
+}  // namespace iqq

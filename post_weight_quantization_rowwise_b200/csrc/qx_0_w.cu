@@ -730,7 +730,7 @@ template <typename XT>
 iqq_status quantize_qx(int bits, const XT* x, const float* qw, void* out, int64_t nrows,
                        int64_t n_per_row, int64_t rows_per_qw, int weight_mode, void* workspace,
                        uint32_t* d_flags, void* stream, double* acc = nullptr, float* y_out = nullptr,
-                       float fudge = 1.0f)
+                       float fudge = 1.0f, bool direct = false)
 {
     if (bits != 4 && bits != 5 && bits != 6 && bits != 8) return IQQ_ERR_ARG;
     if (!iqq::size_ok(nrows, n_per_row, 4) || rows_per_qw < 0) return IQQ_ERR_SHAPE;
@@ -741,6 +741,10 @@ iqq_status quantize_qx(int bits, const XT* x, const float* qw, void* out, int64_
     if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||
         (d_flags && !iqq::aligned(d_flags, 4)))
         return IQQ_ERR_ALIGN;
+    // Q4_0 without the epilogue outputs: the transition-based sweep (q4_0_w.cu), which
+    // computes each row's sigma2 itself and needs no workspace
+    if (bits == 4 && !direct && acc == nullptr && y_out == nullptr && iqq::q4_0_w_fits(n_per_row))
+        return iqq::launch_q4_0_w(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
     const float* rs = nullptr;
     if (workspace != nullptr && workspace_bytes_for(nrows, n_per_row) > 0) {
         float* ws = static_cast<float*>(workspace);
@@ -766,6 +770,14 @@ extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void*
                                           uint32_t* d_flags, void* stream)
 {
     return quantize_qx(4, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, nullptr, d_flags, stream);
+}
+
+extern "C" iqq_status iqq_quantize_q4_0_w_direct(const float* x, const float* qw, void* out, int64_t nrows,
+                                                 int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
+                                                 uint32_t* d_flags, void* stream)
+{
+    return quantize_qx(4, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, nullptr, d_flags, stream, nullptr,
+                       nullptr, 1.0f, true);
 }
 
 extern "C" iqq_status iqq_quantize_qx_0_w(int bits, const float* x, const float* qw, void* out,

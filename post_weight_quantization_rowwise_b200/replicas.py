@@ -12,7 +12,9 @@ does cross ranks is bookkeeping:
   a rate is all ranks' work over the slowest rank's time;
 * ``reduce_rmse``: the weighted-RMSE accumulators of all ranks combined
   (sums added, ``max|e|`` maxed), so that one tensor set split over ranks gives
-  the same statistics as on one rank (up to binary64 rounding order).
+  the same statistics as on one rank (up to binary64 rounding order);
+* ``job_rmse``: the job's round-trip statistics from every rank's accumulator and
+  value count (what the benchmark reports for several GPUs).
 
 The functions take an initialised ``torch.distributed`` process group (NCCL on
 GPUs, gloo on CPU) or work on one process when none is initialised.
@@ -86,3 +88,15 @@ def wrmse(acc) -> float:
     """sqrt(sum qw e^2 / sum qw) of an accumulator."""
     a = [float(v) for v in acc[:2]]
     return (a[0] / a[1]) ** 0.5 if a[1] > 0 else float("nan")
+
+
+def job_rmse(acc, values, device=None) -> dict:
+    """The round-trip statistics of the whole job: every rank passes its accumulator
+    [sum qw e^2, sum qw, sum e^2, max|e|] and the number of values it scored; every rank
+    gets {wrmse, rmse, maxerr, values} of all ranks together (a collective when a process
+    group is initialised: every rank must call it)."""
+    total = reduce_rmse(acc)
+    n = sum_over_ranks([values], device=device)[0]
+    a = [float(v) for v in total]
+    return {"wrmse": (a[0] / a[1]) ** 0.5 if a[1] > 0 else float("nan"),
+            "rmse": (a[2] / n) ** 0.5 if n > 0 else float("nan"), "maxerr": a[3], "values": int(n)}

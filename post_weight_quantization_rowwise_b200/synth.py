@@ -8,10 +8,10 @@ the caller names; the same (seed, device) always gives the same bytes.
 Recipes (no model weights or calibration text exist here; these stand in for
 the tensors the pages discuss):
 
-* weight matrix: N(0, sigma) entries with a Bernoulli(outlier_frac) mask whose
-  entries are replaced by ``outlier_scale * t(3)`` (Student t with 3 degrees of
-  freedom, built as z / sqrt(chi2_3 / 3) from four standard normals), then
-  optionally every entry rounded to bf16 (a bf16 checkpoint's values);
+* weight matrix: N(0, sigma) entries, optionally rounded to bf16 (the values a bf16
+  checkpoint holds), then a Bernoulli(outlier_frac) mask whose entries are replaced
+  by binary32 ``outlier_scale * t(3)`` values (Student t with 3 degrees of freedom,
+  built as z / sqrt(chi2_3 / 3) from four standard normals);
 * imatrix row: qw = exp(N(0, 1)) per column (log-normal), optionally with a
   random ``boost_frac`` of the columns multiplied by ``boost``;
 * activations: N(0, 1) with a Bernoulli(spike_frac) mask set to
@@ -39,19 +39,19 @@ def _student_t3(n: int, g: torch.Generator, device) -> torch.Tensor:
 def weight_matrix(rows: int, cols: int, seed: int, sigma: float = 0.02,
                   outlier_frac: float = 1e-3, outlier_scale: float = 0.2,
                   bf16: bool = False, device="cpu") -> torch.Tensor:
-    """float32 [rows, cols]: N(0, sigma) with t(3) outliers; with bf16, every entry (the
-    outliers too, as in a bf16 checkpoint) is then rounded to bf16, so the tensor is
-    exactly representable in bf16."""
+    """float32 [rows, cols]: N(0, sigma) with t(3) outliers.  With bf16 the N(0, sigma) body is
+    rounded to bf16 first and the outliers, added after, stay binary32: fp32 weights taken from
+    a bf16 checkpoint, plus outliers."""
     g = _gen(seed, device)
     x = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32)
     x.mul_(sigma)
+    if bf16:
+        x = x.to(torch.bfloat16).to(torch.float32)
     if outlier_frac > 0 and rows * cols > 0:
         mask = torch.rand(rows, cols, generator=g, device=device) < outlier_frac
         k = int(mask.sum().item())
         if k:
             x[mask] = outlier_scale * _student_t3(k, g, device)
-    if bf16:
-        x = x.to(torch.bfloat16).to(torch.float32)
     return x
 
 
@@ -122,7 +122,7 @@ LLAMA2_7B_TENSORS = (  # name, rows (output features), cols (n_per_row)
 
 def llama2_7b_layer_set(layers: int = 32) -> list[Tensor2D]:
     """Llama-2-7B-shaped weights: per layer q/k/v/o 4096x4096, gate/up 11008x4096,
-    down 4096x11008; N(0, 0.02) plus 0.1% 0.2*t(3) outliers, all rounded to bf16;
+    down 4096x11008; fp32 from bf16 N(0, 0.02), plus 0.1% binary32 0.2*t(3) outliers;
     seed = 3000 + 10*layer + tensor index."""
     out = []
     for layer in range(layers):

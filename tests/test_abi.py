@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
               "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
               "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch",
               "iqq_quantize_qx_0_w_ex", "iqq_dequant_rmse_qx", "iqq_quantize_qx_0_w_bf16",
-              "iqq_dequant_rmse_qx_bf16"):
+              "iqq_dequant_rmse_qx_bf16", "iqq_quantize_q4_0_w_direct"):
         assert n in names
 
 

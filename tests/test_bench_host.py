@@ -46,8 +46,8 @@ def test_warmup_below_three_is_refused():
 
 
 def test_reference_arm_prints_one_json_line():
-    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
-                        "--cpu-seconds", "1"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     line = json.loads(r.stdout.strip().splitlines()[-1])
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
@@ -62,7 +62,7 @@ def test_reference_arm_other_ranks_exit_quietly():
     without work or output."""
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
-                        "--warmup", "3", "--cpu-seconds", "1"], cwd=ROOT, capture_output=True, text=True,
+                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True,
                        timeout=300, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""

@@ -45,7 +45,9 @@ def _worker(rank, world, port, out):
             acc[:3] += torch.from_numpy(part[:3])
             acc[3] = max(float(acc[3]), float(part[3]))
         total = replicas.reduce_rmse(acc)
-        out[rank] = (mx, total.tolist(), tot)
+        n_mine = sum(t.numel for t in replicas.shard(tensors, rank, world))
+        stats = replicas.job_rmse(acc, n_mine)  # what bench.py reports for several GPUs
+        out[rank] = (mx, total.tolist(), tot, stats)
     finally:
         dist.destroy_process_group()
 
@@ -79,8 +81,12 @@ def test_two_gloo_ranks_combine_like_one_process():
         qw = t.qw().numpy()
         blocks, _ = oracle.quantize_q4_0_w(x, qw)
         oracle.weighted_rmse(x, blocks, qw, acc=ref)
+    n_all = sum(t.numel for t in tensors)
     for rank in range(world):
-        mx, total, tot = out[rank]
+        mx, total, tot, stats = out[rank]
+        assert stats["values"] == n_all
+        assert abs(stats["wrmse"] - np.sqrt(ref[0] / ref[1])) < 1e-12
+        assert abs(stats["rmse"] - np.sqrt(ref[2] / n_all)) < 1e-12 and stats["maxerr"] == ref[3]
         assert mx == [2.0, 5.0]
         assert tot == [3.0, 2.0 ** 41 + 1]
         assert np.allclose(total[:3], ref[:3], rtol=1e-12, atol=0)

@@ -1,8 +1,9 @@
 """The seeded input recipe (host only): the properties the workloads are stated to have.
 
-The end-to-end leg of the benchmark uploads the layer set's weights as bf16, which is only
-the same workload if every entry (outliers included) is a bf16 value; the other checks pin
-the recipe's shapes, fractions and ranges, and that a seed always gives the same bytes.
+The Llama-2-7B-shaped layer set is fp32 from a bf16 N(0, 0.02) body plus binary32 t(3)
+outliers: the body entries are bf16 values, the outliers in general are not.  The other
+checks pin the recipe's shapes, fractions and ranges, and that a seed always gives the
+same bytes.
 """
 import numpy as np
 import torch
@@ -18,12 +19,20 @@ def test_same_seed_same_bytes_and_different_seeds_differ():
     assert torch.equal(synth.activations(2, 256, seed=2), synth.activations(2, 256, seed=2))
 
 
-def test_bf16_weights_are_exactly_bf16_values_outliers_included():
+def test_bf16_body_with_binary32_outliers():
     x = synth.weight_matrix(256, 4096, seed=3000, bf16=True)
-    assert torch.equal(x.to(torch.bfloat16).to(torch.float32), x)
-    # the outliers (0.2 * t(3)) are there: N(0, 0.02) alone stays far below 0.15
+    y = synth.weight_matrix(256, 4096, seed=3000, bf16=False)
+    out = x != y.to(torch.bfloat16).to(torch.float32)
+    # the outliers (0.2 * t(3)) are there, at the same places and with the same binary32
+    # values as without the rounding: N(0, 0.02) alone stays far below 0.15
     big = (x.abs() > 0.15).sum().item()
     assert 0.0002 * x.numel() < big < 0.002 * x.numel()
+    assert torch.equal(x[out], y[out])
+    assert 0.0005 * x.numel() < out.sum().item() < 0.0015 * x.numel()
+    # every other entry is a bf16 value; most outliers are not
+    body = ~out
+    assert torch.equal(x[body].to(torch.bfloat16).to(torch.float32), x[body])
+    assert (x[out].to(torch.bfloat16).to(torch.float32) != x[out]).float().mean() > 0.9
     t = synth.llama2_7b_layer_set(1)
     assert [(u.rows, u.cols) for u in t] == [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
     assert all(u.bf16 for u in t)
