@@ -527,9 +527,10 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         const float margin = __fmul_rn(__fmaf_rn(6.0f, nr, 256.0f), 0x1p-24f);  // 2*(3 nr + 6 + 98 + 24 slack) u
         const float thr = __fmul_rn(mx, __fsub_rn(1.0f, margin));
         if (sc0 >= thr) surv = 1u;
-#pragma unroll 3
+#pragma unroll
         for (int i = 1; i < kCand; ++i)
-            if (!((dom >> i) & 1u) && dcol[32 * (i - 1)].x >= thr) surv |= 1u << i;
+            if (dcol[32 * (i - 1)].x >= thr) surv |= 1u << i;
+        surv &= ~dom;
     }
     // blocks outside the bounds: every candidate gets its exact sums (the direct sweep)
     if (!regular) surv = active ? (1u << kCand) - 1u : 0u;
@@ -629,14 +630,16 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     // an element raises the score (in real arithmetic) by (w/T')(2|r| - 1 + eps) relative,
     // and the binary32 comparison cannot accept it unless that exceeds -7u (u = 2^-24):
     // so it is rejected for certain when w (1 - 2|r| - eps) >= 7u (T + 17 w).  Evaluated
-    // with r, eps from q = fl(x * fl(T/S)) (error below 65u in 1 - 2|r| - eps while
-    // |q| < 8.5) as fl(w * fl(fl(1 - 2^-15 - 2|r|) - eps)) >= 2^-20 T.  The elements not
-    // excluded are tried exactly, in order; at the first accepted move the block is handed
-    // to the warp-cooperative passes, which continue from the next element.
+    // with r, eps from q = fl(x * D), D = T/S and 1/T to within 3u (approximate reciprocals;
+    // error below 100u in 1 - 2|r| - eps while |q| < 8.5) as
+    // fl(w * fl(fl(1 - 2^-15 - 2|r|) - eps)) >= 2^-20 T.  The elements not excluded are tried
+    // exactly, in order; at the first accepted move the block is handed to the
+    // warp-cooperative passes, which continue from the next element.
     bool changed = false;
     int gstart = 0;
     if (mode == 2) {
-        const float D = __fdiv_rn(suml2, sumlx), invT = __fdiv_rn(1.0f, suml2);
+        const float invT = rcp_approx(suml2);
+        const float D = __fmul_rn(suml2, rcp_approx(sumlx));
         const float thr = __fmul_rn(suml2, 0x1p-20f);
         uint32_t maybe = 0u;
 #pragma unroll 1
