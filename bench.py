@@ -45,10 +45,10 @@ Q8_BYTES_PER_VALUE = 4.0 + 140.0 / 128.0
 DEQ_RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0 + 4.0  # read x and the blocks, write y
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
-# DRAM bytes (read + write) per value of qx_0_w_kernel<4> from one ncu capture of the current
-# kernel (4096x4096 launch: see the qx_0_w_kernel profile summary, 4.097 B per value); set
-# to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = 4.0975
+# DRAM bytes (read + write) per value of q4_0_w_kernel<float> from one ncu capture of the
+# current kernel (a 4096x4096 launch of the layer set: see the q4_0_w_kernel profile summary);
+# set to None whenever the kernel changes until it is captured again.
+Q4_0_DRAM_BYTES_PER_VALUE = 4.1013
 
 
 def peaks():
@@ -383,10 +383,9 @@ def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
             qms = _timed(lambda: iqq.iqq_quantize_qx_0_w_ws(4, x, qw, blocks, ws, 0, mode), reps=2)
             a = iqq.weighted_rmse(x, blocks, qw).cpu().tolist()
             row[name] = {"gelem_s": round(x.numel() / qms / 1e6, 3), "wrmse": math.sqrt(a[0] / a[1])}
-        if nws:
-            # the same tensor without the workspace (the fused per-CTA row reduction)
-            qms = _timed(lambda: iqq.iqq_quantize_q4_0_w(x, qw, blocks, 0, 0), reps=2)
-            row["qw_sqrt_s2_x2_fused"] = {"gelem_s": round(x.numel() / qms / 1e6, 3)}
+        # the direct sweep (every candidate's exact sums) on the same tensor, for comparison
+        qms = _timed(lambda: iqq.iqq_quantize_q4_0_w_direct(x, qw, blocks, 0, 0), reps=2)
+        row["qw_sqrt_s2_x2_direct_sweep"] = {"gelem_s": round(x.numel() / qms / 1e6, 3)}
         ab[tt.name] = row
         del x, qw, blocks, ws
     out["sweep_ab"] = ab
@@ -407,6 +406,51 @@ def run_extras(iqq, dev, p_mean: float, peak_ops: float, hbm_gbs: float):
                    "q8_1_gb_s": round(na * (4 + 36 / 32) / m1 / 1e6, 1),
                    "q8_k128_gb_s": round(na * (4 + 140 / 128) / mk / 1e6, 1)}
     return out
+
+
+def run_moe(iqq, dev, peak_ops: float, p_mean: float, experts: int = 256):
+    """DeepSeek-shaped MoE expert tensors (gate/up 2048x7168, down 7168x2048, N(0, 0.015) with
+    outliers, a per-expert imatrix with 5% of the columns boosted x100), streamed expert by
+    expert: each expert's three tensors are drawn on the device (not timed), then quantized
+    (Q4_0, imatrix weighted) with CUDA events around the three launches, and their round trip
+    is accumulated.  Returns Gelem/s, the ALU-model fraction, per-shape rates and the weighted
+    RMSE over all experts."""
+    import torch
+    from post_weight_quantization_rowwise_b200 import synth
+    ts = synth.moe_experts(experts)
+    acc = torch.zeros(4, dtype=torch.float64, device=dev)
+    ms = {"gate": 0.0, "up": 0.0, "down": 0.0}
+    vals = {"gate": 0, "up": 0, "down": 0}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2: the tensors start in HBM
+    for e in range(experts):
+        trio = ts[3 * e:3 * e + 3]
+        xs = [t.weights(device=dev) for t in trio]
+        qs = [t.qw(device=dev) for t in trio]
+        bl = [torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8, device=dev) for t in trio]
+        flush.zero_()
+        ev[0].record()
+        for i, (t, x, q, b) in enumerate(zip(trio, xs, qs, bl)):
+            iqq.iqq_quantize_q4_0_w(x, q, b)
+            ev[i + 1].record()
+        for t, x, q, b in zip(trio, xs, qs, bl):
+            iqq.iqq_weighted_rmse(x, b, q, acc)
+        torch.cuda.synchronize()
+        for i, t in enumerate(trio):
+            kind = t.name.rsplit(".", 1)[1]
+            ms[kind] += ev[i].elapsed_time(ev[i + 1])
+            vals[kind] += t.numel
+    a = acc.cpu().tolist()
+    n = sum(vals.values())
+    total_ms = sum(ms.values())
+    ops = Q4_0_OPS_BASE + Q4_0_OPS_PER_PASS * p_mean
+    return {"experts": experts, "values": n, "quantize_ms": round(total_ms, 3),
+            "gelem_s": round(n / total_ms / 1e6, 3),
+            "frac": round(n * ops / (total_ms / 1e3) / 1e12 / peak_ops, 4),
+            "per_shape_gelem_s": {k: round(vals[k] / ms[k] / 1e6, 3) for k in ms},
+            "wrmse": math.sqrt(a[0] / a[1]), "maxerr": a[3],
+            "timing": "CUDA events around each expert's three quantize launches; tensors drawn, then "
+                      "L2 flushed (256 MB write), between experts"}
 
 
 def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
@@ -562,8 +606,9 @@ def main_ours(args):
     extras = None
     if rank == 0 and not args.no_extras:
         pk0 = peaks()
-        extras = run_extras(iqq, dev, cpu[3] if cpu else 1.1,
-                            B200_SMS * FP32_LANES_PER_SM * pk0["sm_max_mhz"] * 1e6 / 1e12, pk0["hbm_gbs"])
+        peak0 = B200_SMS * FP32_LANES_PER_SM * pk0["sm_max_mhz"] * 1e6 / 1e12
+        extras = run_extras(iqq, dev, cpu[3] if cpu else 1.1, peak0, pk0["hbm_gbs"])
+        extras["moe"] = run_moe(iqq, dev, peak0, cpu[3] if cpu else 1.1, args.moe_experts)
 
     e2e = None
     if not args.no_e2e:
@@ -605,7 +650,7 @@ def main_ours(args):
         "config": {"workload": WORKLOAD, "layers": args.layers, "tensors": n_q4,
                    "q4_0_values": w.q4_elems, "q8_k128_values": w.q8_elems,
                    "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (a layer set per rank, no data-path collective)"},
-        "roofline": {"bound": "alu", "kernel": "qx_0_w_kernel<4>",
+        "roofline": {"bound": "alu", "kernel": "q4_0_w_kernel<float>",
                      "achieved": round(achieved, 3),
                      "peak": round(peak_ops, 3), "unit": "Tops/s",
                      "frac": round(achieved / peak_ops, 4),
@@ -719,6 +764,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--e2e-layers", type=int, default=32)
+    ap.add_argument("--moe-experts", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")

@@ -14,7 +14,8 @@
 // 16-byte load, so a warp reads 512 contiguous bytes), writes qs[4t..4t+3]
 // as one 32-bit store (a warp writes 128 contiguous bytes), and lanes 0, 8,
 // 16, 24 write the four sums.  The work is HBM bound (4 B read + 140/128 B
-// written per value); each warp keeps four blocks in flight.
+// written per value); each warp keeps four blocks in flight, and the two IEEE
+// divisions of the four blocks (d and 1/d) run once, lane u taking block u.
 #include "common.cuh"
 
 namespace {
@@ -54,20 +55,35 @@ q8_k128_kernel(const float4* __restrict__ x, uint8_t* __restrict__ out, int64_t 
             const int64_t g = g0 + u;
             v[u] = g < nblocks ? iqq::ld_stream_f4(x + g * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        // amax of every block in flight (all lanes hold all of them)
+        float amax[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int64_t g = g0 + u;
-            if (g >= nblocks) break;  // warp-uniform
             const float4 a = v[u];
             // NaN/Inf detection: x*0 is NaN exactly for non-finite x
             const float z = __fmul_rn(a.x, 0.f) + __fmul_rn(a.y, 0.f) + __fmul_rn(a.z, 0.f) +
                             __fmul_rn(a.w, 0.f);
             if (z != z) bad |= IQQ_FLAG_NONFINITE_INPUT;
-            float amax = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
+            float m = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const float d = __fdiv_rn(amax, 127.0f);
-            const float id = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            amax[u] = m;
+        }
+        // d = amax/127 and id = 127/amax of block u are computed by lane u (one pass of the
+        // two IEEE divisions for all the blocks in flight), then broadcast
+        float am = amax[0];
+#pragma unroll
+        for (int u = 1; u < kUnroll; ++u)
+            if (lane == u) am = amax[u];
+        const float dl = __fdiv_rn(am, 127.0f);
+        const float idl = am > 0.f ? __fdiv_rn(127.0f, am) : 0.f;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = g0 + u;
+            const float d = __shfl_sync(0xffffffffu, dl, u);
+            const float id = __shfl_sync(0xffffffffu, idl, u);
+            if (g >= nblocks) break;  // warp-uniform
+            const float4 a = v[u];
             const int q0 = code_of(a.x, id), q1 = code_of(a.y, id);
             const int q2 = code_of(a.z, id), q3 = code_of(a.w, id);
             const uint32_t packed = (static_cast<uint32_t>(q0) & 0xffu) |
