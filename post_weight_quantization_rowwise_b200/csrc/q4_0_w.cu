@@ -68,6 +68,20 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr float kEta = 0.0009765625f;           // 2^-10: estimate closer than this to a candidate -> exact
 constexpr long long kWaitCycles = 4000000000LL; // about 2 s at 2 GHz
 
+// Unroll factors of the per-block loops over 4-value groups (larger: more latency hidden per
+// warp, more code for the instruction cache); values measured on the layer set.
+#ifndef IQQ_Q4_T_UNROLL
+#define IQQ_Q4_T_UNROLL 1       // transitions
+#endif
+#ifndef IQQ_Q4_X_UNROLL
+#define IQQ_Q4_X_UNROLL 1       // exact sums of a candidate
+#endif
+#ifndef IQQ_Q4_S_UNROLL
+#define IQQ_Q4_S_UNROLL 1       // weights, codes, greedy screen, final sums
+#endif
+#define IQQ_PRAGMA(x) _Pragma(#x)
+#define IQQ_UNROLL(n) IQQ_PRAGMA(unroll n)
+
 // Per consumer warp: x and w of its 32 blocks (row per lane, stride 36), and an area
 // used in turn by the per-candidate difference sums (float2 [18][32]), the survivors'
 // exact scores (float [32]) and the codes (float [32][33]).
@@ -109,7 +123,7 @@ __device__ __forceinline__ bool wait_at_least(const volatile int* p, int target)
 __device__ __forceinline__ float exact_score(const float* __restrict__ xr, const float* __restrict__ wr, float a)
 {
     float s = 0.0f, t = 0.0f;
-#pragma unroll 2
+    IQQ_UNROLL(IQQ_Q4_X_UNROLL)
     for (int j4 = 0; j4 < QK; j4 += 4) {
         const float4 xv4 = *reinterpret_cast<const float4*>(xr + j4);
         const float4 wv4 = *reinterpret_cast<const float4*>(wr + j4);
@@ -368,7 +382,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             if (qmin < 0.0f) bad |= IQQ_FLAG_NEG_QW;
         }
         const float sigma = weight_mode == 5 ? __fsqrt_rn(sigma2) : 0.0f;
-#pragma unroll 1
+        IQQ_UNROLL(IQQ_Q4_S_UNROLL)
         for (int i = 0; i < QK; i += 4) {
             const float4 v = *reinterpret_cast<const float4*>(my_x + i);
             const float4 q = *reinterpret_cast<const float4*>(my_w + i);
@@ -415,7 +429,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     const float kR = __fmul_rn(10.0f, A);  // 80*|xmax|/nmax: the step index scale
     float S0 = 0.0f, T0 = 0.0f, nsteps = 0.0f;
     uint32_t m_unc = 0u, m_two = 0u;
-#pragma unroll 1
+    IQQ_UNROLL(IQQ_Q4_T_UNROLL)
     for (int j4 = 0; j4 < QK; j4 += 4) {
         const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
         const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
@@ -606,7 +620,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
                 mode = 2;
             }
         }
-#pragma unroll 1
+        IQQ_UNROLL(IQQ_Q4_S_UNROLL)
         for (int j4 = 0; j4 < QK; j4 += 4) {
             const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
             const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
@@ -642,7 +656,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         const float D = __fmul_rn(suml2, rcp_approx(sumlx));
         const float thr = __fmul_rn(suml2, 0x1p-20f);
         uint32_t maybe = 0u;
-#pragma unroll 1
+        IQQ_UNROLL(IQQ_Q4_S_UNROLL)
         for (int j4 = 0; j4 < QK; j4 += 4) {
             const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
             const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
@@ -697,7 +711,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         float d = dfb;
         if (mode == 2) {
             float sfx = 0.0f, sf2 = 0.0f;
-#pragma unroll 1
+            IQQ_UNROLL(IQQ_Q4_S_UNROLL)
             for (int j4 = 0; j4 < QK; j4 += 4) {
                 const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
                 const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
