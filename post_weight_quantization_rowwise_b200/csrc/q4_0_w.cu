@@ -79,6 +79,9 @@ constexpr long long kWaitCycles = 4000000000LL; // about 2 s at 2 GHz
 #ifndef IQQ_Q4_S_UNROLL
 #define IQQ_Q4_S_UNROLL 1       // weights, codes, greedy screen, final sums
 #endif
+#ifndef IQQ_Q4_PDL
+#define IQQ_Q4_PDL 1            // programmatic dependent launch between consecutive launches
+#endif
 #define IQQ_PRAGMA(x) _Pragma(#x)
 #define IQQ_UNROLL(n) IQQ_PRAGMA(unroll n)
 
@@ -435,7 +438,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
         const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
         const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
-        const uint32_t bit = 1u << j4;
+        uint32_t unc4 = 0u, two4 = 0u;  // this group's masks (constant shifts)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float xs = xq[k], w = wq[k];
@@ -463,9 +466,11 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             v.x = __fadd_rn(v.x, p);
             v.y = __fmaf_rn(w, __fmaf_rn(2.0f, m0, 1.0f), v.y);
             if (sure) *c = v;
-            if (step && !sure) m_unc |= bit << k;
-            if (dm > 1.5f) m_two |= bit << k;
+            unc4 |= static_cast<uint32_t>(step && !sure) << k;
+            two4 |= static_cast<uint32_t>(dm > 1.5f) << k;
         }
+        m_unc |= unc4 << j4;
+        m_two |= two4 << j4;
     }
     // The first largest element (|x| = |xmax|) always has one step, 7 -> 8, and it lies on a
     // rounding tie: at candidate 4 (c = 7.5) when fl(fl(7.5/|xmax|)*|xmax|) >= 7.5 (rint
@@ -769,6 +774,11 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
     const int64_t t1 = t0 + per + (static_cast<int64_t>(blockIdx.x) < extra ? 1 : 0);
     if (threadIdx.x < kCand) s_c[threadIdx.x] = __fdiv_rn(static_cast<float>(kNmax * (71 + threadIdx.x)), 80.0f);
     if (threadIdx.x == 0) s_abort = 0;
+    // Programmatic dependent launch: the next kernel of the stream may be scheduled now (its
+    // CTAs start as this grid's retire); this grid waits for the previous kernel's completion
+    // and memory before its first global access.  (No-ops without the launch attribute.)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     int64_t g = t0 * 32;
     const int64_t gend = t1 * 32 < total ? t1 * 32 : total;
     while (g < gend) {
@@ -827,8 +837,19 @@ iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_
     }
     const int64_t tiles = (nrows * (n_per_row / QK) + 31) / 32;
     const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
-    q4_0_w_kernel<XT><<<grid, kThreads, kDynSmem, static_cast<cudaStream_t>(stream)>>>(
-        x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kDynSmem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = IQQ_Q4_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, q4_0_w_kernel<XT>, x, qw, static_cast<uint8_t*>(out), nrows, n_per_row,
+                           rows_per_qw, weight_mode, fudge, d_flags) != cudaSuccess)
+        return iqq::launch_status();
     return iqq::launch_status();
 }
 
