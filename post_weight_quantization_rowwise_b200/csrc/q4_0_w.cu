@@ -40,8 +40,8 @@
 //     non-finite values, empty weights) take the direct sweep.
 //
 // Work layout: a persistent grid splits the tensor's blocks, in row-major order,
-// into equal ranges of 32-block tiles, one range per CTA.  Eight consumer warps
-// take tiles from a shared counter (one block per lane); a ninth, producer, warp
+// into equal ranges of 32-block tiles, one range per CTA.  Eighteen consumer warps
+// take tiles from a shared counter (one block per lane); one more, producer, warp
 // computes each row's sigma2 (binary64 sum of exact squares) just ahead of them,
 // which also brings the rows into L2 before the consumers load their blocks.  A
 // tile may span rows; every lane finds its own row.  Rows of any width are
@@ -58,9 +58,12 @@ namespace {
 constexpr int QK = IQQ_Q4_0_BLOCK_VALUES;
 constexpr int kNmax = 8;
 constexpr int kCand = 19;
-constexpr int kConsumers = 8;                   // consumer warps per CTA
+#ifndef IQQ_Q4_CONSUMERS
+#define IQQ_Q4_CONSUMERS 18     // consumer warps per CTA: 18 fill an SM's shared memory (one CTA per SM)
+#endif
+constexpr int kConsumers = IQQ_Q4_CONSUMERS;
 constexpr int kThreads = (kConsumers + 1) * 32; // plus one producer warp
-constexpr int kRowS = QK + 4;                   // staging row stride: 16-byte rows, LDS.128 conflict-free
+constexpr int kRowS = QK + 4;                   // code row stride: 16-byte rows, LDS.128 conflict-free
 constexpr int kMaxRows = 256;                   // sigma2 rows per chunk of a CTA's range
 constexpr int kLeadRows = 4;                    // rows the producer may run ahead of the consumers
 constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23
@@ -85,12 +88,15 @@ constexpr long long kWaitCycles = 4000000000LL; // about 2 s at 2 GHz
 #define IQQ_PRAGMA(x) _Pragma(#x)
 #define IQQ_UNROLL(n) IQQ_PRAGMA(unroll n)
 
-// Per consumer warp: x and w of its 32 blocks (row per lane, stride 36), and an area
-// used in turn by the per-candidate difference sums (float2 [18][32]), the survivors'
-// exact scores (float [32]) and the codes (float [32][33]).
+// Per consumer warp: x and w of its 32 blocks, chunk-interleaved (the 16-byte chunk c of lane
+// L's block at float 128c + 4L, so that the lanes of a quarter warp loading the same chunk of
+// their blocks hit distinct banks, without padding), and an area used in turn by the
+// per-candidate difference sums (float2 [18][32]), the survivors' exact scores (float2 [32])
+// and the codes (float [32][36], padded rows).  18 warps fill an SM's shared memory:
+// 18 x 12.5 KB.
 struct WarpSmem {
-    float x[32 * kRowS];
-    float w[32 * kRowS];
+    float x[32 * QK];
+    float w[32 * QK];
     union {
         float2 diff[18 * 32];
         float2 res[32];  // (score, k) of an exact check
@@ -98,6 +104,10 @@ struct WarpSmem {
     } u;
 };
 constexpr size_t kDynSmem = sizeof(WarpSmem) * kConsumers;
+
+// Offset of value j of a block in the chunk-interleaved x and w areas, from the block's base
+// (area + 4 * lane).
+__device__ __forceinline__ int xoff(int j) { return ((j & ~3) << 5) | (j & 3); }
 
 __device__ __forceinline__ float rcp_approx(float v)
 {
@@ -122,14 +132,14 @@ __device__ __forceinline__ bool wait_at_least(const volatile int* p, int target)
     return true;
 }
 
-// The exact sequential sums of the candidate iscale = a over a staged row, and its score.
+// The exact sequential sums of the candidate iscale = a over a staged block, and its score.
 __device__ __forceinline__ float exact_score(const float* __restrict__ xr, const float* __restrict__ wr, float a)
 {
     float s = 0.0f, t = 0.0f;
     IQQ_UNROLL(IQQ_Q4_X_UNROLL)
     for (int j4 = 0; j4 < QK; j4 += 4) {
-        const float4 xv4 = *reinterpret_cast<const float4*>(xr + j4);
-        const float4 wv4 = *reinterpret_cast<const float4*>(wr + j4);
+        const float4 xv4 = *reinterpret_cast<const float4*>(xr + 32 * j4);
+        const float4 wv4 = *reinterpret_cast<const float4*>(wr + 32 * j4);
         const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
         const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
 #pragma unroll
@@ -159,8 +169,8 @@ __device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, fl
         float l2 = __shfl_sync(kFull, suml2, bb);
         float sc = __shfl_sync(kFull, score, bb);
         int start = __shfl_sync(kFull, gstart, bb);
-        const float xj = sX[bb * kRowS + lane];
-        const float wj = sW[bb * kRowS + lane];
+        const float xj = sX[4 * bb + xoff(lane)];
+        const float wj = sW[4 * bb + xoff(lane)];
         float lj = sL[bb * kRowS + lane];
         const float wxj = __fmul_rn(wj, xj);
         float d = __fdiv_rn(lx, l2);
@@ -262,26 +272,29 @@ __device__ void produce_rows(const XT* __restrict__ x, int64_t n_per_row, int64_
     }
 }
 
-// Stages the block's 32 values of x into the lane's row: 16-byte asynchronous copies for
-// binary32 storage (no registers held while they are in flight), widened loads for bf16.
+// Stages the block's 32 values of x into the lane's interleaved chunks: 16-byte asynchronous
+// copies for binary32 storage (no registers held while they are in flight), widened loads for
+// bf16.
 __device__ __forceinline__ void stage_x(float* dst, const float* src)
 {
     const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
 #pragma unroll
     for (int i = 0; i < QK / 4; ++i)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + 16 * i), "l"(src + 4 * i) : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + 512 * i), "l"(src + 4 * i)
+                     : "memory");
 }
 __device__ __forceinline__ void stage_x(float* dst, const __nv_bfloat16* src)
 {
 #pragma unroll
-    for (int i = 0; i < QK / 4; ++i) *reinterpret_cast<float4*>(dst + 4 * i) = iqq::ld4(src + 4 * i);
+    for (int i = 0; i < QK / 4; ++i) *reinterpret_cast<float4*>(dst + 128 * i) = iqq::ld4(src + 4 * i);
 }
 __device__ __forceinline__ void stage_qw(float* dst, const float* src)
 {
     const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
 #pragma unroll
     for (int i = 0; i < QK / 4; ++i)
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(d + 16 * i), "l"(src + 4 * i) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(d + 512 * i), "l"(src + 4 * i)
+                     : "memory");
 }
 __device__ __forceinline__ void staged_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
@@ -329,8 +342,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     const int64_t row = rA + rr;
 
     // x and qw of the block into the lane's rows (asynchronous while the row's sigma2 is awaited)
-    float* const my_x = ws.x + lane * kRowS;
-    float* const my_w = ws.w + lane * kRowS;
+    float* const my_x = ws.x + 4 * lane;
+    float* const my_w = ws.w + 4 * lane;
     const int64_t qrow = rows_per_qw > 0 ? row / rows_per_qw : 0;
     const float* qb = qw != nullptr ? qw + qrow * n_per_row + static_cast<int64_t>(b) * QK : nullptr;
     if (valid) {
@@ -367,17 +380,18 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         if (!valid) {
 #pragma unroll
             for (int i = 0; i < QK; i += 4) {
-                *reinterpret_cast<float4*>(my_x + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4*>(my_w + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(my_x + 32 * i) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(my_w + 32 * i) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         } else if (qb == nullptr) {
 #pragma unroll
-            for (int i = 0; i < QK; i += 4) *reinterpret_cast<float4*>(my_w + i) = make_float4(1.f, 1.f, 1.f, 1.f);
+            for (int i = 0; i < QK; i += 4)
+                *reinterpret_cast<float4*>(my_w + 32 * i) = make_float4(1.f, 1.f, 1.f, 1.f);
         } else if (rows_per_qw > 0 ? row % rows_per_qw == 0 : row == 0) {
             float qmin = 0.0f, qnf = 0.0f;
 #pragma unroll 2
             for (int i = 0; i < QK; i += 4) {
-                const float4 q = *reinterpret_cast<const float4*>(my_w + i);
+                const float4 q = *reinterpret_cast<const float4*>(my_w + 32 * i);
                 qmin = fminf(fminf(qmin, fminf(q.x, q.y)), fminf(q.z, q.w));
                 qnf = __fmaf_rn(q.x, 0.0f, __fmaf_rn(q.y, 0.0f, __fmaf_rn(q.z, 0.0f, __fmaf_rn(q.w, 0.0f, qnf))));
             }
@@ -387,8 +401,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         const float sigma = weight_mode == 5 ? __fsqrt_rn(sigma2) : 0.0f;
         IQQ_UNROLL(IQQ_Q4_S_UNROLL)
         for (int i = 0; i < QK; i += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(my_x + i);
-            const float4 q = *reinterpret_cast<const float4*>(my_w + i);
+            const float4 v = *reinterpret_cast<const float4*>(my_x + 32 * i);
+            const float4 q = *reinterpret_cast<const float4*>(my_w + 32 * i);
             const float xq[4] = {v.x, v.y, v.z, v.w};
             float wq[4] = {q.x, q.y, q.z, q.w};
             if (weight_mode == 0) {
@@ -415,7 +429,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
                 const float a = fabsf(xq[k]);
                 if (a > A) { A = a; xmax = xq[k]; jmax = i + k; }
             }
-            *reinterpret_cast<float4*>(my_w + i) = make_float4(wq[0], wq[1], wq[2], wq[3]);
+            *reinterpret_cast<float4*>(my_w + 32 * i) = make_float4(wq[0], wq[1], wq[2], wq[3]);
         }
     }
 
@@ -434,8 +448,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     uint32_t m_unc = 0u, m_two = 0u;
     IQQ_UNROLL(IQQ_Q4_T_UNROLL)
     for (int j4 = 0; j4 < QK; j4 += 4) {
-        const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
-        const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+        const float4 xv4 = *reinterpret_cast<const float4*>(my_x + 32 * j4);
+        const float4 wv4 = *reinterpret_cast<const float4*>(my_w + 32 * j4);
         const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
         const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
         uint32_t unc4 = 0u, two4 = 0u;  // this group's masks (constant shifts)
@@ -478,7 +492,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     // among the uncertain steps below.
     if (active && ((m_unc >> jmax) & 1u)) {
         const float v4 = __fmul_rn(__fdiv_rn(s_c[4], A), A);
-        const float w = my_w[jmax];
+        const float w = my_w[xoff(jmax)];
         float2* c = dcol + 32 * (v4 >= 7.5f ? 3 : 4);
         float2 v = *c;
         v.x = __fadd_rn(v.x, fabsf(__fmul_rn(w, xmax)));
@@ -492,7 +506,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         while (todo != 0u) {
             const int j = __ffs(todo) - 1;
             todo &= todo - 1u;
-            const float xs = my_x[j], w = my_w[j];
+            const float xs = my_x[xoff(j)], w = my_w[xoff(j)];
             const float X = fabsf(xs);
             const float m0 = fabsf(rintf(__fmul_rn(a0, xs)));
             const float R = __fmul_rn(kR, rcp_approx(X));
@@ -503,7 +517,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         while (todo != 0u) {
             const int j = __ffs(todo) - 1;
             todo &= todo - 1u;
-            const float xs = my_x[j], w = my_w[j];
+            const float xs = my_x[xoff(j)], w = my_w[xoff(j)];
             const float X = fabsf(xs);
             const float m0 = fabsf(rintf(__fmul_rn(a0, xs)));
             const float R = __fmul_rn(kR, rcp_approx(X));
@@ -587,7 +601,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             int kk = 0;
             if (q < total) {
                 kk = static_cast<int>(min(__fns(osurv, 0, q - ostart + 1), static_cast<unsigned>(kCand - 1)));
-                r = exact_score(ws.x + owner * kRowS, ws.w + owner * kRowS, __fdiv_rn(-s_c[kk], oxmax));
+                r = exact_score(ws.x + 4 * owner, ws.w + 4 * owner, __fdiv_rn(-s_c[kk], oxmax));
             }
             ws.u.res[lane] = make_float2(r, __int_as_float(kk));
             __syncwarp();
@@ -627,8 +641,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         }
         IQQ_UNROLL(IQQ_Q4_S_UNROLL)
         for (int j4 = 0; j4 < QK; j4 += 4) {
-            const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
-            const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+            const float4 xv4 = *reinterpret_cast<const float4*>(my_x + 32 * j4);
+            const float4 wv4 = *reinterpret_cast<const float4*>(my_w + 32 * j4);
             const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
             const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
             float lq[4];
@@ -663,8 +677,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         uint32_t maybe = 0u;
         IQQ_UNROLL(IQQ_Q4_S_UNROLL)
         for (int j4 = 0; j4 < QK; j4 += 4) {
-            const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
-            const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+            const float4 xv4 = *reinterpret_cast<const float4*>(my_x + 32 * j4);
+            const float4 wv4 = *reinterpret_cast<const float4*>(my_w + 32 * j4);
             const float4 lv4 = *reinterpret_cast<const float4*>(my_l + j4);
             const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
             const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
@@ -683,7 +697,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         while (maybe != 0u) {
             const int j = __ffs(maybe) - 1;
             maybe &= maybe - 1u;
-            const float xj = my_x[j], wj = my_w[j], lj = my_l[j];
+            const float xj = my_x[xoff(j)], wj = my_w[xoff(j)], lj = my_l[j];
             const float g = __fmul_rn(d, __fmul_rn(wj, __fsub_rn(xj, __fmul_rn(d, lj))));
             const float sg = g > 0.0f ? 1.0f : -1.0f;
             const float ln = __fadd_rn(lj, sg);
@@ -718,8 +732,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             float sfx = 0.0f, sf2 = 0.0f;
             IQQ_UNROLL(IQQ_Q4_S_UNROLL)
             for (int j4 = 0; j4 < QK; j4 += 4) {
-                const float4 xv4 = *reinterpret_cast<const float4*>(my_x + j4);
-                const float4 wv4 = *reinterpret_cast<const float4*>(my_w + j4);
+                const float4 xv4 = *reinterpret_cast<const float4*>(my_x + 32 * j4);
+                const float4 wv4 = *reinterpret_cast<const float4*>(my_w + 32 * j4);
                 const float4 lv4 = *reinterpret_cast<const float4*>(my_l + j4);
                 const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
                 const float wq[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
@@ -755,7 +769,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
 }
 
 template <typename XT>
-__global__ void __maxnreg__(96)  // 2 CTAs of 288 threads per SM (at most 5 warps of an SMSP's 16K registers)
+__global__ void __maxnreg__(96)  // one CTA of 608 threads per SM (at most 5 warps of an SMSP's 16K registers)
 q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out, int64_t nrows,
               int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* __restrict__ flags)
 {
