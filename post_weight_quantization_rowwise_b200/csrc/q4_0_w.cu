@@ -220,51 +220,59 @@ __device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, fl
     }
 }
 
-// The producer warp: sigma2 of rows rA .. rA+nr-1 in order, published through s_produced.
+// One warp: sigma2 of the row xr into *sig (lane 0 writes): the binary64 sum of exact squares
+// over n_per_row; an Inf or NaN in x makes it non-finite (the square of any finite binary32
+// value is finite in binary64) and raises the flag.
 template <typename XT>
-__device__ void produce_rows(const XT* __restrict__ x, int64_t n_per_row, int64_t rA, int nr, float* s_sig,
-                             volatile int* s_produced, const volatile int* s_consumed_row,
-                             uint32_t* __restrict__ flags)
+__device__ __forceinline__ void row_sigma2(const XT* __restrict__ xr, int64_t n_per_row, float* sig,
+                                           uint32_t* __restrict__ flags)
 {
     const int lane = threadIdx.x & 31;
     const int64_t n4 = n_per_row / 4;
-    for (int rr = 0; rr < nr; ++rr) {
+    double acc = 0.0;
+    int64_t i = lane;
+    for (; i + 15 * 32 < n4; i += 16 * 32) {
+        float4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] = iqq::ld4(xr + 4 * (i + 32 * u));
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            acc = fma(static_cast<double>(v[u].x), static_cast<double>(v[u].x), acc);
+            acc = fma(static_cast<double>(v[u].y), static_cast<double>(v[u].y), acc);
+            acc = fma(static_cast<double>(v[u].z), static_cast<double>(v[u].z), acc);
+            acc = fma(static_cast<double>(v[u].w), static_cast<double>(v[u].w), acc);
+        }
+    }
+    for (; i < n4; i += 32) {
+        const float4 v = iqq::ld4(xr + 4 * i);
+        acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
+        acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
+        acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
+        acc = fma(static_cast<double>(v.w), static_cast<double>(v.w), acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (lane == 0) {
+        if (!isfinite(acc)) iqq::raise_flags(flags, IQQ_FLAG_NONFINITE_INPUT);
+        *sig = static_cast<float>(acc / static_cast<double>(n_per_row));
+    }
+}
+
+// The producer warp: sigma2 of rows rA+r0 .. rA+nr-1 in order, published through s_produced.
+template <typename XT>
+__device__ void produce_rows(const XT* __restrict__ x, int64_t n_per_row, int64_t rA, int r0, int nr, float* s_sig,
+                             volatile int* s_produced, const volatile int* s_consumed_row,
+                             uint32_t* __restrict__ flags)
+{
+    for (int rr = r0; rr < nr; ++rr) {
         // stay a few rows ahead of the furthest row a grabbed tile needs, so that the rows read
         // here are still in L2 when the consumers load their blocks (bounded: on expiry go on)
         if (rr > kLeadRows) {
             const long long t0 = clock64();
             while (*s_consumed_row + kLeadRows < rr && clock64() - t0 < kWaitCycles / 4) __nanosleep(256);
         }
-        const XT* xr = x + (rA + rr) * n_per_row;
-        // binary64 sum of exact squares; an Inf or NaN in x makes it non-finite (the square of
-        // any finite binary32 value is finite in binary64)
-        double acc = 0.0;
-        int64_t i = lane;
-        for (; i + 15 * 32 < n4; i += 16 * 32) {
-            float4 v[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] = iqq::ld4(xr + 4 * (i + 32 * u));
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                acc = fma(static_cast<double>(v[u].x), static_cast<double>(v[u].x), acc);
-                acc = fma(static_cast<double>(v[u].y), static_cast<double>(v[u].y), acc);
-                acc = fma(static_cast<double>(v[u].z), static_cast<double>(v[u].z), acc);
-                acc = fma(static_cast<double>(v[u].w), static_cast<double>(v[u].w), acc);
-            }
-        }
-        for (; i < n4; i += 32) {
-            const float4 v = iqq::ld4(xr + 4 * i);
-            acc = fma(static_cast<double>(v.x), static_cast<double>(v.x), acc);
-            acc = fma(static_cast<double>(v.y), static_cast<double>(v.y), acc);
-            acc = fma(static_cast<double>(v.z), static_cast<double>(v.z), acc);
-            acc = fma(static_cast<double>(v.w), static_cast<double>(v.w), acc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-        const bool bad = !isfinite(acc);
-        if (lane == 0) {
-            if (bad) iqq::raise_flags(flags, IQQ_FLAG_NONFINITE_INPUT);
-            s_sig[rr] = static_cast<float>(acc / static_cast<double>(n_per_row));
+        row_sigma2(x + (rA + rr) * n_per_row, n_per_row, &s_sig[rr], flags);
+        if ((threadIdx.x & 31) == 0) {
             __threadfence_block();
             *s_produced = rr + 1;
         }
@@ -801,15 +809,21 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
         int64_t gB = (rA + kMaxRows) * nb / 32 * 32;
         if (gB > gend) gB = gend;
         const int nr = static_cast<int>((gB - 1) / nb - rA + 1);
+        // the rows of the first tiles the warps take, one row per warp, side by side; the
+        // producer continues after them
+        const int64_t need = (g - rA * nb + static_cast<int64_t>(kConsumers) * 32 + nb - 1) / nb;
+        const int head =
+            static_cast<int>(min(min(static_cast<int64_t>(nr), need), static_cast<int64_t>(kConsumers + 1)));
         __syncthreads();  // every warp is done with the previous chunk
+        if (warp < head) row_sigma2(x + (rA + warp) * n_per_row, n_per_row, &s_sig[warp], flags);
         if (threadIdx.x == 0) {
-            s_produced = 0;
+            s_produced = head;
             s_next = 0;
             s_consumed_row = 0;
         }
         __syncthreads();
         if (warp == kConsumers) {
-            produce_rows<XT>(x, n_per_row, rA, nr, s_sig, &s_produced, &s_consumed_row, flags);
+            produce_rows<XT>(x, n_per_row, rA, head, nr, s_sig, &s_produced, &s_consumed_row, flags);
         } else {
             WarpSmem& ws = wsm[warp];
             while (true) {
