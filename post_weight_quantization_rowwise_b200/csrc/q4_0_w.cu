@@ -406,38 +406,54 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             if (qnf != qnf) bad |= IQQ_FLAG_NONFINITE_INPUT;
             if (qmin < 0.0f) bad |= IQQ_FLAG_NEG_QW;
         }
-        const float sigma = weight_mode == 5 ? __fsqrt_rn(sigma2) : 0.0f;
-        IQQ_UNROLL(IQQ_Q4_S_UNROLL)
-        for (int i = 0; i < QK; i += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(my_x + 32 * i);
-            const float4 q = *reinterpret_cast<const float4*>(my_w + 32 * i);
-            const float xq[4] = {v.x, v.y, v.z, v.w};
-            float wq[4] = {q.x, q.y, q.z, q.w};
-            if (weight_mode == 0) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    wq[k] = __fmul_rn(wq[k], __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xq[k], xq[k]))));
-            } else if (weight_mode != 1) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float xj = xq[k];
-                    const float t = __fmul_rn(xj, xj);
-                    float m;
-                    switch (weight_mode) {
-                    case 2: m = t; break;
-                    case 3: m = fabsf(xj); break;
-                    case 4: m = __fadd_rn(sigma2, t); break;
-                    default: m = __fadd_rn(sigma, fabsf(xj)); break;
-                    }
-                    wq[k] = __fmul_rn(wq[k], m);
-                }
-            }
+        // |xmax| and xmax, the first element of largest |x|, and its index
+        auto track = [&](const float (&xq)[4], int i) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float a = fabsf(xq[k]);
                 if (a > A) { A = a; xmax = xq[k]; jmax = i + k; }
             }
-            *reinterpret_cast<float4*>(my_w + 32 * i) = make_float4(wq[0], wq[1], wq[2], wq[3]);
+        };
+        if (weight_mode == 0) {  // the default weights: a loop of their own (compact code)
+            IQQ_UNROLL(IQQ_Q4_S_UNROLL)
+            for (int i = 0; i < QK; i += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(my_x + 32 * i);
+                const float4 q = *reinterpret_cast<const float4*>(my_w + 32 * i);
+                const float xq[4] = {v.x, v.y, v.z, v.w};
+                const float wq[4] = {q.x, q.y, q.z, q.w};
+                float wn[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    wn[k] = __fmul_rn(wq[k], __fsqrt_rn(__fadd_rn(sigma2, __fmul_rn(xq[k], xq[k]))));
+                track(xq, i);
+                *reinterpret_cast<float4*>(my_w + 32 * i) = make_float4(wn[0], wn[1], wn[2], wn[3]);
+            }
+        } else {
+            const float sigma = weight_mode == 5 ? __fsqrt_rn(sigma2) : 0.0f;
+#pragma unroll 1
+            for (int i = 0; i < QK; i += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(my_x + 32 * i);
+                const float4 q = *reinterpret_cast<const float4*>(my_w + 32 * i);
+                const float xq[4] = {v.x, v.y, v.z, v.w};
+                float wq[4] = {q.x, q.y, q.z, q.w};
+                if (weight_mode != 1) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float xj = xq[k];
+                        const float t = __fmul_rn(xj, xj);
+                        float m;
+                        switch (weight_mode) {
+                        case 2: m = t; break;
+                        case 3: m = fabsf(xj); break;
+                        case 4: m = __fadd_rn(sigma2, t); break;
+                        default: m = __fadd_rn(sigma, fabsf(xj)); break;
+                        }
+                        wq[k] = __fmul_rn(wq[k], m);
+                    }
+                }
+                track(xq, i);
+                *reinterpret_cast<float4*>(my_w + 32 * i) = make_float4(wq[0], wq[1], wq[2], wq[3]);
+            }
         }
     }
 
@@ -508,34 +524,29 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         *c = v;
         m_unc &= ~(1u << jmax);
     }
-    // the other uncertain first steps, then the second steps, per lane from the staged row
+    // the other uncertain first steps and the second steps, per lane from the staged row, one
+    // pass over the values that have either
     {
-        uint32_t todo = m_unc;
+        uint32_t todo = m_unc | m_two;
         while (todo != 0u) {
             const int j = __ffs(todo) - 1;
             todo &= todo - 1u;
             const float xs = my_x[xoff(j)], w = my_w[xoff(j)];
             const float X = fabsf(xs);
+            const float p = fabsf(__fmul_rn(w, xs));
             const float m0 = fabsf(rintf(__fmul_rn(a0, xs)));
             const float R = __fmul_rn(kR, rcp_approx(X));
             const float t = __fmaf_rn(m0, R, __fmaf_rn(0.5f, R, -70.5f));  // as in the loop above
-            add_step(dcol, exact_step(t, m0, X, A, s_c), fabsf(__fmul_rn(w, xs)), w, m0);
-        }
-        todo = m_two;
-        while (todo != 0u) {
-            const int j = __ffs(todo) - 1;
-            todo &= todo - 1u;
-            const float xs = my_x[xoff(j)], w = my_w[xoff(j)];
-            const float X = fabsf(xs);
-            const float m0 = fabsf(rintf(__fmul_rn(a0, xs)));
-            const float R = __fmul_rn(kR, rcp_approx(X));
-            const float t = __fadd_rn(__fmaf_rn(m0, R, __fmaf_rn(0.5f, R, -70.5f)), R);  // second step
-            const float n = __fadd_rn(m0, 1.0f);
-            const float y = __fadd_rn(t, kMagic);
-            const float dist = __fsub_rn(t, __fsub_rn(y, kMagic));
-            int idx = static_cast<int>(__float_as_uint(y) - __float_as_uint(kMagic));
-            if (!(fabsf(dist) < 0.5f - kEta && idx >= 1 && idx <= 18)) idx = exact_step(t, n, X, A, s_c);
-            add_step(dcol, idx, fabsf(__fmul_rn(w, xs)), w, n);
+            if ((m_unc >> j) & 1u) add_step(dcol, exact_step(t, m0, X, A, s_c), p, w, m0);
+            if ((m_two >> j) & 1u) {
+                const float t2 = __fadd_rn(t, R);  // the second step
+                const float n = __fadd_rn(m0, 1.0f);
+                const float y = __fadd_rn(t2, kMagic);
+                const float dist = __fsub_rn(t2, __fsub_rn(y, kMagic));
+                int idx = static_cast<int>(__float_as_uint(y) - __float_as_uint(kMagic));
+                if (!(fabsf(dist) < 0.5f - kEta && idx >= 1 && idx <= 18)) idx = exact_step(t2, n, X, A, s_c);
+                add_step(dcol, idx, p, w, n);
+            }
         }
     }
 
