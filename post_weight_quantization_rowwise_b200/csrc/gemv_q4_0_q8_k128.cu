@@ -42,15 +42,18 @@
 
 namespace {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = kWarps * 32;
+constexpr int kWarps = 16;      // warps per CTA; 32 for one token when one CTA fits per SM
+constexpr int kWarpsWide = 32;
 constexpr int kUnitPairs = 64;                    // pairs of blocks per streamed unit
 constexpr int kUnitBytes = kUnitPairs * 36 + 16;  // + room for the 8-byte start offset
-constexpr int kStaticSmem = kWarps * 4 * 8;        // the kernel's per-warp range slots
-constexpr int kSmemMax = 227 * 1024 - kStaticSmem;  // dynamic shared memory per CTA, at most
+__host__ __device__ constexpr int static_smem(int warps) { return warps * 4 * 8; }  // per-warp range slots
+constexpr int kSmemCta = 227 * 1024;              // shared memory per CTA, at most
 constexpr int kSmemPerSm = 228 * 1024;
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the maximum SM clock
 constexpr uint32_t kSuspendHintNs = 100000;
+#ifndef IQQ_GEMV_WIDE
+#define IQQ_GEMV_WIDE 1  // 32-warp CTAs for one token on very wide rows
+#endif
 #ifndef IQQ_GEMV_PDL
 #define IQQ_GEMV_PDL 1  // launch with programmatic stream serialization
 #endif
@@ -255,8 +258,8 @@ __device__ __forceinline__ int64_t share_start(const Params& P, uint32_t c)
            static_cast<int64_t>(c * static_cast<uint32_t>(P.share_r) / static_cast<uint32_t>(P.ctas));
 }
 
-template <int TT>
-__global__ void __launch_bounds__(kThreads, TT == 1 ? 2 : 1)
+template <int TT, int W>
+__global__ void __launch_bounds__(W * 32, TT == 1 && W == kWarps ? 2 : 1)
 gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -292,8 +295,8 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
     // The first and last problems it touches and its first / end row in them are found once,
     // here, and parked in shared memory (the 64-bit divisions are calls that would otherwise
     // force the row loops' registers to the stack).
-    __shared__ int64_t s_rng[kWarps][4];
-    static_assert(sizeof(s_rng) == kStaticSmem, "static shared memory of the launch plan");
+    __shared__ int64_t s_rng[W][4];
+    static_assert(sizeof(s_rng) == static_smem(W), "static shared memory of the launch plan");
     {
         const int64_t t0 = share_start(P, share), t1 = share_start(P, share + 1);
         int pf = 0;
@@ -344,7 +347,7 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
                 if (lane == 0) issue_unit(V, stages + is * kUnitBytes, &bars[is], r_begin + irow, iseg);
                 if (++iseg == nseg) {
                     iseg = 0;
-                    irow += kWarps;
+                    irow += W;
                 }
                 if (++is == D) is = 0;
             }
@@ -362,11 +365,11 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
             constexpr int kStageBlocks = TT == 1 ? 4 : 8;
             const int nblk = nt * nb8;
             const uint8_t* abase = pr.a + tok0 * nb8 * 140;
-            for (int b0 = warp; b0 < nblk; b0 += kStageBlocks * kWarps) {
+            for (int b0 = warp; b0 < nblk; b0 += kStageBlocks * W) {
                 uint32_t v[kStageBlocks], e[kStageBlocks];
 #pragma unroll
                 for (int u = 0; u < kStageBlocks; ++u) {
-                    const int b = b0 + u * kWarps;
+                    const int b = b0 + u * W;
                     v[u] = 0u;
                     e[u] = 0u;
                     if (b < nblk) {
@@ -377,7 +380,7 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
                 }
 #pragma unroll
                 for (int u = 0; u < kStageBlocks; ++u) {
-                    const int b = b0 + u * kWarps;
+                    const int b = b0 + u * W;
                     if (b < nblk) {
                         const int t = b / nb8, g = b - t * nb8;
                         *reinterpret_cast<uint32_t*>(q8s + t * act_q8_bytes + q8_swizzle(128 * g + 4 * lane)) = v[u];
@@ -418,7 +421,7 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
                 if (lane == 0) issue_unit(V, stages + s * kUnitBytes, &bars[s], r_begin + irow, iseg);
                 if (++iseg == nseg) {
                     iseg = 0;
-                    irow += kWarps;
+                    irow += W;
                 }
             }
             if (TT == 1) {
@@ -453,7 +456,7 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
 #pragma unroll
                 for (int t = 0; t < TT; ++t) acc[t] = 0.0;
                 seg = 0;
-                row += kWarps;
+                row += W;
             }
             if (++s == D) {
                 s = 0;
@@ -469,7 +472,7 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
                 (void)mbar_wait(&bars[s], ph);
                 if (++seg == nseg) {
                     seg = 0;
-                    row += kWarps;
+                    row += W;
                 }
                 if (++s == D) {
                     s = 0;
@@ -484,8 +487,8 @@ gemv_q4_0_q8_k128_kernel(const __grid_constant__ Params P)
 // time in these queries than a small matrix takes on the GPU).
 struct DeviceCache {
     std::atomic<int> sms{0};
-    std::atomic<int> smem_set[4] = {{0}, {0}, {0}, {0}};  // dynamic smem opted in, per TT
-    std::atomic<int> regs[4] = {{0}, {0}, {0}, {0}};      // registers per thread, per TT
+    std::atomic<int> smem_set[8] = {};  // dynamic smem opted in, per (TT, W)
+    std::atomic<int> regs[8] = {};      // registers per thread, per (TT, W)
 };
 constexpr int kMaxDevices = 64;
 DeviceCache g_cache[kMaxDevices];
@@ -508,7 +511,10 @@ int sm_count_gemv(int dev)
     return sms;
 }
 
-constexpr int tt_slot(int tt) { return tt == 1 ? 0 : (tt == 2 ? 1 : (tt == 4 ? 2 : 3)); }
+constexpr int tt_slot(int tt, int w)
+{
+    return 2 * (tt == 1 ? 0 : (tt == 2 ? 1 : (tt == 4 ? 2 : 3))) + (w == kWarps ? 0 : 1);
+}
 
 int align16(int v) { return (v + 15) & ~15; }
 
@@ -516,54 +522,52 @@ int align16(int v) { return (v + 15) & ~15; }
 // units per warp, then the warps' mbarriers.
 int act_bytes(int tt, int k) { return align16(align16(tt * align16(k) + tt * (k / 128) * 4) + tt * (k / 32) * 2); }
 
-void make_plan(Params& P, int tt, int kmax, int d)
+void make_plan(Params& P, int tt, int kmax, int d, int w)
 {
     P.stages = d;
     P.off_stage = act_bytes(tt, kmax);
-    P.off_bar = P.off_stage + kWarps * d * kUnitBytes;
+    P.off_bar = P.off_stage + w * d * kUnitBytes;
 }
 
-int smem_bytes(const Params& P) { return P.off_bar + kWarps * P.stages * 8; }
+int smem_bytes(const Params& P, int w) { return P.off_bar + w * P.stages * 8; }
 
 // Resident CTAs per SM: 228 KB of shared memory (1 KB reserved per CTA) and 64 K registers
 // (allocated per warp in units of 256).
-int ctas_per_sm(int smem, int regs)
+int ctas_per_sm(int smem, int regs, int w)
 {
-    int occ = kSmemPerSm / (smem + kStaticSmem + 1024);
-    const int regs_cta = ((regs * 32 + 255) / 256) * 256 * kWarps;
+    int occ = kSmemPerSm / (smem + static_smem(w) + 1024);
+    const int regs_cta = ((regs * 32 + 255) / 256) * 256 * w;
     if (65536 / regs_cta < occ) occ = 65536 / regs_cta;
     return occ;
 }
 
-template <int TT>
+template <int TT, int W>
 int kernel_regs(int dev)
 {
-    std::atomic<int>& cached = g_cache[dev].regs[tt_slot(TT)];
+    std::atomic<int>& cached = g_cache[dev].regs[tt_slot(TT, W)];
     int regs = cached.load(std::memory_order_relaxed);
     if (regs == 0) {
         cudaFuncAttributes fa{};
         regs = 64;
-        if (cudaFuncGetAttributes(&fa, gemv_q4_0_q8_k128_kernel<TT>) == cudaSuccess && fa.numRegs > 0)
+        if (cudaFuncGetAttributes(&fa, gemv_q4_0_q8_k128_kernel<TT, W>) == cudaSuccess && fa.numRegs > 0)
             regs = fa.numRegs;
         cached.store(regs, std::memory_order_relaxed);
     }
     return regs;
 }
 
-// Chooses D in 2..4: the most units in flight per SM among the layouts that fit, and at
-// equal flight the layout with more resident warps (measured on B200: 32 warps x 2 units
-// beat 16 warps x 4 units, the per-unit arithmetic needing the extra warps to hide its
-// latency).
-template <int TT>
-bool plan_tt(Params& P, int kmax, int dev, int& ctas)
+// Chooses D in 2..4 for CTAs of w warps: the most units in flight per SM among the layouts
+// that fit, and at equal flight the layout with more resident warps (measured on B200: 32
+// warps x 2 units beat 16 warps x 4 units, the per-unit arithmetic needing the extra warps to
+// hide its latency).  Returns the flight (0: nothing fits).
+int plan_w(Params& P, int tt, int kmax, int regs, int w, int& ctas)
 {
-    const int regs = kernel_regs<TT>(dev);
     int best_d = 0, best_flight = 0, best_ctas = 0;
     for (int d = 2; d <= 4; ++d) {
-        make_plan(P, TT, kmax, d);
-        const int smem = smem_bytes(P);
-        if (smem > kSmemMax) break;
-        const int c = ctas_per_sm(smem, regs);
+        make_plan(P, tt, kmax, d, w);
+        const int smem = smem_bytes(P, w);
+        if (smem > kSmemCta - static_smem(w)) break;
+        const int c = ctas_per_sm(smem, regs, w);
         if (c < 1) break;
         if (c * d > best_flight) {
             best_flight = c * d;
@@ -571,29 +575,77 @@ bool plan_tt(Params& P, int kmax, int dev, int& ctas)
             best_ctas = c;
         }
     }
-    if (best_d == 0) return false;
-    make_plan(P, TT, kmax, best_d);
+    if (best_d == 0) return 0;
+    make_plan(P, tt, kmax, best_d, w);
     ctas = best_ctas;
+    return best_flight * w;
+}
+
+// The launch plan of a token tile: CTAs of 16 warps; at one token, when the activations
+// leave room for only one such CTA per SM (very wide rows), CTAs of 32 warps sharing one
+// activation copy if they keep as many units in flight (twice the warps to hide the
+// per-unit arithmetic).
+template <int TT>
+bool plan_tt(Params& P, int kmax, int dev, int& ctas, int& warps)
+{
+    int c16 = 0;
+    const int f16 = plan_w(P, TT, kmax, kernel_regs<TT, kWarps>(dev), kWarps, c16);
+    if constexpr (TT == 1) {
+        if (IQQ_GEMV_WIDE && (f16 == 0 || c16 == 1)) {
+            Params Q = P;
+            int c32 = 0;
+            const int f32 = plan_w(Q, TT, kmax, kernel_regs<TT, kWarpsWide>(dev), kWarpsWide, c32);
+            if (f32 > 0 && f32 >= f16) {
+                P = Q;
+                ctas = c32;
+                warps = kWarpsWide;
+                return true;
+            }
+        }
+    }
+    if (f16 == 0) return false;
+    ctas = c16;
+    warps = kWarps;
     return true;
 }
 
 // Launches P.count (<= kMaxBatch) problems: c0 byte shares, one wave of CTAs (fewer when the
 // problems have fewer than 16 rows per CTA) splitting the problems' weight bytes evenly, each
 // share times the token tiles, on a one-dimensional grid.
+template <int TT, int W>
+iqq_status opt_in_smem(int dev, int smem)
+{
+    std::atomic<int>& opted = g_cache[dev].smem_set[tt_slot(TT, W)];
+    if (opted.load(std::memory_order_relaxed) < smem) {
+        const int cap = kSmemCta - static_smem(W);
+        if (cudaFuncSetAttribute(gemv_q4_0_q8_k128_kernel<TT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, cap) !=
+            cudaSuccess)
+            return iqq::launch_status();
+        opted.store(cap, std::memory_order_relaxed);
+    }
+    return IQQ_OK;
+}
+
 template <int TT>
 iqq_status launch_tt(Params& P, int kmax, int64_t max_tok, cudaStream_t st, bool& fits)
 {
     const int dev = current_device();
-    int ctas = 0;
-    fits = plan_tt<TT>(P, kmax, dev, ctas);
+    int ctas = 0, warps = kWarps;
+    fits = plan_tt<TT>(P, kmax, dev, ctas, warps);
     if (!fits) return IQQ_OK;
-    const int smem = smem_bytes(P);
-    auto kern = gemv_q4_0_q8_k128_kernel<TT>;
-    std::atomic<int>& opted = g_cache[dev].smem_set[tt_slot(TT)];
-    if (opted.load(std::memory_order_relaxed) < smem) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
-            return iqq::launch_status();
-        opted.store(kSmemMax, std::memory_order_relaxed);
+    const int smem = smem_bytes(P, warps);
+    void (*kern)(Params) = gemv_q4_0_q8_k128_kernel<TT, kWarps>;
+    if constexpr (TT == 1) {
+        if (warps == kWarpsWide) kern = gemv_q4_0_q8_k128_kernel<TT, kWarpsWide>;
+    }
+    {
+        iqq_status o = IQQ_OK;
+        if constexpr (TT == 1) {
+            o = warps == kWarpsWide ? opt_in_smem<TT, kWarpsWide>(dev, smem) : opt_in_smem<TT, kWarps>(dev, smem);
+        } else {
+            o = opt_in_smem<TT, kWarps>(dev, smem);
+        }
+        if (o != IQQ_OK) return o;
     }
     int64_t rows = 0;
     P.cum_bytes[0] = 0;
@@ -602,7 +654,7 @@ iqq_status launch_tt(Params& P, int kmax, int64_t max_tok, cudaStream_t st, bool
         rows += P.prob[i].n_out;
     }
     int64_t c0 = static_cast<int64_t>(sm_count_gemv(dev)) * ctas;
-    if (c0 > (rows + kWarps - 1) / kWarps) c0 = (rows + kWarps - 1) / kWarps;
+    if (c0 > (rows + warps - 1) / warps) c0 = (rows + warps - 1) / warps;
     if (c0 < 1) c0 = 1;
     if (c0 > 65535) c0 = 65535;  // keeps c * (B % C) below 2^32
     P.share_q = P.cum_bytes[P.count] / c0;
@@ -613,7 +665,7 @@ iqq_status launch_tt(Params& P, int kmax, int64_t max_tok, cudaStream_t st, bool
     P.tiles = static_cast<int>(gy);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(c0 * gy));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(static_cast<unsigned>(warps * 32));
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

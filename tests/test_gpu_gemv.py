@@ -71,7 +71,7 @@ def _gpu(iqq, w, a, n_out, k, n_tok):
 @pytest.mark.parametrize("n_out,k,n_tok", [
     (64, 4096, 1), (37, 11008, 3), (5, 128, 1), (9, 384, 8), (130, 4224, 5),
     (1, 256, 9), (17, 14336, 2), (3, 65536, 1), (11, 65408, 2), (200, 1024, 16),
-    (7, 4096, 4), (301, 512, 7)])
+    (7, 4096, 4), (301, 512, 7), (1000, 53248, 1), (333, 40064, 1)])
 def test_gemv_random_blocks(iqq, synth, n_out, k, n_tok):
     """Chunk tails (odd row counts, rows of 8 mod 16 bytes), one and several token tiles,
     every token-tile width, K up to the maximum."""
