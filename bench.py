@@ -735,9 +735,22 @@ def main_reference(args):
 
 def profile_case(name: str):
     """Fixed cases for ncu captures (one GPU, a few launches): gemv_11008x4096 (25 MB of
-    blocks) and gemv_16384x53248 (490 MB, the large matrix of the GEMV phase)."""
+    blocks), gemv_16384x53248 (490 MB, the large matrix of the GEMV phase) and
+    moe_experts_4 (the first 4 MoE experts' gate, up and down tensors quantized once each,
+    12 launches in expert order, 704 MB of x)."""
     import torch
     import post_weight_quantization_rowwise_b200 as iqq
+    if name == "moe_experts_4":
+        from post_weight_quantization_rowwise_b200 import synth
+        ts = synth.moe_experts(4)
+        xs = [t.weights(device="cuda") for t in ts]
+        qs = [t.qw(device="cuda") for t in ts]
+        bl = [torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8, device="cuda") for t in ts]
+        for t, x, q, b in zip(ts, xs, qs, bl):
+            iqq.iqq_quantize_q4_0_w(x, q, b)
+        torch.cuda.synchronize()
+        print("ok", " ".join(f"{t.name}:{t.rows}x{t.cols}" for t in ts))
+        return
     shapes = {"gemv_11008x4096": (11008, 4096), "gemv_16384x53248": (16384, 53248)}
     if name not in shapes:
         raise SystemExit(f"unknown profile case {name}")

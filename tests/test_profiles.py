@@ -19,7 +19,7 @@ def _commands(text):
 def _bench_flags_and_cases():
     src = open(os.path.join(ROOT, "bench.py"), encoding="utf-8").read()
     flags = set(re.findall(r'add_argument\("(--[a-z0-9-]+)"', src))
-    cases = set(re.findall(r'"(gemv_\d+x\d+)": \(', src))
+    cases = set(re.findall(r'"(gemv_\d+x\d+)": \(', src)) | set(re.findall(r'name == "([a-z0-9_]+)"', src))
     return flags, cases
 
 
