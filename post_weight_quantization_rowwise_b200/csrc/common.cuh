@@ -75,10 +75,12 @@ __device__ __forceinline__ void raise_flags(uint32_t* flags, uint32_t bits)
 }
 
 // The Q4_0 weighted quantizer with the transition-based sweep (q4_0_w.cu): rows of fewer
-// than 2^22 blocks; no epilogue outputs.
+// than 2^22 blocks; binary32 x may also take the epilogue outputs (y_out: the dequantized
+// values; acc: the round-trip accumulator), each optional.
 bool q4_0_w_fits(int64_t n_per_row);
 iqq_status launch_q4_0_w(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
-                         int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream);
+                         int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream,
+                         float* y_out = nullptr, double* acc = nullptr);
 iqq_status launch_q4_0_w(const __nv_bfloat16* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
                          int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream);
 

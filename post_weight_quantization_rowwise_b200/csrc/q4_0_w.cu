@@ -328,13 +328,22 @@ __device__ __forceinline__ void add_step(float2* dcol, int idx, float p, float w
     *c = v;
 }
 
-// One tile: blocks g .. g+31 (those below gend) of the chunk whose rows start at rA.
-template <typename XT>
+// The round trip of a lane's blocks (the epilogue variant): sum qw e^2, sum qw, sum e^2 in
+// binary64 and max |e|.
+struct RoundTrip {
+    double ew = 0.0, eq = 0.0, ee = 0.0;
+    float em = 0.0f;
+};
+
+// One tile: blocks g .. g+31 (those below gend) of the chunk whose rows start at rA.  EPI: the
+// blocks' dequantized values go to y_out (when given) and their round trip to rt (when acc).
+template <typename XT, bool EPI>
 __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
                              int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
                              int64_t g, int64_t gend, int64_t rA, int64_t nb, const float* s_sig,
                              const volatile int* s_produced, int* s_consumed_row, const float* s_c, WarpSmem& ws,
-                             volatile int* s_abort, uint32_t* __restrict__ flags)
+                             volatile int* s_abort, uint32_t* __restrict__ flags, float* __restrict__ y_out,
+                             bool acc, RoundTrip& rt)
 {
     const int lane = threadIdx.x & 31;
     uint32_t bad = 0u;
@@ -770,6 +779,14 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             if ((d16 & 0x7fffu) == 0x7c00u && isfinite(d)) bad |= IQQ_FLAG_SCALE_OVERFLOW;
         }
     }
+    if constexpr (EPI) {
+        // the round trip weighs by qw: stage the block's qw again, over its weights (the final
+        // sums were their last use), while the block is packed
+        if (acc && valid && qb != nullptr) {
+            stage_qw(my_w, qb);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+    }
     if (valid) {
         uint16_t* o16 = reinterpret_cast<uint16_t*>(out + (row * nb + b) * IQQ_Q4_0_BLOCK_BYTES);
         o16[0] = d16;
@@ -782,15 +799,51 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             const uint32_t n3 = __float_as_uint(__fadd_rn(my_l[2 * i + 17], kMagic + 8.0f)) & 15u;
             o16[1 + i] = static_cast<uint16_t>(n0 | (n2 << 4) | (n1 << 8) | (n3 << 12));
         }
+        if constexpr (EPI) {
+            // y = fp16(d) * l (the bits of the dequantization) and the round trip e = x - y in
+            // binary32, accumulated as the weighted-RMSE reduction does (qw restaged above)
+            const float dq = __half2float(__ushort_as_half(d16));
+            float4* yb = y_out != nullptr
+                             ? reinterpret_cast<float4*>(y_out + row * n_per_row + static_cast<int64_t>(b) * QK)
+                             : nullptr;
+            if (acc) staged_wait();
+#pragma unroll 1
+            for (int j4 = 0; j4 < QK; j4 += 4) {
+                const float4 lv4 = *reinterpret_cast<const float4*>(my_l + j4);
+                const float yk[4] = {__fmul_rn(dq, lv4.x), __fmul_rn(dq, lv4.y), __fmul_rn(dq, lv4.z),
+                                     __fmul_rn(dq, lv4.w)};
+                if (yb != nullptr) __stcs(yb + j4 / 4, make_float4(yk[0], yk[1], yk[2], yk[3]));
+                if (acc) {
+                    const float4 xv4 = *reinterpret_cast<const float4*>(my_x + 32 * j4);
+                    const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+                    const float4 qv = qb != nullptr ? *reinterpret_cast<const float4*>(my_w + 32 * j4)
+                                                    : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+                    const float qk[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float e = __fsub_rn(xq[k], yk[k]);
+                        const double ed = static_cast<double>(e);
+                        const double e2 = ed * ed;  // exact
+                        rt.ew = fma(static_cast<double>(qk[k]), e2, rt.ew);
+                        rt.eq += static_cast<double>(qk[k]);
+                        rt.ee += e2;
+                        rt.em = fmaxf(rt.em, fabsf(e));
+                    }
+                }
+            }
+        }
     }
     iqq::raise_flags(flags, bad);
     __syncwarp();  // the warp's shared memory is rewritten by the next tile
 }
 
-template <typename XT>
+// EPI: also the dequantized values (y_out, optional) and the round-trip accumulator (acc,
+// optional): per lane across its tiles, then one set of atomics per CTA.
+template <typename XT, bool EPI>
 __global__ void __maxnreg__(96)  // one CTA of 608 threads per SM (at most 5 warps of an SMSP's 16K registers)
 q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out, int64_t nrows,
-              int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* __restrict__ flags)
+              int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* __restrict__ flags,
+              float* __restrict__ y_out, double* __restrict__ acc)
 {
     extern __shared__ float4 smem4[];
     WarpSmem* const wsm = reinterpret_cast<WarpSmem*>(smem4);
@@ -814,6 +867,7 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
     asm volatile("griddepcontrol.wait;" ::: "memory");
     int64_t g = t0 * 32;
     const int64_t gend = t1 * 32 < total ? t1 * 32 : total;
+    RoundTrip rt;
     while (g < gend) {
         // a chunk of whole tiles touching at most kMaxRows rows
         const int64_t rA = g / nb;
@@ -843,32 +897,68 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
                 t = __shfl_sync(kFull, t, 0);
                 const int64_t gt = g + static_cast<int64_t>(t) * 32;
                 if (gt >= gB || *reinterpret_cast<volatile int*>(&s_abort) != 0) break;
-                consume_tile<XT>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, gt, gB, rA, nb,
-                                 s_sig, &s_produced, &s_consumed_row, s_c, ws, &s_abort, flags);
+                consume_tile<XT, EPI>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, gt, gB, rA,
+                                      nb, s_sig, &s_produced, &s_consumed_row, s_c, ws, &s_abort, flags, y_out,
+                                      acc != nullptr, rt);
             }
         }
         g = gB;
     }
+    if constexpr (EPI) {
+        if (acc != nullptr) {  // uniform: warp sums, then the CTA's, then one atomic per quantity
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                rt.ew += __shfl_xor_sync(kFull, rt.ew, o);
+                rt.eq += __shfl_xor_sync(kFull, rt.eq, o);
+                rt.ee += __shfl_xor_sync(kFull, rt.ee, o);
+                rt.em = fmaxf(rt.em, __shfl_xor_sync(kFull, rt.em, o));
+            }
+            __syncthreads();  // every warp is done with its staging area
+            double* s_red = reinterpret_cast<double*>(smem4);  // [kConsumers][4]
+            if (lane == 0 && warp < kConsumers) {
+                s_red[4 * warp + 0] = rt.ew;
+                s_red[4 * warp + 1] = rt.eq;
+                s_red[4 * warp + 2] = rt.ee;
+                s_red[4 * warp + 3] = static_cast<double>(rt.em);
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                double a = 0.0, bq = 0.0, c = 0.0, m = 0.0;
+                for (int w = 0; w < kConsumers; ++w) {
+                    a += s_red[4 * w + 0];
+                    bq += s_red[4 * w + 1];
+                    c += s_red[4 * w + 2];
+                    m = fmax(m, s_red[4 * w + 3]);
+                }
+                atomicAdd(acc + 0, a);
+                atomicAdd(acc + 1, bq);
+                atomicAdd(acc + 2, c);
+                // non-negative binary64 values order like their bit patterns
+                atomicMax(reinterpret_cast<unsigned long long*>(acc + 3),
+                          static_cast<unsigned long long>(__double_as_longlong(m)));
+            }
+        }
+    }
 }
 
-template <typename XT>
+template <typename XT, bool EPI>
 iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
-                  int weight_mode, float fudge, uint32_t* d_flags, void* stream)
+                  int weight_mode, float fudge, uint32_t* d_flags, void* stream, float* y_out, double* acc)
 {
     static thread_local int configured_device = -1;
     static thread_local int grid_cap = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return iqq::launch_status();
     if (configured_device != dev) {
-        if (cudaFuncSetAttribute(q4_0_w_kernel<XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(q4_0_w_kernel<XT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kDynSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(q4_0_w_kernel<XT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+            cudaFuncSetAttribute(q4_0_w_kernel<XT, EPI>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return iqq::launch_status();
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return iqq::launch_status();
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, q4_0_w_kernel<XT>, kThreads, kDynSmem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, q4_0_w_kernel<XT, EPI>, kThreads, kDynSmem) !=
             cudaSuccess)
             return iqq::launch_status();
         grid_cap = sms * (per_sm > 0 ? per_sm : 1);
@@ -886,8 +976,8 @@ iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_
     attr[0].val.programmaticStreamSerializationAllowed = IQQ_Q4_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, q4_0_w_kernel<XT>, x, qw, static_cast<uint8_t*>(out), nrows, n_per_row,
-                           rows_per_qw, weight_mode, fudge, d_flags) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, q4_0_w_kernel<XT, EPI>, x, qw, static_cast<uint8_t*>(out), nrows, n_per_row,
+                           rows_per_qw, weight_mode, fudge, d_flags, y_out, acc) != cudaSuccess)
         return iqq::launch_status();
     return iqq::launch_status();
 }
@@ -899,15 +989,21 @@ iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_
 bool q4_0_w_fits(int64_t n_per_row) { return n_per_row / QK < (int64_t(1) << 22); }
 
 iqq_status launch_q4_0_w(const float* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
-                         int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream)
+                         int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream,
+                         float* y_out, double* acc)
 {
-    return launch<float>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
+    if (y_out != nullptr || acc != nullptr)
+        return launch<float, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
+                                   y_out, acc);
+    return launch<float, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
+                                nullptr, nullptr);
 }
 
 iqq_status launch_q4_0_w(const __nv_bfloat16* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
                          int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream)
 {
-    return launch<__nv_bfloat16>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
+    return launch<__nv_bfloat16, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags,
+                                        stream, nullptr, nullptr);
 }
 
 }  // namespace iqq

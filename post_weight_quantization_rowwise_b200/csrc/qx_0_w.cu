@@ -51,6 +51,8 @@
 // contraction except the explicit __fmaf_rn calls.
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace {
@@ -741,10 +743,15 @@ iqq_status quantize_qx(int bits, const XT* x, const float* qw, void* out, int64_
     if (!iqq::aligned(x, 16) || (qw && !iqq::aligned(qw, 16)) || !iqq::aligned(out, 2) ||
         (d_flags && !iqq::aligned(d_flags, 4)))
         return IQQ_ERR_ALIGN;
-    // Q4_0 without the epilogue outputs: the transition-based sweep (q4_0_w.cu), which
-    // computes each row's sigma2 itself and needs no workspace
-    if (bits == 4 && !direct && acc == nullptr && y_out == nullptr && iqq::q4_0_w_fits(n_per_row))
-        return iqq::launch_q4_0_w(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
+    // Q4_0: the transition-based sweep (q4_0_w.cu), which computes each row's sigma2 itself
+    // and needs no workspace; binary32 x with or without the epilogue outputs, bf16 x without
+    if (bits == 4 && !direct && iqq::q4_0_w_fits(n_per_row)) {
+        if constexpr (std::is_same<XT, float>::value)
+            return iqq::launch_q4_0_w(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
+                                      y_out, acc);
+        else if (acc == nullptr && y_out == nullptr)
+            return iqq::launch_q4_0_w(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream);
+    }
     const float* rs = nullptr;
     if (workspace != nullptr && workspace_bytes_for(nrows, n_per_row) > 0) {
         float* ws = static_cast<float*>(workspace);

@@ -140,3 +140,30 @@ def test_expert_tensor_against_oracle(iqq, synth, which):
     o, _ = oracle.quantize_q4_0_w(xs, qw.numpy())
     stats = compare_q4_0(xs, qw.numpy(), blocks.reshape(t.rows, -1)[rows], o, rows=None)
     assert stats["blocks"] == len(rows) * (t.cols // 32)
+
+
+@pytest.mark.parametrize("rows,n,rpq,with_y", [(4096, 4096, 0, True), (2048, 7168, 0, True), (333, 1056, 0, True),
+                                               (129, 64, 10, False), (3, 53248, 1, True)])
+def test_epilogue_variant(iqq, synth, rows, n, rpq, with_y):
+    """The quantizer with its epilogue (iqq_quantize_qx_0_w_ex with y and acc): the blocks are
+    those of the plain entry point byte for byte, y is the dequantization kernel's bit for bit,
+    and the round-trip sums are the weighted-RMSE kernel's up to the order of the binary64
+    additions (max |e| exact)."""
+    x = synth.weight_matrix(rows, n, seed=rows + n, bf16=True, device="cuda")
+    nq = 1 if rpq == 0 else (rows + rpq - 1) // rpq
+    qw = torch.stack([synth.imatrix(n, seed=n + i, boost_frac=0.05, device="cuda") for i in range(nq)])
+    qw = qw if rpq else qw[0]
+    out = torch.empty(iqq.q4_0_nbytes(rows, n), dtype=torch.uint8, device="cuda")
+    acc = torch.zeros(4, dtype=torch.float64, device="cuda")
+    y = torch.empty_like(x) if with_y else None
+    iqq.iqq_quantize_qx_0_w_ex(4, x, qw, out, None, acc, rpq, y=y)
+    plain = torch.empty_like(out)
+    iqq.iqq_quantize_q4_0_w(x, qw, plain, rpq)
+    ref = torch.zeros(4, dtype=torch.float64, device="cuda")
+    iqq.iqq_weighted_rmse(x, plain, qw, ref, rpq)
+    torch.cuda.synchronize()
+    assert torch.equal(out, plain)
+    if with_y:
+        assert torch.equal(y, iqq.dequant_q4_0(out, rows, n))
+    a, r = acc.cpu().numpy(), ref.cpu().numpy()
+    assert np.allclose(a[:3], r[:3], rtol=1e-10, atol=0) and a[3] == r[3]
