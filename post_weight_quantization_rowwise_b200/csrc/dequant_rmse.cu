@@ -62,6 +62,9 @@ __device__ __forceinline__ float code_value(uint32_t nib4, int k)
 #ifndef IQQ_RMSE_CTAS
 #define IQQ_RMSE_CTAS 4    // CTAs per SM in the grid (weighted RMSE; measured best of 4-32 with 1-8 rows in flight)
 #endif
+#ifndef IQQ_RMSE_PDL
+#define IQQ_RMSE_PDL 1     // programmatic dependent launch between consecutive launches
+#endif
 #ifndef IQQ_RMSE_MIN_ROWS
 #define IQQ_RMSE_MIN_ROWS 8  // rows per CTA at least (weighted RMSE)
 #endif
@@ -208,6 +211,11 @@ weighted_rmse_kernel(const XT* __restrict__ x, const uint8_t* __restrict__ block
     const int64_t cq = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
     const int64_t r1 = min(nrows, r0 + rows_per_cta);
+    // Programmatic dependent launch: the next kernel of the stream may be scheduled as this
+    // grid's CTAs retire; this grid waits for its predecessor (the blocks' writer, typically)
+    // before its first global access.  (No-ops without the launch attribute.)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     double sw = 0.0, sq = 0.0, se = 0.0;
     float emax = 0.0f;
@@ -350,10 +358,18 @@ iqq_status rmse_launch(const XT* x, const void* blocks, const float* qw, int64_t
     if (rpc < IQQ_RMSE_MIN_ROWS) rpc = IQQ_RMSE_MIN_ROWS;
     gy = (nrows + rpc - 1) / rpc;
     if (gx > 0x7fffffff || gy > 65535) return IQQ_ERR_SHAPE;
-    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-    weighted_rmse_kernel<BITS, XT><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        x, static_cast<const uint8_t*>(blocks), qw, nrows, n_per_row, rows_per_qw,
-        static_cast<int>(rpc), d_acc, y);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = IQQ_RMSE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, weighted_rmse_kernel<BITS, XT>, x, static_cast<const uint8_t*>(blocks), qw, nrows,
+                           n_per_row, rows_per_qw, static_cast<int>(rpc), d_acc, y) != cudaSuccess)
+        return iqq::launch_status();
     return iqq::launch_status();
 }
 
