@@ -29,9 +29,9 @@
 //     candidate to the boundary (exact ties included) is settled by evaluating
 //     the code there exactly.  Each step adds |w*xs| and w*(2m+1) to per-candidate
 //     difference sums.
-//  3. Filter.  Prefix sums of the differences give every candidate's sums with a
-//     relative error below (max(32, steps) + 18)*2^-24; the exact sequential sums
-//     are within 32*2^-24 of the same real values.  A candidate whose approximate
+//  3. Filter.  Prefix sums of the differences give candidate k's sums with a
+//     relative error below (max(10, steps) + 1 + k)*2^-24; the exact sequential sums
+//     are within 33*2^-24 of the same real values.  A candidate whose approximate
 //     score lies further below the best approximate score than the two bounds
 //     allow cannot be the exact winner, and a candidate with no step has the same
 //     sums as its predecessor, so it cannot win the tie either.  The surviving
@@ -477,7 +477,10 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     const float a0 = active ? __fdiv_rn(-s_c[0], xmax) : 0.0f;
     const float a18 = active ? __fdiv_rn(-s_c[kCand - 1], xmax) : 0.0f;
     const float kR = __fmul_rn(10.0f, A);  // 80*|xmax|/nmax: the step index scale
-    float S0 = 0.0f, T0 = 0.0f, nsteps = 0.0f;
+    // candidate 0's sums in four interleaved chains (value j in chain j mod 4): a term goes
+    // through at most 8 + 2 roundings there, not 32
+    float S0k[4] = {0.0f, 0.0f, 0.0f, 0.0f}, T0k[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float nsteps = 0.0f;
     uint32_t m_unc = 0u, m_two = 0u;
     IQQ_UNROLL(IQQ_Q4_T_UNROLL)
     for (int j4 = 0; j4 < QK; j4 += 4) {
@@ -493,8 +496,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             const float l0 = rintf(__fmul_rn(a0, xs));            // |l0| <= 7: no clamp needed
             const float l18 = clamp8(rintf(__fmul_rn(a18, xs)));
             const float m0 = fabsf(l0);
-            S0 = __fmaf_rn(p, m0, S0);
-            T0 = __fmaf_rn(w, __fmul_rn(m0, m0), T0);
+            S0k[k] = __fmaf_rn(p, m0, S0k[k]);
+            T0k[k] = __fmaf_rn(w, __fmul_rn(m0, m0), T0k[k]);
             const float dm = __fsub_rn(fabsf(l18), m0);          // 0, 1 or 2 steps
             nsteps = __fadd_rn(nsteps, dm);
             // t + 0.5, t = (m0 + 0.5)*R - 71: the (real) candidate index of the first step; the
@@ -519,6 +522,8 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         m_unc |= unc4 << j4;
         m_two |= two4 << j4;
     }
+    const float S0 = __fadd_rn(__fadd_rn(S0k[0], S0k[1]), __fadd_rn(S0k[2], S0k[3]));
+    const float T0 = __fadd_rn(__fadd_rn(T0k[0], T0k[1]), __fadd_rn(T0k[2], T0k[3]));
     // The first largest element (|x| = |xmax|) always has one step, 7 -> 8, and it lies on a
     // rounding tie: at candidate 4 (c = 7.5) when fl(fl(7.5/|xmax|)*|xmax|) >= 7.5 (rint
     // rounds 7.5 to 8), else at candidate 5.  It is placed here, per block, rather than
@@ -578,19 +583,27 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
         c->x = sci;
         mx = fmaxf(mx, sci);
     }
-    // bounds: |approx - real| <= (max(32, steps) + 18) u per sum, exact sums within 32 u,
-    // 6 u for the approximate quotient, 2 u for the exact one (u = 2^-24)
+    // Bounds (u = 2^-24, sums of non-negative terms, first order): a term of candidate k's
+    // approximate sums goes through at most max(10, steps) + 1 + k roundings (candidate 0's
+    // chains 1 + 8 + 2, a difference sum's steps + 1, then k prefix additions), so its score
+    // S^2/T is within 3 (max(10, steps) + 1 + k) + 6 u of the real one (6 u: the approximate
+    // quotient); an exact score is within 2*33 + 32 + 2 = 100 u (its sequential chains and two
+    // roundings).  Candidate i cannot be the exact winner when its approximate score lies
+    // below the best approximate score (candidate m) by more than the sum of i's and m's
+    // bounds plus twice the exact one: 6 max(10, steps) + 3 i + 3 m + 6 + 12 + 200 u, with
+    // m <= 18 and 20 u of slack for the roundings of the threshold itself.
     const bool regular = active && A >= 0x1p-100f && A <= 0x1p100f && S0 >= 0x1p-50f && T0 >= 0x1p-50f &&
                          S <= 0x1p50f && T <= 0x1p50f && mx >= 0x1p-100f && mx <= 0x1p100f;
     uint32_t surv = 0u;
     {
-        const float nr = __fadd_rn(fmaxf(nsteps, 32.0f), 18.0f);
-        const float margin = __fmul_rn(__fmaf_rn(6.0f, nr, 256.0f), 0x1p-24f);  // 2*(3 nr + 6 + 98 + 24 slack) u
-        const float thr = __fmul_rn(mx, __fsub_rn(1.0f, margin));
-        if (sc0 >= thr) surv = 1u;
+        // threshold of candidate i: mx (1 - (6 max(10, steps) + 3 i + 292) u)
+        const float mu = __fmul_rn(mx, 0x1p-24f);
+        const float thr0 = __fsub_rn(mx, __fmul_rn(mu, __fmaf_rn(6.0f, fmaxf(nsteps, 10.0f), 292.0f)));
+        const float d3 = __fmul_rn(mu, 3.0f);
+        if (sc0 >= thr0) surv = 1u;
 #pragma unroll
         for (int i = 1; i < kCand; ++i)
-            if (dcol[32 * (i - 1)].x >= thr) surv |= 1u << i;
+            if (dcol[32 * (i - 1)].x >= __fmaf_rn(-d3, static_cast<float>(i), thr0)) surv |= 1u << i;
         surv &= ~dom;
     }
     // blocks outside the bounds: every candidate gets its exact sums (the direct sweep)
