@@ -48,7 +48,7 @@ FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of q4_0_w_kernel<float> from one ncu capture of the
 # current kernel (a 4096x4096 launch of the layer set: see the q4_0_w_kernel profile summary);
 # set to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = None
+Q4_0_DRAM_BYTES_PER_VALUE = 4.1199
 
 
 def peaks():
@@ -650,7 +650,7 @@ def main_ours(args):
         "config": {"workload": WORKLOAD, "layers": args.layers, "tensors": n_q4,
                    "q4_0_values": w.q4_elems, "q8_k128_values": w.q8_elems,
                    "l2": "inputs 25.9 GB >> 126 MB L2, no flush", "parallelism": f"dp{world} (a layer set per rank, no data-path collective)"},
-        "roofline": {"bound": "alu", "kernel": "q4_0_w_kernel<float>",
+        "roofline": {"bound": "alu", "kernel": "q4_0_w_kernel<float, false>",
                      "achieved": round(achieved, 3),
                      "peak": round(peak_ops, 3), "unit": "Tops/s",
                      "frac": round(achieved / peak_ops, 4),
