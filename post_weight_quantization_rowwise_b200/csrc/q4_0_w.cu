@@ -157,7 +157,9 @@ __device__ __forceinline__ float exact_score(const float* __restrict__ xr, const
 // element j.  All trial moves of a pass that precede the next accepted move see the same
 // (sumlx, suml2, score), so they are evaluated together; the lowest accepting lane is the move
 // the sequential pass accepts first.  The state then advances and the scan resumes after that
-// element: the accepted moves and every rounding are those of the sequential passes.
+// element: the accepted moves and every rounding are those of the sequential passes.  Every
+// lane's trial is evaluated each time: when the rest of a pass accepts nothing, the next
+// pass starts from element 0 in the same state, so the same ballot gives its first move.
 __device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, float* sL, unsigned pending,
                                             float sumlx, float suml2, float score, int gstart)
 {
@@ -186,7 +188,7 @@ __device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, fl
             // rejected for certain when fl(nlx^2) <= fl(fl(sc*nl2)*(1 - 2^-22)) with that bound in
             // [1e-30, 1e30]: then nlx^2/nl2 < sc exactly, and so is its rounded quotient
             const float thr = __fmul_rn(__fmul_rn(sc, nl2), 0.99999976158142089844f);
-            bool ok = lane >= start && (g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f &&
+            bool ok = (g > 0.0f || g < 0.0f) && ln >= -8.0f && ln <= 7.0f && nl2 > 0.0f &&
                       !(a2 <= thr && thr >= 1e-30f && thr <= 1e30f);
             float ns = 0.0f;
             if (ok) {
@@ -194,14 +196,15 @@ __device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, fl
                 ok = ns > sc;
             }
             const unsigned m = __ballot_sync(kFull, ok);
-            if (m == 0u) {                       // the rest of this pass accepts nothing
+            unsigned mh = start < QK ? m & (kFull << start) : 0u;  // the rest of this pass
+            if (mh == 0u) {                      // the rest of this pass accepts nothing
                 if (!changed || passes == 5) break;
-                ++passes;
+                ++passes;                        // the next pass, from element 0, same state
                 changed = false;
-                start = 0;
-                continue;
+                mh = m;
+                if (mh == 0u) break;             // it accepts nothing either
             }
-            const int j0 = __ffs(m) - 1;
+            const int j0 = __ffs(mh) - 1;
             if (lane == j0) lj = ln;
             lx = __shfl_sync(kFull, nlx, j0);
             l2 = __shfl_sync(kFull, nl2, j0);
