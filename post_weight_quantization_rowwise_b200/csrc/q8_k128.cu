@@ -24,7 +24,7 @@ namespace {
 #define IQQ_Q8_UNROLL 4  // 128-value blocks in flight per warp
 #endif
 #ifndef IQQ_Q8_CTAS
-#define IQQ_Q8_CTAS 8    // resident CTAs of 256 threads per SM in the grid
+#define IQQ_Q8_CTAS 16   // CTAs of 256 threads per SM in the grid (8 resident: two waves; measured best of 4-16)
 #endif
 constexpr int kThreads = 256;
 constexpr int kUnroll = IQQ_Q8_UNROLL;
