@@ -119,6 +119,33 @@ iqq_status iqq_quantize_q4_0_w_direct(const float* x, const float* qw, void* out
                                       uint32_t* d_flags, void* stream);
 
 /*
+ * iqq_quantize_q4_0_w_batch -- iqq_quantize_q4_0_w ([W] §一) for several tensors in few
+ * launches.  The pages have no counterpart: this is a launch form, not an operation.  A
+ * launch lays the 32-block tiles of up to 64 tensors end to end and spreads them evenly over
+ * one wave of CTAs, so the start and drain of a launch (about 13 us on B200, against about
+ * 230 us of work for a 4096x4096 tensor) are paid once per 64 tensors, not once per tensor.
+ * Every tensor's blocks and flags are those of iqq_quantize_q4_0_w on it, byte for byte.
+ *  problems   host array of `count` descriptions (read before the call returns): x, qw, out,
+ *             nrows, n_per_row and rows_per_qw of each tensor, as for iqq_quantize_q4_0_w
+ *             (device pointers; tensors may share qw; outputs must not overlap).
+ *  weight_mode, fudge  as for iqq_quantize_qx_0_w_ex, shared by all the tensors.
+ *  d_flags    one optional flag word for all the tensors.
+ * Errors: those of iqq_quantize_q4_0_w for any tensor, and a row of 2^22 blocks or more
+ * (IQQ_ERR_SHAPE; iqq_quantize_q4_0_w serves those), all checked before anything is
+ * enqueued; count < 0: IQQ_ERR_SHAPE; problems NULL with count > 0: IQQ_ERR_NULL.
+ */
+typedef struct iqq_q4_0_problem {
+    const float* x;
+    const float* qw;
+    void* out;
+    int64_t nrows;
+    int64_t n_per_row;
+    int64_t rows_per_qw;
+} iqq_q4_0_problem;
+iqq_status iqq_quantize_q4_0_w_batch(const iqq_q4_0_problem* problems, int64_t count, int weight_mode,
+                                     float fudge, uint32_t* d_flags, void* stream);
+
+/*
  * iqq_quantize_qx_0_w -- the same weighted search for the other 32-value formats
  * of the family ([W] §一: the weighting appears in quantize_row_q5_0_impl,
  * quantize_row_q6_0_impl, ...): bits = 4 (Q4_0, exactly iqq_quantize_q4_0_w),

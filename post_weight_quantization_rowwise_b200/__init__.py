@@ -47,6 +47,7 @@ def _load():
     sigs = {
         "iqq_quantize_q4_0_w": [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
         "iqq_quantize_q4_0_w_direct": [_vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp],
+        "iqq_quantize_q4_0_w_batch": [_vp, _i64, ctypes.c_int, ctypes.c_float, _vp, _vp],
         "iqq_quantize_q8_k128": [_vp, _vp, _i64, _i64, _vp, _vp],
         "iqq_dequant_q4_0": [_vp, _vp, _i64, _i64, _vp],
         "iqq_quantize_q8_1": [_vp, _vp, _i64, _i64, _vp, _vp, _vp],
@@ -237,6 +238,48 @@ def iqq_quantize_q4_0_w_direct(x, qw, out, rows_per_qw: int = 0, weight_mode: in
            _lib.iqq_quantize_q4_0_w_direct(_ptr(x), _ptr(qw), _ptr(out), nrows, n, rows_per_qw,
                                            weight_mode, _ptr(flags), _stream(stream)))
     return out
+
+
+class Q4_0Problem(ctypes.Structure):
+    """iqq_q4_0_problem."""
+    _fields_ = [("x", ctypes.c_void_p), ("qw", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("nrows", ctypes.c_int64), ("n_per_row", ctypes.c_int64), ("rows_per_qw", ctypes.c_int64)]
+
+
+def q4_0_problems(items):
+    """A ctypes array of iqq_q4_0_problem from (x, qw, out) or (x, qw, out, rows_per_qw) tuples
+    of CUDA tensors on one device (qw may be None), checked here; the tensors must outlive
+    every call that uses the array."""
+    import torch
+    arr = (Q4_0Problem * len(items))()
+    dev = None
+    for i, it in enumerate(items):
+        x, qw, out = it[0], it[1], it[2]
+        rpq = it[3] if len(it) > 3 else 0
+        _need_cuda("x", x, torch.float32)
+        _need_cuda("qw", qw, torch.float32)
+        _need_cuda("out", out, torch.uint8)
+        nrows, n = _shape2(x)
+        _check_qw(qw, nrows, n, rpq, x.device)
+        _same_device(x, out=out)
+        if dev is not None and x.device != dev:
+            raise ValueError(f"problem {i}: every tensor must be on the same device")
+        dev = x.device
+        if out.numel() < q4_0_nbytes(nrows, n):
+            raise ValueError(f"problem {i}: out is too small")
+        arr[i] = Q4_0Problem(x.data_ptr(), qw.data_ptr() if qw is not None else None, out.data_ptr(), nrows, n,
+                             rpq)
+    return arr
+
+
+def iqq_quantize_q4_0_w_batch(problems, weight_mode: int = 0, flags=None, stream=None, fudge: float = 1.0):
+    """iqq_quantize_q4_0_w for every tensor of a q4_0_problems() array, in launches of up to 64
+    tensors."""
+    import torch
+    _need_cuda("flags", flags, torch.int32)
+    _check("iqq_quantize_q4_0_w_batch",
+           _lib.iqq_quantize_q4_0_w_batch(ctypes.cast(problems, ctypes.c_void_p), len(problems), weight_mode,
+                                          fudge, _ptr(flags), _stream(stream)))
 
 
 QX_0_BLOCK_BYTES = {4: 18, 5: 22, 6: 26, 8: 34}

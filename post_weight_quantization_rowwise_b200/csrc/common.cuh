@@ -83,5 +83,8 @@ iqq_status launch_q4_0_w(const float* x, const float* qw, void* out, int64_t nro
                          float* y_out = nullptr, double* acc = nullptr);
 iqq_status launch_q4_0_w(const __nv_bfloat16* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
                          int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream);
+// Several binary32 tensors, validated by the caller, in launches of up to 64 tensors.
+iqq_status launch_q4_0_w_batch(const iqq_q4_0_problem* probs, int64_t count, int weight_mode, float fudge,
+                               uint32_t* d_flags, void* stream);
 
 }  // namespace iqq

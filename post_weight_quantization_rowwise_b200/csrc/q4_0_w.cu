@@ -853,12 +853,30 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     __syncwarp();  // the warp's shared memory is rewritten by the next tile
 }
 
-// EPI: also the dequantized values (y_out, optional) and the round-trip accumulator (acc,
-// optional): per lane across its tiles, then one set of atomics per CTA.
+// One tensor of a launch, and a launch: up to kMaxBatch tensors whose 32-block tiles are laid
+// end to end (a tile never spans two tensors).
+template <typename XT>
+struct Prob {
+    const XT* x;
+    const float* qw;
+    uint8_t* out;
+    int64_t nrows, n_per_row, rows_per_qw;
+};
+constexpr int kMaxBatch = 64;
+template <typename XT>
+struct Batch {
+    Prob<XT> p[kMaxBatch];
+    int64_t cum[kMaxBatch + 1];  // tiles before tensor i
+    int count;
+};
+static_assert(sizeof(Batch<float>) + 64 <= 4096, "kernel parameters");
+
+// EPI: also the dequantized values (y_out, optional; launches of one tensor) and the
+// round-trip accumulator (acc, optional): per lane across its tiles, then one set of atomics
+// per CTA.
 template <typename XT, bool EPI>
 __global__ void __maxnreg__(96)  // one CTA of 608 threads per SM (at most 5 warps of an SMSP's 16K registers)
-q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out, int64_t nrows,
-              int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* __restrict__ flags,
+q4_0_w_kernel(const __grid_constant__ Batch<XT> B, int weight_mode, float fudge, uint32_t* __restrict__ flags,
               float* __restrict__ y_out, double* __restrict__ acc)
 {
     extern __shared__ float4 smem4[];
@@ -867,10 +885,8 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
     __shared__ float s_c[kCand];
     __shared__ int s_produced, s_next, s_consumed_row, s_abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t nb = n_per_row / QK;
-    const int64_t total = nrows * nb;
-    const int64_t tiles = (total + 31) / 32;
-    // this CTA's tiles: an equal share (+-1) of the tensor's
+    const int64_t tiles = B.cum[B.count];
+    // this CTA's tiles: an equal share (+-1) of the launch's
     const int64_t per = tiles / gridDim.x, extra = tiles % gridDim.x;
     const int64_t t0 = blockIdx.x * per + min(static_cast<int64_t>(blockIdx.x), extra);
     const int64_t t1 = t0 + per + (static_cast<int64_t>(blockIdx.x) < extra ? 1 : 0);
@@ -881,44 +897,57 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
     // and memory before its first global access.  (No-ops without the launch attribute.)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    int64_t g = t0 * 32;
-    const int64_t gend = t1 * 32 < total ? t1 * 32 : total;
     RoundTrip rt;
-    while (g < gend) {
-        // a chunk of whole tiles touching at most kMaxRows rows
-        const int64_t rA = g / nb;
-        int64_t gB = (rA + kMaxRows) * nb / 32 * 32;
-        if (gB > gend) gB = gend;
-        const int nr = static_cast<int>((gB - 1) / nb - rA + 1);
-        // the rows of the first tiles the warps take, one row per warp, side by side; the
-        // producer continues after them
-        const int64_t need = (g - rA * nb + static_cast<int64_t>(kConsumers) * 32 + nb - 1) / nb;
-        const int head =
-            static_cast<int>(min(min(static_cast<int64_t>(nr), need), static_cast<int64_t>(kConsumers + 1)));
-        __syncthreads();  // every warp is done with the previous chunk
-        if (warp < head) row_sigma2(x + (rA + warp) * n_per_row, n_per_row, &s_sig[warp], flags);
-        if (threadIdx.x == 0) {
-            s_produced = head;
-            s_next = 0;
-            s_consumed_row = 0;
-        }
-        __syncthreads();
-        if (warp == kConsumers) {
-            produce_rows<XT>(x, n_per_row, rA, head, nr, s_sig, &s_produced, &s_consumed_row, flags);
-        } else {
-            WarpSmem& ws = wsm[warp];
-            while (true) {
-                int t = 0;
-                if (lane == 0) t = atomicAdd(&s_next, 1);
-                t = __shfl_sync(kFull, t, 0);
-                const int64_t gt = g + static_cast<int64_t>(t) * 32;
-                if (gt >= gB || *reinterpret_cast<volatile int*>(&s_abort) != 0) break;
-                consume_tile<XT, EPI>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, gt, gB, rA,
-                                      nb, s_sig, &s_produced, &s_consumed_row, s_c, ws, &s_abort, flags, y_out,
-                                      acc != nullptr, rt);
+    int pi = 0;
+    while (pi + 1 < B.count && B.cum[pi + 1] <= t0) ++pi;
+    for (; pi < B.count && B.cum[pi] < t1; ++pi) {
+        // the tensor's blocks [g, gend) in this CTA's share
+        const XT* const x = B.p[pi].x;
+        const float* const qw = B.p[pi].qw;
+        uint8_t* const out = B.p[pi].out;
+        const int64_t nrows = B.p[pi].nrows, n_per_row = B.p[pi].n_per_row, rows_per_qw = B.p[pi].rows_per_qw;
+        const int64_t nb = n_per_row / QK;
+        const int64_t total = nrows * nb;
+        int64_t g = (max(t0, B.cum[pi]) - B.cum[pi]) * 32;
+        const int64_t gl = (min(t1, B.cum[pi + 1]) - B.cum[pi]) * 32;
+        const int64_t gend = gl < total ? gl : total;
+        while (g < gend) {
+            // a chunk of whole tiles touching at most kMaxRows rows
+            const int64_t rA = g / nb;
+            int64_t gB = (rA + kMaxRows) * nb / 32 * 32;
+            if (gB > gend) gB = gend;
+            const int nr = static_cast<int>((gB - 1) / nb - rA + 1);
+            // the rows of the first tiles the warps take, one row per warp, side by side; the
+            // producer continues after them
+            const int64_t need = (g - rA * nb + static_cast<int64_t>(kConsumers) * 32 + nb - 1) / nb;
+            const int head =
+                static_cast<int>(min(min(static_cast<int64_t>(nr), need), static_cast<int64_t>(kConsumers + 1)));
+            __syncthreads();  // every warp is done with the previous chunk
+            if (*reinterpret_cast<volatile int*>(&s_abort) != 0) break;  // uniform: a wait ran out
+            if (warp < head) row_sigma2(x + (rA + warp) * n_per_row, n_per_row, &s_sig[warp], flags);
+            if (threadIdx.x == 0) {
+                s_produced = head;
+                s_next = 0;
+                s_consumed_row = 0;
             }
+            __syncthreads();
+            if (warp == kConsumers) {
+                produce_rows<XT>(x, n_per_row, rA, head, nr, s_sig, &s_produced, &s_consumed_row, flags);
+            } else {
+                WarpSmem& ws = wsm[warp];
+                while (true) {
+                    int t = 0;
+                    if (lane == 0) t = atomicAdd(&s_next, 1);
+                    t = __shfl_sync(kFull, t, 0);
+                    const int64_t gt = g + static_cast<int64_t>(t) * 32;
+                    if (gt >= gB || *reinterpret_cast<volatile int*>(&s_abort) != 0) break;
+                    consume_tile<XT, EPI>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, gt, gB, rA,
+                                          nb, s_sig, &s_produced, &s_consumed_row, s_c, ws, &s_abort, flags, y_out,
+                                          acc != nullptr, rt);
+                }
+            }
+            g = gB;
         }
-        g = gB;
     }
     if constexpr (EPI) {
         if (acc != nullptr) {  // uniform: warp sums, then the CTA's, then one atomic per quantity
@@ -958,8 +987,8 @@ q4_0_w_kernel(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* _
 }
 
 template <typename XT, bool EPI>
-iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
-                  int weight_mode, float fudge, uint32_t* d_flags, void* stream, float* y_out, double* acc)
+iqq_status launch(const Batch<XT>& B, int weight_mode, float fudge, uint32_t* d_flags, void* stream, float* y_out,
+                  double* acc)
 {
     static thread_local int configured_device = -1;
     static thread_local int grid_cap = 0;
@@ -980,7 +1009,8 @@ iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_
         grid_cap = sms * (per_sm > 0 ? per_sm : 1);
         configured_device = dev;
     }
-    const int64_t tiles = (nrows * (n_per_row / QK) + 31) / 32;
+    const int64_t tiles = B.cum[B.count];
+    if (tiles == 0) return IQQ_OK;
     const int grid = static_cast<int>(tiles < grid_cap ? tiles : grid_cap);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -992,10 +1022,22 @@ iqq_status launch(const XT* x, const float* qw, void* out, int64_t nrows, int64_
     attr[0].val.programmaticStreamSerializationAllowed = IQQ_Q4_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, q4_0_w_kernel<XT, EPI>, x, qw, static_cast<uint8_t*>(out), nrows, n_per_row,
-                           rows_per_qw, weight_mode, fudge, d_flags, y_out, acc) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, q4_0_w_kernel<XT, EPI>, B, weight_mode, fudge, d_flags, y_out, acc) != cudaSuccess)
         return iqq::launch_status();
     return iqq::launch_status();
+}
+
+// A launch of one tensor.
+template <typename XT, bool EPI>
+iqq_status launch_one(const XT* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row, int64_t rows_per_qw,
+                      int weight_mode, float fudge, uint32_t* d_flags, void* stream, float* y_out, double* acc)
+{
+    Batch<XT> B;
+    B.count = 1;
+    B.p[0] = Prob<XT>{x, qw, static_cast<uint8_t*>(out), nrows, n_per_row, rows_per_qw};
+    B.cum[0] = 0;
+    B.cum[1] = (nrows * (n_per_row / QK) + 31) / 32;
+    return launch<XT, EPI>(B, weight_mode, fudge, d_flags, stream, y_out, acc);
 }
 
 }  // namespace
@@ -1009,17 +1051,40 @@ iqq_status launch_q4_0_w(const float* x, const float* qw, void* out, int64_t nro
                          float* y_out, double* acc)
 {
     if (y_out != nullptr || acc != nullptr)
-        return launch<float, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
-                                   y_out, acc);
-    return launch<float, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
-                                nullptr, nullptr);
+        return launch_one<float, true>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
+                                       y_out, acc);
+    return launch_one<float, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags, stream,
+                                    nullptr, nullptr);
 }
 
 iqq_status launch_q4_0_w(const __nv_bfloat16* x, const float* qw, void* out, int64_t nrows, int64_t n_per_row,
                          int64_t rows_per_qw, int weight_mode, float fudge, uint32_t* d_flags, void* stream)
 {
-    return launch<__nv_bfloat16, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags,
-                                        stream, nullptr, nullptr);
+    return launch_one<__nv_bfloat16, false>(x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, fudge, d_flags,
+                                            stream, nullptr, nullptr);
+}
+
+// Several binary32 tensors (validated by the caller), kMaxBatch per launch.
+iqq_status launch_q4_0_w_batch(const iqq_q4_0_problem* probs, int64_t count, int weight_mode, float fudge,
+                               uint32_t* d_flags, void* stream)
+{
+    Batch<float> B;
+    B.count = 0;
+    B.cum[0] = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        const iqq_q4_0_problem& q = probs[i];
+        const int64_t tiles = (q.nrows * (q.n_per_row / QK) + 31) / 32;
+        if (tiles == 0) continue;
+        B.p[B.count] = Prob<float>{q.x, q.qw, static_cast<uint8_t*>(q.out), q.nrows, q.n_per_row, q.rows_per_qw};
+        B.cum[B.count + 1] = B.cum[B.count] + tiles;
+        if (++B.count == kMaxBatch) {
+            const iqq_status st = launch<float, false>(B, weight_mode, fudge, d_flags, stream, nullptr, nullptr);
+            if (st != IQQ_OK) return st;
+            B.count = 0;
+        }
+    }
+    if (B.count == 0) return IQQ_OK;
+    return launch<float, false>(B, weight_mode, fudge, d_flags, stream, nullptr, nullptr);
 }
 
 }  // namespace iqq

@@ -779,6 +779,27 @@ extern "C" iqq_status iqq_quantize_q4_0_w(const float* x, const float* qw, void*
     return quantize_qx(4, x, qw, out, nrows, n_per_row, rows_per_qw, weight_mode, nullptr, d_flags, stream);
 }
 
+extern "C" iqq_status iqq_quantize_q4_0_w_batch(const iqq_q4_0_problem* problems, int64_t count, int weight_mode,
+                                                float fudge, uint32_t* d_flags, void* stream)
+{
+    if (count < 0) return IQQ_ERR_SHAPE;
+    if (count > 0 && problems == nullptr) return IQQ_ERR_NULL;
+    if (weight_mode < 0 || weight_mode > 5) return IQQ_ERR_ARG;
+    if (!(fudge >= 0.0f) || !isfinite(fudge)) return IQQ_ERR_ARG;
+    if (!iqq::aligned(d_flags, 4)) return IQQ_ERR_ALIGN;
+    for (int64_t i = 0; i < count; ++i) {
+        const iqq_q4_0_problem& q = problems[i];
+        if (!iqq::size_ok(q.nrows, q.n_per_row, 4) || q.rows_per_qw < 0 || q.n_per_row % QK != 0)
+            return IQQ_ERR_SHAPE;
+        if (q.nrows == 0 || q.n_per_row == 0) continue;
+        if (!iqq::q4_0_w_fits(q.n_per_row)) return IQQ_ERR_SHAPE;
+        if (q.x == nullptr || q.out == nullptr) return IQQ_ERR_NULL;
+        if (!iqq::aligned(q.x, 16) || (q.qw && !iqq::aligned(q.qw, 16)) || !iqq::aligned(q.out, 2))
+            return IQQ_ERR_ALIGN;
+    }
+    return iqq::launch_q4_0_w_batch(problems, count, weight_mode, fudge, d_flags, stream);
+}
+
 extern "C" iqq_status iqq_quantize_q4_0_w_direct(const float* x, const float* qw, void* out, int64_t nrows,
                                                  int64_t n_per_row, int64_t rows_per_qw, int weight_mode,
                                                  uint32_t* d_flags, void* stream)

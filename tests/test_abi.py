@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
               "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
               "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch",
               "iqq_quantize_qx_0_w_ex", "iqq_dequant_rmse_qx", "iqq_quantize_qx_0_w_bf16",
-              "iqq_dequant_rmse_qx_bf16", "iqq_quantize_q4_0_w_direct"):
+              "iqq_dequant_rmse_qx_bf16", "iqq_quantize_q4_0_w_direct", "iqq_quantize_q4_0_w_batch"):
         assert n in names
 
 
@@ -128,6 +128,29 @@ def test_host_validation_without_gpu(lib):
     assert B(ctypes.cast(empty, V), 2, None, None) == 0
     unaligned = (m.GemvProblem * 1)(m.GemvProblem(8, 16, 16, 4, 128, 1))
     assert B(ctypes.cast(unaligned, V), 1, None, None) == 3
+    # the batched Q4_0 quantizer: checks of every tensor before anything is enqueued
+    QB4 = lib.iqq_quantize_q4_0_w_batch
+    QB4.argtypes = [V, ctypes.c_int64, ctypes.c_int, ctypes.c_float, V, V]
+    good = m.Q4_0Problem(16, None, 16, 2, 4096, 0)
+    arr = (m.Q4_0Problem * 3)(good, m.Q4_0Problem(16, None, 16, 2, 4097, 0), good)
+    assert QB4(ctypes.cast(arr, V), 3, 0, 1.0, None, None) == 2
+    assert QB4(None, 2, 0, 1.0, None, None) == 1
+    assert QB4(ctypes.cast(arr, V), -1, 0, 1.0, None, None) == 2
+    assert QB4(None, 0, 0, 1.0, None, None) == 0
+    one = (m.Q4_0Problem * 1)(good)
+    assert QB4(ctypes.cast(one, V), 1, 6, 1.0, None, None) == 5             # weight mode
+    assert QB4(ctypes.cast(one, V), 1, 0, float("nan"), None, None) == 5    # fudge
+    assert QB4(ctypes.cast(one, V), 1, 0, 1.0, V(2), None) == 3             # flags alignment
+    for prob, code in ((m.Q4_0Problem(8, None, 16, 2, 4096, 0), 3),         # x alignment
+                       (m.Q4_0Problem(16, 8, 16, 2, 4096, 0), 3),           # qw alignment
+                       (m.Q4_0Problem(16, None, 1, 2, 4096, 0), 3),         # out alignment
+                       (m.Q4_0Problem(None, None, 16, 2, 4096, 0), 1),
+                       (m.Q4_0Problem(16, None, None, 2, 4096, 0), 1),
+                       (m.Q4_0Problem(16, None, 16, 2, 4096, -1), 2),
+                       (m.Q4_0Problem(16, None, 16, 2, 1 << 27, 0), 2),     # 2^22 blocks a row
+                       (m.Q4_0Problem(None, None, None, 0, 4096, 0), 0)):   # empty: nothing to do
+        two = (m.Q4_0Problem * 2)(prob, prob)
+        assert QB4(ctypes.cast(two, V), 2, 0, 1.0, None, None) == code, (prob.x, prob.qw, prob.out, code)
     X = lib.iqq_quantize_qx_0_w_ex
     assert X(4, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, None, V(12), None, None) == 3   # d_acc alignment
     assert X(4, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, V(8), None, None, None) == 3    # y alignment

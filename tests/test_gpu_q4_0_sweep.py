@@ -167,3 +167,44 @@ def test_epilogue_variant(iqq, synth, rows, n, rpq, with_y):
         assert torch.equal(y, iqq.dequant_q4_0(out, rows, n))
     a, r = acc.cpu().numpy(), ref.cpu().numpy()
     assert np.allclose(a[:3], r[:3], rtol=1e-10, atol=0) and a[3] == r[3]
+
+
+def test_batched_launches_equal_single_tensor_calls(iqq, synth):
+    """iqq_quantize_q4_0_w_batch: 70 tensors of mixed shapes (more than one launch's 64; ragged
+    last tiles, one-block rows, stacked and shared imatrix rows, an empty tensor, a row with a
+    NaN) give the blocks of single-tensor calls byte for byte, and the flags of the tensors."""
+    rng = np.random.default_rng(5)
+    shapes = [(4096, 4096), (333, 1056), (129, 64), (65, 96), (3, 53248), (1, 32), (257, 32), (0, 4096)]
+    items, singles = [], []
+    shared = synth.imatrix(1056, seed=77, device="cuda")
+    for i in range(70):
+        rows, n = shapes[i % len(shapes)] if i < 16 else (int(rng.integers(1, 300)), 32 * int(rng.integers(1, 40)))
+        x = synth.weight_matrix(rows, n, seed=500 + i, bf16=(i % 2 == 0), device="cuda") if rows else \
+            torch.empty(0, n, device="cuda")
+        rpq = 0 if i % 3 else 4
+        if n == 1056 and rpq == 0:
+            qw = shared
+        elif rpq:
+            nq = max(1, (rows + rpq - 1) // rpq)
+            qw = torch.stack([synth.imatrix(n, seed=600 + i * 10 + j, device="cuda") for j in range(nq)])
+        else:
+            qw = synth.imatrix(n, seed=600 + i, boost_frac=0.05, device="cuda")
+        out = torch.empty(max(1, iqq.q4_0_nbytes(rows, n)), dtype=torch.uint8, device="cuda")
+        ref = torch.empty_like(out)
+        if rows:
+            iqq.iqq_quantize_q4_0_w(x, qw, ref, rpq)
+        items.append((x, qw, out, rpq))
+        singles.append(ref)
+    bad = items[0][0].clone()
+    bad[7, 100] = float("nan")
+    items.append((bad, items[0][1], torch.empty_like(items[0][2]), 0))
+    fb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    iqq.iqq_quantize_q4_0_w_batch(iqq.q4_0_problems(items[:-1]), flags=fb)
+    fn = torch.zeros(1, dtype=torch.int32, device="cuda")
+    iqq.iqq_quantize_q4_0_w_batch(iqq.q4_0_problems(items[-1:]), flags=fn)
+    torch.cuda.synchronize()
+    for i, ((x, _, out, _), ref) in enumerate(zip(items[:-1], singles)):
+        if x.shape[0]:
+            assert torch.equal(out, ref), i
+    assert int(fb.item()) == 0
+    assert int(fn.item()) & iqq.FLAG_NONFINITE_INPUT
