@@ -419,15 +419,17 @@ def run_moe(iqq, dev, peak_ops: float, p_mean: float, experts: int = 256):
     """DeepSeek-shaped MoE expert tensors (gate/up 2048x7168, down 7168x2048, N(0, 0.015) with
     outliers, a per-expert imatrix with 5% of the columns boosted x100), streamed expert by
     expert: each expert's three tensors are drawn on the device (not timed), then quantized
-    (Q4_0, imatrix weighted) with CUDA events around the three launches, and their round trip
-    is accumulated.  Returns Gelem/s, the ALU-model fraction, per-shape rates and the weighted
-    RMSE over all experts."""
+    (Q4_0, imatrix weighted) in one launch of the batched entry, timed with CUDA events, and
+    again in three single launches (the per-shape rates); their round trip is accumulated.
+    Returns Gelem/s and the ALU-model fraction of the batched launches, the single launches'
+    rate, per-shape rates and the weighted RMSE over all experts."""
     import torch
     from post_weight_quantization_rowwise_b200 import synth
     ts = synth.moe_experts(experts)
     acc = torch.zeros(4, dtype=torch.float64, device=dev)
     ms = {"gate": 0.0, "up": 0.0, "down": 0.0}
     vals = {"gate": 0, "up": 0, "down": 0}
+    batched_ms = 0.0
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2: the tensors start in HBM
     for e in range(experts):
@@ -435,6 +437,15 @@ def run_moe(iqq, dev, peak_ops: float, p_mean: float, experts: int = 256):
         xs = [t.weights(device=dev) for t in trio]
         qs = [t.qw(device=dev) for t in trio]
         bl = [torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8, device=dev) for t in trio]
+        # the expert's three tensors in one launch of the batched entry
+        probs = iqq.q4_0_problems(list(zip(xs, qs, bl)))
+        flush.zero_()
+        ev[0].record()
+        iqq.iqq_quantize_q4_0_w_batch(probs)
+        ev[1].record()
+        torch.cuda.synchronize()
+        batched_ms += ev[0].elapsed_time(ev[1])
+        # and one launch per tensor, for the rates of the three shapes
         flush.zero_()
         ev[0].record()
         for i, (t, x, q, b) in enumerate(zip(trio, xs, qs, bl)):
@@ -451,13 +462,15 @@ def run_moe(iqq, dev, peak_ops: float, p_mean: float, experts: int = 256):
     n = sum(vals.values())
     total_ms = sum(ms.values())
     ops = Q4_0_OPS_BASE + Q4_0_OPS_PER_PASS * p_mean
-    return {"experts": experts, "values": n, "quantize_ms": round(total_ms, 3),
-            "gelem_s": round(n / total_ms / 1e6, 3),
-            "frac": round(n * ops / (total_ms / 1e3) / 1e12 / peak_ops, 4),
+    return {"experts": experts, "values": n, "quantize_ms": round(batched_ms, 3),
+            "gelem_s": round(n / batched_ms / 1e6, 3),
+            "frac": round(n * ops / (batched_ms / 1e3) / 1e12 / peak_ops, 4),
+            "entry": "iqq_quantize_q4_0_w_batch, one launch per expert (its gate, up and down)",
+            "single_launches": {"quantize_ms": round(total_ms, 3), "gelem_s": round(n / total_ms / 1e6, 3)},
             "per_shape_gelem_s": {k: round(vals[k] / ms[k] / 1e6, 3) for k in ms},
             "wrmse": math.sqrt(a[0] / a[1]), "maxerr": a[3],
-            "timing": "CUDA events around each expert's three quantize launches; tensors drawn, then "
-                      "L2 flushed (256 MB write), between experts"}
+            "timing": "CUDA events around each expert's batched launch and around its three single "
+                      "launches; tensors drawn, then L2 flushed (256 MB write), before each"}
 
 
 def run_e2e(iqq, w: Workload, dev, steps: int, layers: int, barrier=None):
