@@ -45,10 +45,10 @@ Q8_BYTES_PER_VALUE = 4.0 + 140.0 / 128.0
 DEQ_RMSE_BYTES_PER_VALUE = 4.0 + 18.0 / 32.0 + 4.0  # read x and the blocks, write y
 B200_SMS = 148
 FP32_LANES_PER_SM = 128
-# DRAM bytes (read + write) per value of q4_0_w_kernel<float> from one ncu capture of the
-# current kernel (a 4096x4096 launch of the layer set: see the q4_0_w_kernel profile summary);
-# set to None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = None
+# DRAM bytes (read + write) per value of q4_0_w_kernel<float, false> from one ncu capture of
+# the current kernel (the batched launch of the layer set's first layer, 7 tensors: see the
+# q4_0_w_kernel profile summary); None whenever the kernel changes until it is captured again.
+Q4_0_DRAM_BYTES_PER_VALUE = 4.5323
 
 
 def peaks():
