@@ -183,7 +183,8 @@ __device__ __forceinline__ void greedy_rest(const float* sX, const float* sW, fl
             const float sg = g > 0.0f ? 1.0f : -1.0f;
             const float ln = __fadd_rn(lj, sg);
             const float nlx = __fadd_rn(lx, __fmul_rn(sg, wxj));
-            const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), l2);
+            // 2*sg*lj + 1 is a small integer: exact in one fma, as in the definition's three steps
+            const float nl2 = __fmaf_rn(wj, __fmaf_rn(g > 0.0f ? 2.0f : -2.0f, lj, 1.0f), l2);
             const float a2 = __fmul_rn(nlx, nlx);
             // rejected for certain when fl(nlx^2) <= fl(fl(sc*nl2)*(1 - 2^-22)) with that bound in
             // [1e-30, 1e30]: then nlx^2/nl2 < sc exactly, and so is its rounded quotient
@@ -747,7 +748,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             const float ln = __fadd_rn(lj, sg);
             if (!(g > 0.0f || g < 0.0f) || ln < -8.0f || ln > 7.0f) continue;
             const float nlx = __fadd_rn(sumlx, __fmul_rn(sg, __fmul_rn(wj, xj)));
-            const float nl2 = __fmaf_rn(wj, __fadd_rn(__fmul_rn(__fmul_rn(2.0f, sg), lj), 1.0f), suml2);
+            const float nl2 = __fmaf_rn(wj, __fmaf_rn(g > 0.0f ? 2.0f : -2.0f, lj, 1.0f), suml2);
             if (!(nl2 > 0.0f)) continue;
             const float ns = __fdiv_rn(__fmul_rn(nlx, nlx), nl2);
             if (ns > score) {
