@@ -645,7 +645,10 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             float r = -INFINITY;
             int kk = 0;
             if (q < total) {
-                kk = static_cast<int>(min(__fns(osurv, 0, q - ostart + 1), static_cast<unsigned>(kCand - 1)));
+                // the (q - ostart)-th survivor of the owner: drop that many lowest set bits
+                unsigned m = osurv;
+                for (int i = q - ostart; i > 0 && m != 0u; --i) m &= m - 1u;
+                kk = m != 0u ? min(__ffs(m) - 1, kCand - 1) : kCand - 1;
                 r = exact_score(ws.x + 4 * owner, ws.w + 4 * owner, __fdiv_rn(-s_c[kk], oxmax));
             }
             ws.u.res[lane] = make_float2(r, __int_as_float(kk));
