@@ -48,7 +48,7 @@ FP32_LANES_PER_SM = 128
 # DRAM bytes (read + write) per value of q4_0_w_kernel<float, false> from one ncu capture of
 # the current kernel (the batched launch of the layer set's first layer, 7 tensors: see the
 # q4_0_w_kernel profile summary); None whenever the kernel changes until it is captured again.
-Q4_0_DRAM_BYTES_PER_VALUE = None
+Q4_0_DRAM_BYTES_PER_VALUE = 4.5362
 
 
 def peaks():
