@@ -39,14 +39,16 @@
 //     warp's lanes.  Blocks outside the range where the bounds hold (tiny, huge or
 //     non-finite values, empty weights) take the direct sweep.
 //
-// Work layout: a persistent grid splits the tensor's blocks, in row-major order,
-// into equal ranges of 32-block tiles, one range per CTA.  Eighteen consumer warps
-// take tiles from a shared counter (one block per lane); one more, producer, warp
-// computes each row's sigma2 (binary64 sum of exact squares) just ahead of them,
-// which also brings the rows into L2 before the consumers load their blocks.  A
-// tile may span rows; every lane finds its own row.  Rows of any width are
-// balanced to a tile per CTA, so short rows (64 blocks) and rows that are not a
-// multiple of 32 blocks (344) leave no lanes idle.  Every wait is bounded.
+// Work layout: a launch serves up to 64 tensors, whose blocks, each tensor in row-major
+// order, are cut into 32-block tiles laid end to end; a persistent grid (one CTA per SM)
+// splits the tiles into equal ranges, one per CTA, which walks the tensors its range
+// touches.  Eighteen consumer warps take tiles from a shared counter (one block per lane);
+// one more, producer, warp computes each row's sigma2 (binary64 sum of exact squares)
+// just ahead of them, which also brings the rows into L2 before the consumers load their
+// blocks.  A tile may span rows; every lane finds its own row.  Rows of any width are
+// balanced to a tile per CTA, so short rows (64 blocks) and rows that are not a multiple
+// of 32 blocks (344) leave no lanes idle.  Every wait is bounded.  A variant of the kernel
+// (EPI) also writes each block's dequantized values and accumulates its round trip.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
