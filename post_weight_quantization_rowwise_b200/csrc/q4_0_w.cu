@@ -342,14 +342,15 @@ struct RoundTrip {
 };
 
 // One tile: blocks g .. g+31 (those below gend) of the chunk whose rows start at rA.  EPI: the
-// blocks' dequantized values go to y_out (when given) and their round trip to rt (when acc).
+// blocks' dequantized values go to y_out (when given) and their round trip to rt (when
+// want_rt).
 template <typename XT, bool EPI>
 __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__ qw, uint8_t* __restrict__ out,
                              int64_t nrows, int64_t n_per_row, int64_t rows_per_qw, int weight_mode, float fudge,
                              int64_t g, int64_t gend, int64_t rA, int64_t nb, const float* s_sig,
                              const volatile int* s_produced, int* s_consumed_row, const float* s_c, WarpSmem& ws,
                              volatile int* s_abort, uint32_t* __restrict__ flags, float* __restrict__ y_out,
-                             bool acc, RoundTrip& rt)
+                             bool want_rt, RoundTrip& rt)
 {
     const int lane = threadIdx.x & 31;
     uint32_t bad = 0u;
@@ -804,7 +805,7 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
     if constexpr (EPI) {
         // the round trip weighs by qw: stage the block's qw again, over its weights (the final
         // sums were their last use), while the block is packed
-        if (acc && valid && qb != nullptr) {
+        if (want_rt && valid && qb != nullptr) {
             stage_qw(my_w, qb);
             asm volatile("cp.async.commit_group;" ::: "memory");
         }
@@ -828,14 +829,14 @@ __device__ void consume_tile(const XT* __restrict__ x, const float* __restrict__
             float4* yb = y_out != nullptr
                              ? reinterpret_cast<float4*>(y_out + row * n_per_row + static_cast<int64_t>(b) * QK)
                              : nullptr;
-            if (acc) staged_wait();
+            if (want_rt) staged_wait();
 #pragma unroll 1
             for (int j4 = 0; j4 < QK; j4 += 4) {
                 const float4 lv4 = *reinterpret_cast<const float4*>(my_l + j4);
                 const float yk[4] = {__fmul_rn(dq, lv4.x), __fmul_rn(dq, lv4.y), __fmul_rn(dq, lv4.z),
                                      __fmul_rn(dq, lv4.w)};
                 if (yb != nullptr) __stcs(yb + j4 / 4, make_float4(yk[0], yk[1], yk[2], yk[3]));
-                if (acc) {
+                if (want_rt) {
                     const float4 xv4 = *reinterpret_cast<const float4*>(my_x + 32 * j4);
                     const float xq[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
                     const float4 qv = qb != nullptr ? *reinterpret_cast<const float4*>(my_w + 32 * j4)
