@@ -49,6 +49,8 @@ FP32_LANES_PER_SM = 128
 # the current kernel (the batched launch of the layer set's first layer, 7 tensors: see the
 # q4_0_w_kernel profile summary); None whenever the kernel changes until it is captured again.
 Q4_0_DRAM_BYTES_PER_VALUE = 4.5362
+# tensors per launch of the batched dequantization + round-trip entry
+RMSE_BATCH = 48
 
 
 def peaks():
@@ -217,43 +219,59 @@ class Workload:
             self.qw.append(g.qw(device=dev))
             self.blocks.append(torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8,
                                            device=dev))
-        maxn = max(t.numel for t in self.tensors)
-        self.y = torch.empty(maxn, dtype=torch.float32, device=dev)
+        # y of the dequantization: the tensors of one launch of the batched entry (48 a launch)
+        # write disjoint slices; successive launches reuse them (they run in stream order)
+        self.y_off, ysize = [], 0
+        for i, t in enumerate(self.tensors):
+            if i % RMSE_BATCH == 0:
+                off = 0
+            self.y_off.append(off)
+            off += -(-t.numel // 4) * 4  # 16-byte aligned slices
+            ysize = max(ysize, off)
+        self.y = torch.empty(ysize, dtype=torch.float32, device=dev)
         self.acc = torch.zeros(4, dtype=torch.float64, device=dev)
         self.act = synth.activations(4096, 7168, seed=2 + seed_off, device=dev)
         self.q8 = torch.empty(4096 * 56 * 140, dtype=torch.uint8, device=dev)
         self.q4_elems = sum(t.numel for t in self.tensors)
         self.q8_elems = self.act.numel()
         self.q4_problems = None
+        self.rmse_problems = None
 
 
 def run_step(iqq, w: Workload, stream, ev=None):
     """Enqueues one step.  ev: optional list of 4 events bracketing the 3 phases: the
     weighted Q4_0 quantization of every tensor (the batched entry: 64 tensors a launch); the
     dequantization of every tensor with its round-trip weighted error accumulated in the same
-    pass; Q8_K_128 of the activations."""
+    pass (the batched entry: 48 tensors a launch); Q8_K_128 of the activations."""
     import torch
-    if w.q4_problems is None:  # the batched entry's descriptions, built and checked once
+    if w.q4_problems is None:  # the batched entries' descriptions, built and checked once
         w.q4_problems = iqq.q4_0_problems(list(zip(w.x, w.qw, w.blocks)))
+        w.rmse_problems = iqq.dequant_rmse_problems(
+            [(x, b, qw, w.y[o:o + t.numel].view(t.rows, t.cols))
+             for t, x, qw, b, o in zip(w.tensors, w.x, w.qw, w.blocks, w.y_off)])
     if ev is not None:
         ev[0].record(stream)
     iqq.iqq_quantize_q4_0_w_batch(w.q4_problems, stream=stream)
     if ev is not None:
         ev[1].record(stream)
     w.acc.zero_()
-    for t, x, qw, b in zip(w.tensors, w.x, w.qw, w.blocks):
-        iqq.iqq_dequant_rmse_qx(4, x, b, qw, w.y[:t.numel].view(t.rows, t.cols), w.acc, stream=stream)
+    iqq.iqq_dequant_rmse_q4_0_batch(w.rmse_problems, w.acc, stream=stream)
     if ev is not None:
         ev[2].record(stream)
     iqq.iqq_quantize_q8_k128(w.act, w.q8, stream=stream)
     if ev is not None:
         ev[3].record(stream)
-    return q4_launches(w) + len(w.tensors) + 1
+    return q4_launches(w) + rmse_launches(w) + 1
 
 
 def q4_launches(w: Workload) -> int:
     """The quantization phase's launches: 64 tensors per launch of the batched entry."""
     return (len(w.tensors) + 63) // 64
+
+
+def rmse_launches(w: Workload) -> int:
+    """The dequantization phase's launches: RMSE_BATCH tensors per launch of the batched entry."""
+    return (len(w.tensors) + RMSE_BATCH - 1) // RMSE_BATCH
 
 
 def run_gemv_phase(iqq, w: Workload, dev, reps: int = 5):
@@ -685,7 +703,7 @@ def main_ours(args):
             "q4_0_w": {"ms": round(q4_ms, 4), "gelem_s": round(w.q4_elems / (q4_ms / 1e3) / 1e9, 3)},
             "dequant_rmse_q4_0": {"ms": round(phase[1] / K, 4), "gb_s": round(drm_gbs, 1),
                                   "hbm_frac": round(drm_gbs / pk["hbm_gbs"], 4),
-                                  "kernel": "weighted_rmse_kernel<4> writing y",
+                                  "kernel": "weighted_rmse_batch_kernel (48 tensors a launch) writing y",
                                   "bytes_per_value": DEQ_RMSE_BYTES_PER_VALUE,
                                   "wrmse": rt["wrmse"], "rmse": rt["rmse"], "maxerr": rt["maxerr"],
                                   "round_trip_values": rt["values"],

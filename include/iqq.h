@@ -316,6 +316,35 @@ iqq_status iqq_dequant_rmse_qx(int bits, const float* x, const void* blocks, con
                                int64_t n_per_row, int64_t rows_per_qw, float* y, double* d_acc, void* stream);
 
 /*
+ * iqq_dequant_rmse_q4_0_batch -- iqq_dequant_rmse_qx (bits 4) on up to any number of
+ * float32 tensors, 48 per launch: each tensor's CTAs are those of its own call, laid end to
+ * end on one grid, so the start and drain of a launch are paid once per 48 tensors.  Each
+ * tensor's y is bit for bit that of its own call, and all the tensors add to the one
+ * accumulator as their calls would in turn (the binary64 sums and so d_acc[0..2] can differ
+ * in the last bits with the order of the atomic adds, as between two runs of one call;
+ * d_acc[3], a maximum, is the same).
+ *  problems   host array of `count` descriptions (read before the call returns): x, blocks,
+ *             qw, y, nrows, n_per_row and rows_per_qw of each tensor, as for
+ *             iqq_dequant_rmse_qx (device pointers; tensors may share qw; the y must not
+ *             overlap one another); y NULL adds only the round trip (iqq_weighted_rmse).
+ *  d_acc      double[4] accumulator shared by all the tensors, as for iqq_weighted_rmse.
+ * Errors: those of iqq_dequant_rmse_qx for any tensor (y excepted), and a tensor of 2^31/48
+ * CTAs or more (IQQ_ERR_SHAPE), all checked before anything is enqueued; count < 0:
+ * IQQ_ERR_SHAPE; problems NULL with count > 0: IQQ_ERR_NULL.
+ */
+typedef struct iqq_dequant_rmse_problem {
+    const float* x;
+    const void* blocks;
+    const float* qw;
+    float* y;
+    int64_t nrows;
+    int64_t n_per_row;
+    int64_t rows_per_qw;
+} iqq_dequant_rmse_problem;
+iqq_status iqq_dequant_rmse_q4_0_batch(const iqq_dequant_rmse_problem* problems, int64_t count, double* d_acc,
+                                       void* stream);
+
+/*
  * iqq_dequant_rmse_qx_bf16 -- iqq_dequant_rmse_qx against x stored as bf16 [nrows,
  * n_per_row] (16-byte aligned), widened exactly to binary32: y and the accumulator are bit
  * for bit those of iqq_dequant_rmse_qx on the widened tensor.  Other arguments and errors

@@ -66,6 +66,7 @@ def _load():
         "iqq_quantize_qx_0_w_bf16": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp,
                                      ctypes.c_size_t, _vp, _vp],
         "iqq_dequant_rmse_qx_bf16": [ctypes.c_int, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
+        "iqq_dequant_rmse_q4_0_batch": [_vp, _i64, _vp, _vp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -509,6 +510,53 @@ def iqq_dequant_rmse_qx(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, strea
     return y
 
 
+class DequantRmseProblem(ctypes.Structure):
+    """iqq_dequant_rmse_problem."""
+    _fields_ = [("x", ctypes.c_void_p), ("blocks", ctypes.c_void_p), ("qw", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("nrows", ctypes.c_int64), ("n_per_row", ctypes.c_int64),
+                ("rows_per_qw", ctypes.c_int64)]
+
+
+def dequant_rmse_problems(items):
+    """A ctypes array of iqq_dequant_rmse_problem from (x, blocks, qw, y) or (x, blocks, qw, y,
+    rows_per_qw) tuples of CUDA tensors on one device (qw and y may be None), checked here; the
+    tensors must outlive every call that uses the array."""
+    import torch
+    arr = (DequantRmseProblem * len(items))()
+    dev = None
+    for i, it in enumerate(items):
+        x, blocks, qw, y = it[0], it[1], it[2], it[3]
+        rpq = it[4] if len(it) > 4 else 0
+        _need_cuda("x", x, torch.float32)
+        _need_cuda("blocks", blocks, torch.uint8)
+        _need_cuda("qw", qw, torch.float32)
+        _need_cuda("y", y, torch.float32)
+        nrows, n = _shape2(x)
+        _check_qw(qw, nrows, n, rpq, x.device)
+        _same_device(x, blocks=blocks, y=y)
+        if dev is not None and x.device != dev:
+            raise ValueError(f"problem {i}: every tensor must be on the same device")
+        dev = x.device
+        if blocks.numel() < q4_0_nbytes(nrows, n) or (y is not None and y.numel() < x.numel()):
+            raise ValueError(f"problem {i}: blocks or y is too small")
+        arr[i] = DequantRmseProblem(x.data_ptr(), blocks.data_ptr(), qw.data_ptr() if qw is not None else None,
+                                    y.data_ptr() if y is not None else None, nrows, n, rpq)
+    return arr
+
+
+def iqq_dequant_rmse_q4_0_batch(problems, acc, stream=None):
+    """iqq_dequant_rmse_qx (bits 4) for every tensor of a dequant_rmse_problems() array, in
+    launches of up to 48 tensors, all adding to acc."""
+    import torch
+    _need_cuda("acc", acc, torch.float64)
+    if acc is None or acc.numel() < 4:
+        raise ValueError("acc must hold 4 doubles")
+    _check("iqq_dequant_rmse_q4_0_batch",
+           _lib.iqq_dequant_rmse_q4_0_batch(ctypes.cast(problems, ctypes.c_void_p), len(problems), _ptr(acc),
+                                            _stream(stream)))
+    return acc
+
+
 def iqq_dequant_rmse_qx_bf16(bits, x, blocks, qw, y, acc, rows_per_qw: int = 0, stream=None):
     """iqq_dequant_rmse_qx against bf16 x (widened exactly: y and acc equal those of the
     binary32 tensor)."""
@@ -684,4 +732,4 @@ def weighted_rmse(x, blocks, qw=None, rows_per_qw: int = 0, stream=None):
 
 
 __all__ = [n for n in dir() if n.startswith(("iqq_", "quantize", "dequant", "weighted", "Q", "FLAG",
-                                             "q4", "q8", "version", "status", "IQQError", "LIB"))]
+                                             "q4", "q8", "version", "status", "IQQError", "LIB", "Dequant"))]

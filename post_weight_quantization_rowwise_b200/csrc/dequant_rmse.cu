@@ -197,25 +197,20 @@ __device__ __forceinline__ void rmse_quad(const float4 xv, const QuadC q, double
     }
 }
 
-// Rows [blockIdx.y*rows_per_cta, ...) x column quad blockIdx.x*kThreads + threadIdx.x.
+// One CTA's work: rows [by*rows_per_cta, ...) x column quad bx*kThreads + threadIdx.x.
 // Per column the thread keeps sum_r e^2 (binary64) and multiplies by qw once per
 // imatrix row, so qw is read and converted once per row segment, not per value.
 template <int BITS, typename XT>
-__global__ void __launch_bounds__(kThreads)
-weighted_rmse_kernel(const XT* __restrict__ x, const uint8_t* __restrict__ blocks,
-                     const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
-                     int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc, float* __restrict__ y)
+__device__ __forceinline__ void rmse_unit(const XT* __restrict__ x, const uint8_t* __restrict__ blocks,
+                                          const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
+                                          int64_t rows_per_qw, int rows_per_cta, int64_t bx, int64_t by,
+                                          double* __restrict__ acc, float* __restrict__ y)
 {
     const int64_t nq = n_per_row / 4;
     const int64_t nb = n_per_row / IQQ_Q4_0_BLOCK_VALUES;
-    const int64_t cq = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
+    const int64_t cq = bx * kThreads + threadIdx.x;
+    const int64_t r0 = by * rows_per_cta;
     const int64_t r1 = min(nrows, r0 + rows_per_cta);
-    // Programmatic dependent launch: the next kernel of the stream may be scheduled as this
-    // grid's CTAs retire; this grid waits for its predecessor (the blocks' writer, typically)
-    // before its first global access.  (No-ops without the launch attribute.)
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     double sw = 0.0, sq = 0.0, se = 0.0;
     float emax = 0.0f;
@@ -286,6 +281,57 @@ weighted_rmse_kernel(const XT* __restrict__ x, const uint8_t* __restrict__ block
     }
 }
 
+// Programmatic dependent launch: the next kernel of the stream may be scheduled as this
+// grid's CTAs retire; the grid waits for its predecessor (the blocks' writer, typically)
+// before its first global access.  (No-ops without the launch attribute.)
+__device__ __forceinline__ void pdl_prologue()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <int BITS, typename XT>
+__global__ void __launch_bounds__(kThreads)
+weighted_rmse_kernel(const XT* __restrict__ x, const uint8_t* __restrict__ blocks,
+                     const float* __restrict__ qw, int64_t nrows, int64_t n_per_row,
+                     int64_t rows_per_qw, int rows_per_cta, double* __restrict__ acc, float* __restrict__ y)
+{
+    pdl_prologue();
+    rmse_unit<BITS, XT>(x, blocks, qw, nrows, n_per_row, rows_per_qw, rows_per_cta, blockIdx.x, blockIdx.y, acc,
+                        y);
+}
+
+// Several Q4_0 tensors in one launch: their CTAs (column tiles x row groups, each tensor's
+// as its single launch has them) laid end to end on a one-dimensional grid.
+struct RmseProb {
+    const float* x;
+    const uint8_t* blocks;
+    const float* qw;
+    float* y;
+    int64_t nrows, n_per_row, rows_per_qw;
+    int rows_per_cta, gx;
+};
+constexpr int kRmseBatch = 48;
+struct RmseBatch {
+    RmseProb p[kRmseBatch];
+    int64_t cum[kRmseBatch + 1];  // CTAs before tensor i
+    int count;
+};
+static_assert(sizeof(RmseBatch) + 16 <= 4096, "kernel parameters");
+
+__global__ void __launch_bounds__(kThreads)
+weighted_rmse_batch_kernel(const __grid_constant__ RmseBatch B, double* __restrict__ acc)
+{
+    pdl_prologue();
+    const int64_t b = blockIdx.x;
+    int pi = 0;
+    while (pi + 1 < B.count && B.cum[pi + 1] <= b) ++pi;
+    const RmseProb& P = B.p[pi];
+    const int64_t u = b - B.cum[pi];
+    rmse_unit<4, float>(P.x, P.blocks, P.qw, P.nrows, P.n_per_row, P.rows_per_qw, P.rows_per_cta, u % P.gx,
+                        u / P.gx, acc, P.y);
+}
+
 int sm_count()
 {
     int dev = 0, sms = 148;
@@ -337,6 +383,20 @@ extern "C" iqq_status iqq_dequant_qx_0(int bits, const void* blocks, float* y, i
 
 namespace {
 
+// The weighted-RMSE grid of a tensor: gx column tiles of kThreads quads, gy row groups of rpc
+// rows (IQQ_RMSE_CTAS CTAs per SM, at least IQQ_RMSE_MIN_ROWS rows per CTA).
+void rmse_grid(int64_t nrows, int64_t n_per_row, int64_t& gx, int64_t& gy, int64_t& rpc)
+{
+    const int64_t nq = n_per_row / 4;
+    gx = (nq + kThreads - 1) / kThreads;
+    const int64_t target = static_cast<int64_t>(sm_count()) * IQQ_RMSE_CTAS;
+    gy = target / gx;
+    if (gy < 1) gy = 1;
+    rpc = (nrows + gy - 1) / gy;
+    if (rpc < IQQ_RMSE_MIN_ROWS) rpc = IQQ_RMSE_MIN_ROWS;
+    gy = (nrows + rpc - 1) / rpc;
+}
+
 template <int BITS, typename XT = float>
 iqq_status rmse_launch(const XT* x, const void* blocks, const float* qw, int64_t nrows, int64_t n_per_row,
                        int64_t rows_per_qw, double* d_acc, void* stream, float* y = nullptr)
@@ -348,15 +408,8 @@ iqq_status rmse_launch(const XT* x, const void* blocks, const float* qw, int64_t
     if (!iqq::aligned(x, 16) || !iqq::aligned(blocks, 2) || (qw && !iqq::aligned(qw, 16)) ||
         !iqq::aligned(d_acc, 8) || !iqq::aligned(y, 16))
         return IQQ_ERR_ALIGN;
-    const int64_t nq = n_per_row / 4;
-    const int64_t gx = (nq + kThreads - 1) / kThreads;
-    // IQQ_RMSE_CTAS CTAs per SM, at least IQQ_RMSE_MIN_ROWS rows per CTA
-    const int64_t target = static_cast<int64_t>(sm_count()) * IQQ_RMSE_CTAS;
-    int64_t gy = target / gx;
-    if (gy < 1) gy = 1;
-    int64_t rpc = (nrows + gy - 1) / gy;
-    if (rpc < IQQ_RMSE_MIN_ROWS) rpc = IQQ_RMSE_MIN_ROWS;
-    gy = (nrows + rpc - 1) / rpc;
+    int64_t gx = 0, gy = 0, rpc = 0;
+    rmse_grid(nrows, n_per_row, gx, gy, rpc);
     if (gx > 0x7fffffff || gy > 65535) return IQQ_ERR_SHAPE;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
@@ -422,4 +475,65 @@ extern "C" iqq_status iqq_dequant_rmse_qx_bf16(int bits, const void* x, const vo
     case 8: return rmse_launch<8>(xb, blocks, qw, nrows, n_per_row, rows_per_qw, d_acc, stream, y);
     default: return IQQ_ERR_ARG;
     }
+}
+
+namespace {
+
+iqq_status rmse_batch_launch(const RmseBatch& B, double* d_acc, void* stream)
+{
+    const int64_t ctas = B.cum[B.count];
+    if (ctas == 0) return IQQ_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = IQQ_RMSE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, weighted_rmse_batch_kernel, B, d_acc) != cudaSuccess) return iqq::launch_status();
+    return iqq::launch_status();
+}
+
+}  // namespace
+
+extern "C" iqq_status iqq_dequant_rmse_q4_0_batch(const iqq_dequant_rmse_problem* problems, int64_t count,
+                                                  double* d_acc, void* stream)
+{
+    if (count < 0) return IQQ_ERR_SHAPE;
+    if (count > 0 && problems == nullptr) return IQQ_ERR_NULL;
+    if (!iqq::aligned(d_acc, 8)) return IQQ_ERR_ALIGN;
+    for (int64_t i = 0; i < count; ++i) {
+        const iqq_dequant_rmse_problem& q = problems[i];
+        if (!iqq::size_ok(q.nrows, q.n_per_row, 4) || q.rows_per_qw < 0) return IQQ_ERR_SHAPE;
+        if (q.n_per_row % IQQ_Q4_0_BLOCK_VALUES != 0) return IQQ_ERR_SHAPE;
+        if (q.nrows == 0 || q.n_per_row == 0) continue;
+        if (q.x == nullptr || q.blocks == nullptr || d_acc == nullptr) return IQQ_ERR_NULL;
+        if (!iqq::aligned(q.x, 16) || !iqq::aligned(q.blocks, 2) || (q.qw && !iqq::aligned(q.qw, 16)) ||
+            !iqq::aligned(q.y, 16))
+            return IQQ_ERR_ALIGN;
+        int64_t gx = 0, gy = 0, rpc = 0;
+        rmse_grid(q.nrows, q.n_per_row, gx, gy, rpc);
+        if (gx * gy > 0x7fffffff / kRmseBatch || rpc > 0x7fffffff) return IQQ_ERR_SHAPE;
+    }
+    RmseBatch B;
+    B.count = 0;
+    B.cum[0] = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        const iqq_dequant_rmse_problem& q = problems[i];
+        if (q.nrows == 0 || q.n_per_row == 0) continue;
+        int64_t gx = 0, gy = 0, rpc = 0;
+        rmse_grid(q.nrows, q.n_per_row, gx, gy, rpc);
+        B.p[B.count] = RmseProb{q.x, static_cast<const uint8_t*>(q.blocks), q.qw, q.y, q.nrows, q.n_per_row,
+                                q.rows_per_qw, static_cast<int>(rpc), static_cast<int>(gx)};
+        B.cum[B.count + 1] = B.cum[B.count] + gx * gy;
+        if (++B.count == kRmseBatch) {
+            const iqq_status st = rmse_batch_launch(B, d_acc, stream);
+            if (st != IQQ_OK) return st;
+            B.count = 0;
+        }
+    }
+    if (B.count == 0) return IQQ_OK;
+    return rmse_batch_launch(B, d_acc, stream);
 }

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
               "iqq_weighted_rmse_qx", "iqq_quantize_qx_0_w_ws", "iqq_quantize_qx_0_w_workspace_bytes",
               "iqq_quantize_qx_0_w_static", "iqq_gemv_q4_0_q8_k128_batch",
               "iqq_quantize_qx_0_w_ex", "iqq_dequant_rmse_qx", "iqq_quantize_qx_0_w_bf16",
-              "iqq_dequant_rmse_qx_bf16", "iqq_quantize_q4_0_w_direct", "iqq_quantize_q4_0_w_batch"):
+              "iqq_dequant_rmse_qx_bf16", "iqq_quantize_q4_0_w_direct", "iqq_quantize_q4_0_w_batch",
+              "iqq_dequant_rmse_q4_0_batch"):
         assert n in names
 
 
@@ -151,6 +152,31 @@ def test_host_validation_without_gpu(lib):
                        (m.Q4_0Problem(None, None, None, 0, 4096, 0), 0)):   # empty: nothing to do
         two = (m.Q4_0Problem * 2)(prob, prob)
         assert QB4(ctypes.cast(two, V), 2, 0, 1.0, None, None) == code, (prob.x, prob.qw, prob.out, code)
+    # the batched dequantization + round trip: the same, with the accumulator shared
+    RB = lib.iqq_dequant_rmse_q4_0_batch
+    RB.argtypes = [V, ctypes.c_int64, V, V]
+    P = m.DequantRmseProblem
+    bad = P(16, 16, None, 16, 2, 4097, 0)
+    arr = (P * 2)(bad, P(16, 16, None, 16, 2, 4096, 0))
+    assert RB(ctypes.cast(arr, V), 2, V(16), None) == 2
+    assert RB(None, 2, V(16), None) == 1
+    assert RB(ctypes.cast(arr, V), -1, V(16), None) == 2
+    assert RB(None, 0, None, None) == 0
+    one = (P * 1)(P(16, 16, None, 16, 2, 4096, 0))
+    assert RB(ctypes.cast(one, V), 1, V(12), None) == 3                      # acc alignment
+    assert RB(ctypes.cast(one, V), 1, None, None) == 1                       # acc NULL
+    for prob, code in ((P(8, 16, None, 16, 2, 4096, 0), 3),                  # x alignment
+                       (P(16, 1, None, 16, 2, 4096, 0), 3),                  # blocks alignment
+                       (P(16, 16, 8, 16, 2, 4096, 0), 3),                    # qw alignment
+                       (P(16, 16, None, 8, 2, 4096, 0), 3),                  # y alignment
+                       (P(None, 16, None, 16, 2, 4096, 0), 1),
+                       (P(16, None, None, 16, 2, 4096, 0), 1),
+                       (P(16, 16, None, 16, 2, 4096, -1), 2),
+                       (P(16, 16, None, 16, -2, 4096, 0), 2),
+                       (P(16, 16, None, 16, 2, 4100, 0), 2),
+                       (P(None, None, None, None, 0, 4096, 0), 0)):          # empty: nothing to do
+        two = (P * 2)(prob, prob)
+        assert RB(ctypes.cast(two, V), 2, V(16), None) == code, (prob.x, prob.blocks, prob.qw, prob.y, code)
     X = lib.iqq_quantize_qx_0_w_ex
     assert X(4, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, None, V(12), None, None) == 3   # d_acc alignment
     assert X(4, V(16), None, V(16), 2, 4096, 0, 0, 1.0, None, 0, V(8), None, None, None) == 3    # y alignment

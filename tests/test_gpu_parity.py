@@ -433,6 +433,56 @@ def test_weighted_rmse(iqq, synth, rows_per_qw):
     assert np.allclose(acc[:3], ref[:3], rtol=1e-9, atol=0) and acc[1] == x.size
 
 
+def _random_q4_0_blocks(rng, nrows, n):
+    """Seeded Q4_0 block bytes: random nibbles, finite binary16 scales of either sign."""
+    raw = rng.integers(0, 256, size=(nrows * (n // 32), 18), dtype=np.uint8)
+    d16 = rng.integers(0x1000, 0x3C00, size=raw.shape[0]).astype(np.uint16)
+    d16 |= (rng.integers(0, 2, raw.shape[0]) << 15).astype(np.uint16)
+    raw[:, 0:2] = d16.view(np.uint8).reshape(-1, 2)
+    return raw.reshape(nrows, -1) if nrows else raw.reshape(0, 0)
+
+
+def test_dequant_rmse_batch(iqq, synth):
+    """The batched dequantization + round trip over 54 tensors (two launches of 48 and 6):
+    mixed widths with ragged column tiles, shared and per-row-group imatrices, no imatrix, no
+    y, an empty tensor.  Every y is bit-exact against the oracle's decoder and the per-tensor
+    call, the accumulator holds the oracle's sums over all the tensors within 1e-9 and their
+    exact max|e|."""
+    rng = np.random.default_rng(31)
+    specs = [(5, 4096, 0, True, True), (37, 4192, 0, True, True), (64, 11008, 16, True, True),
+             (3, 32, 0, False, True), (0, 4096, 0, True, True), (9, 128, 1, True, False)]
+    specs += [(2 + i % 5, 64 * (1 + i % 3), 0, i % 2 == 0, True) for i in range(48)]
+    items, ref = [], np.zeros(4, np.float64)
+    for i, (r, n, rpq, has_qw, has_y) in enumerate(specs):
+        x = synth.weight_matrix(max(r, 1), n, seed=900 + i)[:r].contiguous()
+        qrows = (r + rpq - 1) // rpq if rpq else 1
+        qw = torch.stack([synth.imatrix(n, seed=i * 11 + k) for k in range(max(qrows, 1))]) if has_qw else None
+        if qw is not None and rpq == 0:
+            qw = qw[0].contiguous()
+        b = _random_q4_0_blocks(rng, r, n)
+        oracle.weighted_rmse(x.numpy(), b, None if qw is None else qw.numpy(), rpq, acc=ref)
+        items.append((x, b, qw, rpq, has_y))
+    dev = [(x.cuda(), torch.from_numpy(b).cuda(), None if qw is None else qw.cuda(),
+            torch.full_like(x, float("nan"), device="cuda") if has_y else None, rpq)
+           for x, b, qw, rpq, has_y in items]
+    acc = torch.zeros(4, dtype=torch.float64, device="cuda")
+    iqq.iqq_dequant_rmse_q4_0_batch(iqq.dequant_rmse_problems(dev), acc)
+    torch.cuda.synchronize()
+    a = acc.cpu().numpy()
+    assert np.allclose(a[:3], ref[:3], rtol=1e-9, atol=0) and a[3] == ref[3]
+    acc1 = torch.zeros(4, dtype=torch.float64, device="cuda")
+    for (x, b, qw, y, rpq), (r, n, _, _, _) in zip(dev, specs):
+        if y is not None:
+            assert np.array_equal(y.cpu().numpy(), oracle.dequant_q4_0(b.cpu().numpy(), r, n))
+            y1 = torch.empty_like(y)
+            iqq.iqq_dequant_rmse_qx(4, x, b, qw, y1, acc1, rows_per_qw=rpq)
+            assert torch.equal(y1, y)
+        else:
+            iqq.iqq_weighted_rmse(x, b, qw, acc1, rows_per_qw=rpq)
+    a1 = acc1.cpu().numpy()
+    assert np.allclose(a[:3], a1[:3], rtol=1e-12, atol=0) and a[3] == a1[3]
+
+
 # ------------------------------------------------------------------ the C ABI's host checks
 
 def test_abi_rejects_bad_arguments(iqq):
