@@ -204,6 +204,20 @@ def oracle_sample(cores: int | None = None, pool=None):
 
 # ----------------------------------------------------------------------------- the GPU step
 
+def y_slices(numels, batch: int = RMSE_BATCH):
+    """Offsets (floats) of the tensors' dequantized outputs in one buffer, and its size: the
+    tensors of one launch of the batched entry (`batch` a launch) write disjoint 16-byte
+    aligned slices; the next launch reuses them (launches run in stream order)."""
+    offs, size, off = [], 0, 0
+    for i, n in enumerate(numels):
+        if i % batch == 0:
+            off = 0
+        offs.append(off)
+        off += -(-n // 4) * 4
+        size = max(size, off)
+    return offs, size
+
+
 class Workload:
     def __init__(self, dev, rank: int, layers: int = 32):
         import torch
@@ -219,15 +233,7 @@ class Workload:
             self.qw.append(g.qw(device=dev))
             self.blocks.append(torch.empty(t.rows * (t.cols // 32) * 18, dtype=torch.uint8,
                                            device=dev))
-        # y of the dequantization: the tensors of one launch of the batched entry (48 a launch)
-        # write disjoint slices; successive launches reuse them (they run in stream order)
-        self.y_off, ysize = [], 0
-        for i, t in enumerate(self.tensors):
-            if i % RMSE_BATCH == 0:
-                off = 0
-            self.y_off.append(off)
-            off += -(-t.numel // 4) * 4  # 16-byte aligned slices
-            ysize = max(ysize, off)
+        self.y_off, ysize = y_slices([t.numel for t in self.tensors])
         self.y = torch.empty(ysize, dtype=torch.float32, device=dev)
         self.acc = torch.zeros(4, dtype=torch.float64, device=dev)
         self.act = synth.activations(4096, 7168, seed=2 + seed_off, device=dev)

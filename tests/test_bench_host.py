@@ -66,3 +66,18 @@ def test_reference_arm_other_ranks_exit_quietly():
                        timeout=300, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_y_slices_of_a_launch_are_disjoint():
+    """The bench's dequantized outputs: within each launch of the batched entry the tensors'
+    slices are disjoint, 16-byte aligned and inside the buffer."""
+    import bench
+    from post_weight_quantization_rowwise_b200 import synth
+    numels = [t.numel for t in synth.llama2_7b_layer_set(32)] + [5, 3, 4096]
+    offs, size = bench.y_slices(numels)
+    for g in range(0, len(numels), bench.RMSE_BATCH):
+        spans = sorted((offs[i], offs[i] + numels[i]) for i in range(g, min(g + bench.RMSE_BATCH, len(numels))))
+        assert all(a % 4 == 0 and b <= size for a, b in spans)
+        assert all(spans[k][1] <= spans[k + 1][0] for k in range(len(spans) - 1))
+    assert size == max(sum(-(-n // 4) * 4 for n in numels[g:g + bench.RMSE_BATCH])
+                       for g in range(0, len(numels), bench.RMSE_BATCH))
